@@ -1,0 +1,379 @@
+"""Benchmark of one MLRA decode step on B200: KV-cache read GB/s.
+
+A step is the whole hot path on one batch: split-KV decode attention with its
+log-sum-exp combine (mlra_decode: paged gather, per-branch scores against the
+branch latent plus the shared RoPE key, per-(head, branch) softmax,
+value-absorbed output, out_scale) followed by the per-branch W_UV
+up-projection and branch sum (mlra_up_proj).
+
+value: algorithmic KV bytes of all ranks' steps / device time (GB/s), the
+KV cache resident in HBM.  L2 cannot serve the cache: each step reads the
+next of k copies of the pools, k * KV bytes >= 4x the L2 size.
+e2e: the same metric through the public Python API with the step's inputs
+(queries, block table, seqlens) copied from pinned host memory and the result
+y copied back, inside the timed region, one host synchronisation per step.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+       [--impl ours|reference]
+Under torchrun every rank runs the same workload on its own GPU (replicas,
+weak scaling); rank 0 prints one JSON line.  --impl reference times the fp64
+CPU oracle on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from branch_latent_kv_b200 import binding as b  # noqa: E402
+from branch_latent_kv_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "MLRA decode-attention KV GB/s and tokens/s at 1 B200; % of HBM roofline"
+FALLBACK_HBM_GBS = 6650.0
+
+# DRAM traffic of the decode split kernel per launch on decode_2p9b, from one
+# ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the
+# hash of the kernel sources it was taken on.  Reported as null whenever the
+# kernel sources differ from the captured ones.
+TRAFFIC_CAPTURE = {"sources_sha1": None, "bytes_per_launch": None}
+KERNEL_SOURCES = ["branch_latent_kv_b200/csrc/decode_simt.cu", "branch_latent_kv_b200/csrc/common.cuh"]
+
+
+def kernel_sources_sha1() -> str:
+    h = hashlib.sha1()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the GPU is busy."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 100):
+        self.gpu_index, self.period_ms = gpu_index, period_ms
+        self.proc, self.lines, self.thread = None, [], None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", f"-lms={self.period_ms}"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=5)
+
+    def summary(self, t0=None, t1=None):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ts, line in self.lines:
+            if t0 is not None and not (t0 <= ts <= t1):
+                continue
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def kv_bytes_of(x) -> int:
+    return x.kv_bytes
+
+
+def run_reference(args, world, rank):
+    """fp64 oracle on the host cores, each step a bounded sample."""
+    if rank != 0:
+        return
+    from oracle import oracle
+    w = WORKLOADS[args.workload]
+    threads = len(os.sched_getaffinity(0))
+    oracle.set_num_threads(threads)
+    sample_tokens = args.ref_sample_tokens
+    seqlens = torch.full((1,), sample_tokens, dtype=torch.int32)
+    ws = w.with_(batch=1, seqlen=sample_tokens, seqlen_range=None)
+    x = make_inputs(ws, seqlens=seqlens, with_w_uv=True)
+    kv = x.kv_bytes
+
+    def step():
+        out, _, _ = oracle.decode(x.q_lat, x.q_rope, x.latent_cache, x.rope_cache, x.block_table,
+                                  x.seqlens, x.scale, x.out_scale)
+        oracle.up_proj(out, x.w_uv, w.d_h)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    gbs = kv * args.steps / dt / 1e9
+    sample = (f"sequence 0 of {w.name} cut to {sample_tokens} tokens (model shape H={w.heads}, "
+              f"B={w.branches}, d_c={w.d_c}, d_r={w.d_r}), decode + up-projection per step")
+    line = {"impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w, None),
+            "tokens_per_s": 1 * args.steps / dt,
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, copies):
+    cfg = {"workload": w.name, "batch": w.batch, "heads": w.heads, "branches": w.branches,
+           "d_c": w.d_c, "d_r": w.d_r, "page_size": w.page_size, "d_h": w.d_h,
+           "seq_len": w.seqlen if w.seqlen is not None else f"U{{{w.seqlen_range[0]}..{w.seqlen_range[1]}}}",
+           "page_order": w.page_order, "parallelism": "replicas (one independent step per GPU)",
+           "step": "mlra_decode (split-KV kernel + LSE combine) + mlra_up_proj"}
+    if copies is not None:
+        cfg["l2"] = f"inputs larger than L2: {copies} rotating copies of the KV pools"
+    return cfg
+
+
+def cpu_baseline(w, x_dev, threads_hint=None):
+    """Oracle on a bounded sample (leading sequences, whole lengths)."""
+    from oracle import oracle
+    threads = len(os.sched_getaffinity(0))
+    oracle.set_num_threads(threads)
+    seqlens = x_dev.seqlens.cpu()
+    # pick leading sequences until ~1/8 of the step (at least one)
+    budget = max(int(seqlens.sum()) // 8, int(seqlens[0]))
+    ids, acc = [], 0
+    for n, L in enumerate(seqlens.tolist()):
+        if acc >= budget:
+            break
+        ids.append(n)
+        acc += L
+    host = [t.cpu() for t in (x_dev.q_lat, x_dev.q_rope, x_dev.latent_cache, x_dev.rope_cache,
+                              x_dev.block_table, x_dev.seqlens)]
+    t0 = time.perf_counter()
+    out, _, _ = oracle.decode(*host, x_dev.scale, x_dev.out_scale, seq_ids=ids)
+    dt = time.perf_counter() - t0
+    kv = acc * (w.branches * w.d_c + w.d_r) * 2
+    return {"value": kv / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{len(ids)} of {w.batch} sequences ({acc} tokens) of {w.name}, decode only, "
+                      f"{dt:.1f} s"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="decode_2p9b", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-sample-tokens", type=int, default=2048)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world, rank, local = dist_setup()
+
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+    b.library()
+    w = WORKLOADS[args.workload]
+    x = make_inputs(w, device=str(dev))
+    kv = x.kv_bytes
+    tokens = w.batch
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    copies = max(2, math.ceil(4 * l2 / kv))
+    lat = [x.latent_cache] + [x.latent_cache.clone() for _ in range(copies - 1)]
+    rope = [x.rope_cache] + [x.rope_cache.clone() for _ in range(copies - 1)]
+    dims = b.decode_dims(x.q_lat, x.q_rope, x.latent_cache, x.block_table)
+    ws = torch.zeros(b.mlra_decode_workspace_bytes(dims), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(x.q_lat)
+    y = torch.empty((w.batch, w.heads * w.d_h), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        b.mlra_decode(x.q_lat, x.q_rope, lat[i % copies], rope[i % copies], x.block_table,
+                      x.seqlens, x.scale, x.out_scale, out=out, workspace=ws)
+        if ev is not None:
+            ev[1].record(stream)
+        b.mlra_up_proj(out, x.w_uv, y=y)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    # warm-up: at least W steps and ~1.5 s of load so the clock sampler sees it
+    t_warm = time.time()
+    i = 0
+    while i < args.warmup or time.time() - t_warm < 1.5:
+        step(i)
+        i += 1
+        if i % 64 == 0:
+            torch.cuda.synchronize(dev)
+    torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_load0 = time.time()
+    start.record(stream)
+    for k in range(args.steps):
+        step(i + k, evs[k])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    t_load1 = time.time()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    elapsed_ms = start.elapsed_time(end)
+    decode_ms = sum(e0.elapsed_time(e1) for e0, e1 in evs) / args.steps
+    if pg:
+        t = torch.tensor([elapsed_ms, decode_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        elapsed_ms, decode_ms = float(t[0]), float(t[1])
+
+    # end to end through the public API, host buffers
+    h_q_lat = x.q_lat.cpu().pin_memory()
+    h_q_rope = x.q_rope.cpu().pin_memory()
+    h_bt = x.block_table.cpu().pin_memory()
+    h_sl = x.seqlens.cpu().pin_memory()
+    h_y = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    d_q_lat, d_q_rope = torch.empty_like(x.q_lat), torch.empty_like(x.q_rope)
+    d_bt, d_sl = torch.empty_like(x.block_table), torch.empty_like(x.seqlens)
+    h2d = sum(t.numel() * t.element_size() for t in (h_q_lat, h_q_rope, h_bt, h_sl))
+    d2h = h_y.numel() * h_y.element_size()
+
+    def e2e_step(i):
+        d_q_lat.copy_(h_q_lat, non_blocking=True)
+        d_q_rope.copy_(h_q_rope, non_blocking=True)
+        d_bt.copy_(h_bt, non_blocking=True)
+        d_sl.copy_(h_sl, non_blocking=True)
+        b.mlra_decode(d_q_lat, d_q_rope, lat[i % copies], rope[i % copies], d_bt, d_sl, x.scale,
+                      x.out_scale, out=out, workspace=ws)
+        b.mlra_up_proj(out, x.w_uv, y=y)
+        h_y.copy_(y, non_blocking=True)
+        stream.synchronize()
+
+    for k in range(args.warmup):
+        e2e_step(k)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for k in range(args.steps):
+        e2e_step(k)
+    e_end.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e_start.elapsed_time(e_end)
+    if pg:
+        t = torch.tensor([e2e_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    sampler.stop()
+
+    err = b.mlra_read_device_error(ws)
+    if err != 0:
+        raise RuntimeError(f"device error during the benchmark: {b.mlra_status_string(err)}")
+
+    clocks = sampler.summary(t_warm, t_load1)
+    peaks, peak_kind = measured_peaks()
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    gbs = kv * world * args.steps / (elapsed_ms / 1e3) / 1e9
+    achieved = kv / (decode_ms / 1e3) / 1e9
+    traffic = None
+    if TRAFFIC_CAPTURE["sources_sha1"] == kernel_sources_sha1():
+        traffic = TRAFFIC_CAPTURE["bytes_per_launch"]
+    line = {
+        "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w, copies),
+        "tokens_per_s": tokens * world * args.steps / (elapsed_ms / 1e3),
+        "hbm_roofline_frac": gbs / world / hbm_peak,
+        "kv_bytes_per_step": kv,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": traffic,
+                     "kernel": "mlra_decode (split-KV decode kernel + LSE combine), CUDA events "
+                               "around each call in the timed region",
+                     "peak_source": f"{peak_kind} hbm_gbs"},
+        "e2e": {"value": kv * world * args.steps / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, x)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,216 @@
+"""Python binding of the C ABI in ``include/mlra.h`` (ctypes, argument
+marshalling only).
+
+Every function here checks tensor types, shapes and devices, passes raw
+device pointers and the current CUDA stream to ``libmlra.so`` and raises
+``MlraError`` on a non-OK status.  All arithmetic happens in the library's
+CUDA kernels; there is no fallback.  If ``libmlra.so`` has not been built the
+first call raises immediately.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmlra.so")
+
+MLRA_OK = 0
+MLRA_ERR_INVALID_ARG = 1
+MLRA_ERR_UNSUPPORTED = 2
+MLRA_ERR_WORKSPACE = 3
+MLRA_ERR_CUDA = 4
+MLRA_ERR_DEVICE_BAD_INDEX = 5
+MLRA_ERR_DEVICE_BAD_SEQLEN = 6
+MLRA_ERR_DEVICE_TIMEOUT = 7
+
+
+class MlraError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {mlra_status_string(status)}")
+
+
+class mlra_dims(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_int32) for name in
+                ("batch", "heads", "branches", "d_c", "d_r", "page_size", "max_pages_per_seq",
+                 "num_pages")]
+
+
+_lib = None
+_lib_lock = threading.Lock()
+
+
+def library() -> ctypes.CDLL:
+    """Load libmlra.so (raises if it is missing: build it first)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lib_lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                                   "`python -m branch_latent_kv_b200.build`")
+            lib = ctypes.CDLL(LIB_PATH)
+            vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+            dp = ctypes.POINTER(mlra_dims)
+            lib.mlra_decode_workspace_bytes.argtypes = [dp, i32]
+            lib.mlra_decode_workspace_bytes.restype = sz
+            lib.mlra_decode.argtypes = [dp, vp, vp, vp, vp, vp, vp, ctypes.c_float, ctypes.c_float,
+                                        vp, vp, sz, vp]
+            lib.mlra_decode.restype = ctypes.c_int
+            lib.mlra_up_proj.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp]
+            lib.mlra_up_proj.restype = ctypes.c_int
+            lib.mlra_read_device_error.argtypes = [vp, vp]
+            lib.mlra_read_device_error.restype = ctypes.c_int
+            lib.mlra_status_string.argtypes = [ctypes.c_int]
+            lib.mlra_status_string.restype = ctypes.c_char_p
+            lib.mlra_decode_plan.argtypes = [i32, i32, i32, vp, i32, vp, vp]
+            lib.mlra_decode_plan.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def mlra_status_string(status: int) -> str:
+    return library().mlra_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != MLRA_OK:
+        raise MlraError(status, where)
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream], device: torch.device) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return int(s.cuda_stream)
+
+
+def _ptr(t: torch.Tensor) -> int:
+    return int(t.data_ptr())
+
+
+def _require(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int, device: torch.device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got shape {tuple(t.shape)}")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def decode_dims(q_lat, q_rope, latent_cache, block_table) -> mlra_dims:
+    N, H, B, d_c = q_lat.shape
+    num_pages, P = latent_cache.shape[:2]
+    return mlra_dims(N, H, B, d_c, q_rope.shape[2], P, block_table.shape[1], num_pages)
+
+
+def mlra_decode_workspace_bytes(dims: mlra_dims, num_ctas: int = 0) -> int:
+    n = library().mlra_decode_workspace_bytes(ctypes.byref(dims), int(num_ctas))
+    if n == 0:
+        raise MlraError(MLRA_ERR_INVALID_ARG, "mlra_decode_workspace_bytes")
+    return int(n)
+
+
+_ws_cache = {}
+
+
+def workspace_for(dims: mlra_dims, device: torch.device) -> torch.Tensor:
+    """A zeroed workspace of the required size, cached per device and grown
+    on demand.  Calls sharing it must not overlap on the GPU."""
+    need = mlra_decode_workspace_bytes(dims)
+    key = device.index if device.index is not None else torch.cuda.current_device()
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < need:
+        ws = torch.zeros(need, dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def mlra_decode(q_lat, q_rope, latent_cache, rope_cache, block_table, seqlens, scale, out_scale,
+                out=None, workspace=None, stream=None) -> torch.Tensor:
+    """MLRA decode attention (see mlra_decode in include/mlra.h).
+
+    q_lat bf16 [N,H,B,d_c], q_rope bf16 [N,H,d_r], latent_cache bf16
+    [pages,P,B,d_c], rope_cache bf16 [pages,P,d_r], block_table int32
+    [N,max_pages], seqlens int32 [N]; returns out bf16 [N,H,B,d_c].
+    """
+    dev = q_lat.device
+    if dev.type != "cuda":
+        raise ValueError("mlra_decode runs on CUDA tensors only")
+    _require(q_lat, "q_lat", torch.bfloat16, 4, dev)
+    _require(q_rope, "q_rope", torch.bfloat16, 3, dev)
+    _require(latent_cache, "latent_cache", torch.bfloat16, 4, dev)
+    _require(rope_cache, "rope_cache", torch.bfloat16, 3, dev)
+    _require(block_table, "block_table", torch.int32, 2, dev)
+    _require(seqlens, "seqlens", torch.int32, 1, dev)
+    N, H, B, d_c = q_lat.shape
+    if (tuple(q_rope.shape[:2]) != (N, H) or tuple(latent_cache.shape[2:]) != (B, d_c)
+            or tuple(rope_cache.shape) != (latent_cache.shape[0], latent_cache.shape[1], q_rope.shape[2])
+            or block_table.shape[0] != N or seqlens.shape[0] != N):
+        raise ValueError("inconsistent mlra_decode shapes")
+    dims = decode_dims(q_lat, q_rope, latent_cache, block_table)
+    if out is None:
+        out = torch.empty_like(q_lat)
+    else:
+        _require(out, "out", torch.bfloat16, 4, dev)
+        if out.shape != q_lat.shape:
+            raise ValueError("out must have the shape of q_lat")
+    if workspace is None:
+        workspace = workspace_for(dims, dev)
+    st = library().mlra_decode(ctypes.byref(dims), _ptr(q_lat), _ptr(q_rope), _ptr(latent_cache),
+                               _ptr(rope_cache), _ptr(block_table), _ptr(seqlens), float(scale),
+                               float(out_scale), _ptr(out), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(),
+                               _stream_ptr(stream, dev))
+    _check(st, "mlra_decode")
+    return out
+
+
+def mlra_up_proj(out_lat, w_uv, d_h: Optional[int] = None, y=None, stream=None) -> torch.Tensor:
+    """y bf16 [N, H*d_h] = per-branch W_UV up-projection summed over branches."""
+    dev = out_lat.device
+    if dev.type != "cuda":
+        raise ValueError("mlra_up_proj runs on CUDA tensors only")
+    _require(out_lat, "out_lat", torch.bfloat16, 4, dev)
+    _require(w_uv, "w_uv", torch.bfloat16, 3, dev)
+    N, H, B, d_c = out_lat.shape
+    if w_uv.shape[0] != B or w_uv.shape[1] != d_c or w_uv.shape[2] % H != 0:
+        raise ValueError("w_uv must be [branches, d_c, heads*d_h]")
+    if d_h is None:
+        d_h = w_uv.shape[2] // H
+    if w_uv.shape[2] != H * d_h:
+        raise ValueError("w_uv last dimension must be heads*d_h")
+    if y is None:
+        y = torch.empty((N, H * d_h), dtype=torch.bfloat16, device=dev)
+    else:
+        _require(y, "y", torch.bfloat16, 2, dev)
+    st = library().mlra_up_proj(N, H, B, d_c, d_h, _ptr(out_lat), _ptr(w_uv), _ptr(y),
+                                _stream_ptr(stream, dev))
+    _check(st, "mlra_up_proj")
+    return y
+
+
+def mlra_read_device_error(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise the stream; return and clear the device error code."""
+    return int(library().mlra_read_device_error(_ptr(workspace),
+                                                _stream_ptr(stream, workspace.device)))
+
+
+def mlra_decode_plan(seqlens: torch.Tensor, page_size: int, max_pages_per_seq: int,
+                     num_ctas: int, stream=None) -> torch.Tensor:
+    """The split-KV work partition as int32 [num_ctas*4 + N*2] (see mlra.h)."""
+    dev = seqlens.device
+    _require(seqlens, "seqlens", torch.int32, 1, dev)
+    out = torch.empty(num_ctas * 4 + seqlens.numel() * 2, dtype=torch.int32, device=dev)
+    st = library().mlra_decode_plan(seqlens.numel(), page_size, max_pages_per_seq, _ptr(seqlens),
+                                    num_ctas, _ptr(out), _stream_ptr(stream, dev))
+    _check(st, "mlra_decode_plan")
+    return out

@@ -1,0 +1,163 @@
+// api.cu -- the C ABI declared in include/mlra.h: host-side validation,
+// workspace sizing and kernel launches.  No allocation, no synchronisation
+// (except mlra_read_device_error), no exceptions across the boundary.
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+using namespace mlra;
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool is_pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1)) == 0; }
+
+// Structural validity (INVALID_ARG) then kernel coverage (UNSUPPORTED).
+mlra_status check_dims(const mlra_dims* d) {
+    if (d == nullptr) return MLRA_ERR_INVALID_ARG;
+    if (d->batch < 1 || d->heads < 1 || d->branches < 1 || d->d_c < 1 || d->d_r < 1 ||
+        d->page_size < 1 || d->max_pages_per_seq < 1 || d->num_pages < 1)
+        return MLRA_ERR_INVALID_ARG;
+    // every flat index must fit the kernels' 64-bit arithmetic and the
+    // 32-bit row coordinates of the cache tensor maps
+    if ((int64_t)d->num_pages * d->page_size > INT32_MAX) return MLRA_ERR_INVALID_ARG;
+    if ((int64_t)d->max_pages_per_seq * d->page_size > INT32_MAX) return MLRA_ERR_INVALID_ARG;
+    if ((int64_t)d->batch * d->max_pages_per_seq > INT32_MAX) return MLRA_ERR_INVALID_ARG;
+    // the plan counts 128-token tiles in int32
+    if ((int64_t)d->batch * d->max_pages_per_seq * d->page_size / kTileTokens > (int64_t(1) << 30))
+        return MLRA_ERR_INVALID_ARG;
+    if (d->heads > 16) return MLRA_ERR_UNSUPPORTED;
+    if (!is_pow2_in(d->d_c, 64, 512) || d->branches * d->d_c > 512) return MLRA_ERR_UNSUPPORTED;
+    if (d->d_r != 32 && d->d_r != 64) return MLRA_ERR_UNSUPPORTED;
+    if (!is_pow2_in(d->page_size, 16, 128)) return MLRA_ERR_UNSUPPORTED;
+    if (d->batch > 65535) return MLRA_ERR_UNSUPPORTED;  // combine grid.x limit is far above; keep a sane cap
+    return MLRA_OK;
+}
+
+int device_sm_count() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
+    if (dev < 64 && cache[dev] > 0) return cache[dev];
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    if (dev < 64) cache[dev] = sms;
+    return sms;
+}
+
+mlra_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MLRA_OK : MLRA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t mlra_decode_workspace_bytes(const mlra_dims* dims, int32_t num_ctas) {
+    if (check_dims(dims) != MLRA_OK) return 0;
+    if (num_ctas <= 0) num_ctas = device_sm_count();
+    if (num_ctas <= 0) return 0;
+    return workspace_layout(dims->batch, dims->heads, dims->branches, dims->d_c, num_ctas).total;
+}
+
+mlra_status mlra_decode(const mlra_dims* dims, const void* q_lat, const void* q_rope,
+                        const void* latent_cache, const void* rope_cache,
+                        const int32_t* block_table, const int32_t* seqlens, float scale,
+                        float out_scale, void* out, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+    const mlra_status s = check_dims(dims);
+    if (s != MLRA_OK) return s;
+    if (!aligned16(q_lat) || !aligned16(q_rope) || !aligned16(latent_cache) ||
+        !aligned16(rope_cache) || !aligned16(block_table) || !aligned16(seqlens) ||
+        !aligned16(out))
+        return MLRA_ERR_INVALID_ARG;
+    if (!(scale == scale) || !(out_scale == out_scale)) return MLRA_ERR_INVALID_ARG;  // NaN
+    if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return MLRA_ERR_WORKSPACE;
+    const int ctas = device_sm_count();
+    if (ctas <= 0) return MLRA_ERR_CUDA;
+    const WorkspaceLayout wl =
+        workspace_layout(dims->batch, dims->heads, dims->branches, dims->d_c, ctas);
+    if (workspace_bytes < wl.total) return MLRA_ERR_WORKSPACE;
+
+    DecodeArgs a;
+    a.q_lat = static_cast<const __nv_bfloat16*>(q_lat);
+    a.q_rope = static_cast<const __nv_bfloat16*>(q_rope);
+    a.latent = static_cast<const __nv_bfloat16*>(latent_cache);
+    a.rope = static_cast<const __nv_bfloat16*>(rope_cache);
+    a.block_table = block_table;
+    a.seqlens = seqlens;
+    a.out = static_cast<__nv_bfloat16*>(out);
+    char* ws = static_cast<char*>(workspace);
+    a.err = reinterpret_cast<int*>(ws + wl.err_off);
+    a.lse_part = reinterpret_cast<float*>(ws + wl.lse_off);
+    a.o_part = reinterpret_cast<float*>(ws + wl.o_off);
+    a.batch = dims->batch;
+    a.heads = dims->heads;
+    a.branches = dims->branches;
+    a.d_c = dims->d_c;
+    a.d_r = dims->d_r;
+    a.page_size = dims->page_size;
+    a.max_pages = dims->max_pages_per_seq;
+    a.num_pages = dims->num_pages;
+    a.num_ctas = ctas;
+    a.scale_log2 = scale * kLog2e;
+    a.out_scale = out_scale;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    mlra_status r = cuda_status(launch_decode_simt(a, st));
+    if (r != MLRA_OK) return r;
+    return cuda_status(launch_combine(a, st));
+}
+
+mlra_status mlra_up_proj(int32_t batch, int32_t heads, int32_t branches, int32_t d_c, int32_t d_h,
+                         const void* out_lat, const void* w_uv, void* y, void* stream) {
+    if (batch < 1 || heads < 1 || branches < 1 || d_c < 1 || d_h < 1) return MLRA_ERR_INVALID_ARG;
+    if (!aligned16(out_lat) || !aligned16(w_uv) || !aligned16(y)) return MLRA_ERR_INVALID_ARG;
+    if ((int64_t)batch * heads * d_h > INT32_MAX) return MLRA_ERR_INVALID_ARG;
+    const int K = branches * d_c;
+    if (K % 64 != 0 || K > 512 || (d_h != 64 && d_h != 128)) return MLRA_ERR_UNSUPPORTED;
+    return cuda_status(launch_up_proj(batch, heads, branches, d_c, d_h,
+                                      static_cast<const __nv_bfloat16*>(out_lat),
+                                      static_cast<const __nv_bfloat16*>(w_uv),
+                                      static_cast<__nv_bfloat16*>(y),
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+mlra_status mlra_read_device_error(void* workspace, void* stream) {
+    if (workspace == nullptr) return MLRA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MLRA_ERR_CUDA;
+    int code = 0;
+    if (cudaMemcpy(&code, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MLRA_ERR_CUDA;
+    if (code != 0 && cudaMemset(workspace, 0, sizeof(int)) != cudaSuccess) return MLRA_ERR_CUDA;
+    return static_cast<mlra_status>(code);
+}
+
+const char* mlra_status_string(mlra_status status) {
+    switch (status) {
+        case MLRA_OK: return "MLRA_OK";
+        case MLRA_ERR_INVALID_ARG: return "MLRA_ERR_INVALID_ARG: invalid argument";
+        case MLRA_ERR_UNSUPPORTED: return "MLRA_ERR_UNSUPPORTED: shape not implemented";
+        case MLRA_ERR_WORKSPACE: return "MLRA_ERR_WORKSPACE: workspace missing or too small";
+        case MLRA_ERR_CUDA: return "MLRA_ERR_CUDA: CUDA call or launch failed";
+        case MLRA_ERR_DEVICE_BAD_INDEX: return "MLRA_ERR_DEVICE_BAD_INDEX: block-table entry out of range";
+        case MLRA_ERR_DEVICE_BAD_SEQLEN: return "MLRA_ERR_DEVICE_BAD_SEQLEN: sequence length out of range";
+        case MLRA_ERR_DEVICE_TIMEOUT: return "MLRA_ERR_DEVICE_TIMEOUT: bounded wait expired in a kernel";
+    }
+    return "MLRA: unknown status";
+}
+
+mlra_status mlra_decode_plan(int32_t batch, int32_t page_size, int32_t max_pages_per_seq,
+                             const int32_t* seqlens, int32_t num_ctas, int32_t* plan_out,
+                             void* stream) {
+    if (batch < 1 || page_size < 1 || max_pages_per_seq < 1 || num_ctas < 1) return MLRA_ERR_INVALID_ARG;
+    if (!aligned16(seqlens) || !aligned16(plan_out)) return MLRA_ERR_INVALID_ARG;
+    if ((int64_t)max_pages_per_seq * page_size > INT32_MAX) return MLRA_ERR_INVALID_ARG;
+    return cuda_status(launch_plan_dump(batch, page_size, max_pages_per_seq, seqlens, num_ctas,
+                                        plan_out, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,166 @@
+/*
+ * mlra.h -- C ABI of the MLRA decode-attention library (sm_100a, one GPU).
+ *
+ * Multi-Head Low-Rank Attention keeps B independent latent branches per token
+ * (B = 4 for MLRA-4) plus one decoupled RoPE key shared by all branches and
+ * heads.  A decode step scores every query head against every branch's
+ * latent, runs an independent softmax per (head, branch), forms the
+ * value-absorbed latent output of each branch, up-projects each branch with
+ * its own W_UV and sums the branches.
+ *
+ * Sources:
+ *  - "MLRA: Breaking the Sharding Bottleneck in Latent Attention"
+ *    (wispaper.ai blog), section "The Core Insight: Sum of Branches, Not Sum
+ *    of Keys": attention on each latent block independently, outputs summed.
+ *  - same page, section "Mathematical Calibration: Scaling the Latents": a
+ *    final rescaling factor on the attention output (here `out_scale`).
+ *  - "Multi-Head Low-Rank Attention" abstract (arXiv 2603.02188, shd-paper.top
+ *    and searcharxiv pages): decoding is bound by moving the KV cache from HBM
+ *    to on-chip memory at every step.
+ *  - "TransMLA: Multi-head latent attention is all you need" (Hacker News
+ *    thread), comment quoting its section 3.3: only the latents are cached.
+ *
+ * Conventions for every entry point:
+ *  - All tensors are dense, row-major, in device memory owned by the caller,
+ *    and 16-byte aligned.  bf16 is IEEE bfloat16; results are rounded to
+ *    nearest even.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Work is enqueued asynchronously; no entry point allocates,
+ *    frees or synchronises, except mlra_read_device_error (documented below).
+ *  - Arguments are validated on the host before anything is enqueued; a
+ *    rejected call enqueues nothing.  No C++ exception crosses this ABI.
+ *  - Problems that only the device can see (a bad block-table entry or
+ *    sequence length) do not trap: the affected sequence's output is written
+ *    as zeros and the first such code is recorded in the workspace error
+ *    word, read back with mlra_read_device_error.
+ */
+#ifndef MLRA_H
+#define MLRA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MLRA_API __attribute__((visibility("default")))
+#else
+#define MLRA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MLRA_OK = 0,
+    MLRA_ERR_INVALID_ARG = 1,      /* null/misaligned pointer, bad size, inconsistent dims */
+    MLRA_ERR_UNSUPPORTED = 2,      /* valid but outside the shapes the kernels implement */
+    MLRA_ERR_WORKSPACE = 3,        /* workspace missing or smaller than required */
+    MLRA_ERR_CUDA = 4,             /* a CUDA call or kernel launch failed */
+    MLRA_ERR_DEVICE_BAD_INDEX = 5, /* device: block-table entry outside [0, num_pages) */
+    MLRA_ERR_DEVICE_BAD_SEQLEN = 6,/* device: seqlen < 1 or > max_pages_per_seq * page_size */
+    MLRA_ERR_DEVICE_TIMEOUT = 7    /* device: a bounded wait inside a kernel gave up */
+} mlra_status;
+
+/* Shape of one decode step. */
+typedef struct {
+    int32_t batch;             /* N: sequences, one new query token each            */
+    int32_t heads;             /* H: query heads                                     */
+    int32_t branches;          /* B: latent branches (4 for MLRA-4, 1 = MLA)         */
+    int32_t d_c;               /* latent width of one branch                         */
+    int32_t d_r;               /* width of the shared decoupled RoPE key             */
+    int32_t page_size;         /* P: tokens per cache page                           */
+    int32_t max_pages_per_seq; /* columns of the block table                         */
+    int32_t num_pages;         /* pages in the physical pool                         */
+} mlra_dims;
+
+/*
+ * Bytes of workspace mlra_decode needs for `dims` when its grid has
+ * `num_ctas` CTAs; num_ctas <= 0 means "the current device's SM count"
+ * (the grid mlra_decode launches).  Pure host computation (the SM count query
+ * is the only CUDA call).  Returns 0 if dims are invalid.
+ * The workspace holds the split-KV partial outputs (fp32), their
+ * log-sum-exps and the device error word.  Zero it once before first use
+ * (the error word must start at 0); mlra_decode never needs it re-zeroed.
+ */
+MLRA_API size_t mlra_decode_workspace_bytes(const mlra_dims* dims, int32_t num_ctas);
+
+/*
+ * MLRA decode attention for one step (the value-absorbed latent output of
+ * every head and branch).  For sequence n of length L = seqlens[n], token t
+ * lives at latent_cache[block_table[n][t / P]][t % P]; for every head h and
+ * branch b independently:
+ *   s_t = scale * (q_lat[n,h,b,:] . c_b[t] + q_rope[n,h,:] . k_r[t])
+ *   out[n,h,b,:] = out_scale * sum_t softmax_t(s)_t * c_b[t]
+ * ("The Core Insight" and "Mathematical Calibration" sections of the blog
+ * page named above; the RoPE query is one per head, the RoPE key one per
+ * token, both shared by the branches and already rotated.)
+ *
+ *   q_lat        bf16 [batch, heads, branches, d_c]   absorbed no-RoPE queries
+ *   q_rope       bf16 [batch, heads, d_r]             RoPE queries
+ *   latent_cache bf16 [num_pages, page_size, branches, d_c]
+ *   rope_cache   bf16 [num_pages, page_size, d_r]
+ *   block_table  int32 [batch, max_pages_per_seq]     page of each block; only
+ *                the first ceil(L/P) entries of a row are read
+ *   seqlens      int32 [batch]                        device memory
+ *   scale        softmax scale applied to the raw dot products
+ *   out_scale    variance-calibration factor applied to the output
+ *   out          bf16 [batch, heads, branches, d_c]   written
+ *   workspace    device buffer of >= mlra_decode_workspace_bytes(dims, 0)
+ *                bytes, zeroed before its first use; one call at a time
+ *
+ * Supported shapes: heads <= 16, d_c in {64, 128, 256, 512} with
+ * branches * d_c <= 512, d_r in {32, 64}, page_size in {16, 32, 64, 128}.
+ * Other shapes return MLRA_ERR_UNSUPPORTED.
+ * Returns MLRA_OK once the kernels are enqueued.
+ */
+MLRA_API mlra_status mlra_decode(const mlra_dims* dims, const void* q_lat, const void* q_rope,
+                        const void* latent_cache, const void* rope_cache,
+                        const int32_t* block_table, const int32_t* seqlens, float scale,
+                        float out_scale, void* out, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/*
+ * Per-branch W_UV up-projection followed by the branch sum ("The Core
+ * Insight" section: each branch is up-projected by its own matrix and the
+ * branch outputs are summed at the end):
+ *   y[n, h*d_h + j] = sum_b sum_k out_lat[n,h,b,k] * w_uv[b][k][h*d_h + j]
+ * fp32 accumulation, bf16 result.
+ *   out_lat bf16 [batch, heads, branches, d_c]  (the output of mlra_decode)
+ *   w_uv    bf16 [branches, d_c, heads * d_h]
+ *   y       bf16 [batch, heads * d_h]           written
+ * Supported: branches * d_c in {64, 128, ..., 512} (a multiple of 64),
+ * d_h in {64, 128}, any batch >= 1.
+ */
+MLRA_API mlra_status mlra_up_proj(int32_t batch, int32_t heads, int32_t branches, int32_t d_c, int32_t d_h,
+                         const void* out_lat, const void* w_uv, void* y, void* stream);
+
+/*
+ * Synchronises `stream`, returns the first device-side error code recorded
+ * in `workspace` since the last read (MLRA_OK if none) and resets it to 0.
+ * Returns MLRA_ERR_CUDA if the synchronisation or copy fails.
+ */
+MLRA_API mlra_status mlra_read_device_error(void* workspace, void* stream);
+
+/* Static, human-readable name of a status code. */
+MLRA_API const char* mlra_status_string(mlra_status status);
+
+/*
+ * The split-KV work partition mlra_decode uses, written for inspection.
+ * Sequence n has tiles_n = ceil(L_n / 128) token tiles (0 if L_n is
+ * invalid); the concatenation of all tiles is cut into `num_ctas` contiguous
+ * ranges of ceil(total / num_ctas) tiles, CTA c taking range c.
+ *   plan_out int32 device [num_ctas * 4 + batch * 2]:
+ *     per CTA c:  first tile (global), end tile (global), first sequence,
+ *                 last sequence touched (-1, -1 when the range is empty)
+ *     per seq n:  number of CTAs covering it (0 if invalid), first such CTA
+ * Returns after enqueueing one small kernel.
+ */
+MLRA_API mlra_status mlra_decode_plan(int32_t batch, int32_t page_size, int32_t max_pages_per_seq,
+                             const int32_t* seqlens, int32_t num_ctas, int32_t* plan_out,
+                             void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLRA_H */

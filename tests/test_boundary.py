@@ -1,0 +1,143 @@
+"""The C ABI without a GPU: the library loads, exports every symbol the
+header declares, and rejects bad arguments on the host before any CUDA work.
+Also checks the host-side plan statement's invariants."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from branch_latent_kv_b200 import binding as b
+from tests import plan_model
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"MLRA_API[^;{(]*?\b(mlra_\w+)\s*\(", text, flags=re.S))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = b.library()
+    declared = _declared_symbols()
+    assert {"mlra_decode", "mlra_up_proj", "mlra_decode_workspace_bytes",
+            "mlra_read_device_error", "mlra_status_string", "mlra_decode_plan"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings():
+    for code in range(8):
+        s = b.mlra_status_string(code)
+        assert s.startswith("MLRA_")
+    assert "unknown" in b.mlra_status_string(99)
+
+
+def _dims(**kw):
+    base = dict(batch=16, heads=16, branches=4, d_c=128, d_r=64, page_size=64,
+                max_pages_per_seq=128, num_pages=2048)
+    base.update(kw)
+    return b.mlra_dims(*[base[k] for k, _ in b.mlra_dims._fields_])
+
+
+def test_workspace_bytes_layout():
+    d = _dims()
+    n = b.mlra_decode_workspace_bytes(d, 148)
+    slots = 148 + 16
+
+    def a256(x):
+        return (x + 255) // 256 * 256
+    lse = 256 + 4 * slots * 4 * 16
+    assert n == a256(a256(lse) + 4 * slots * 4 * 16 * 128)
+    assert b.library().mlra_decode_workspace_bytes(ctypes.byref(_dims(batch=0)), 148) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(batch=0), b.MLRA_ERR_INVALID_ARG),
+    (dict(heads=0), b.MLRA_ERR_INVALID_ARG),
+    (dict(num_pages=0), b.MLRA_ERR_INVALID_ARG),
+    (dict(num_pages=2 ** 30), b.MLRA_ERR_INVALID_ARG),
+    (dict(heads=17), b.MLRA_ERR_UNSUPPORTED),
+    (dict(d_c=96), b.MLRA_ERR_UNSUPPORTED),
+    (dict(d_c=256, branches=4), b.MLRA_ERR_UNSUPPORTED),
+    (dict(d_r=48), b.MLRA_ERR_UNSUPPORTED),
+    (dict(page_size=8), b.MLRA_ERR_UNSUPPORTED),
+    (dict(page_size=256), b.MLRA_ERR_UNSUPPORTED),
+])
+def test_decode_rejects_bad_dims_before_any_cuda_call(kw, code):
+    lib = b.library()
+    fake = 1 << 20  # never dereferenced: validation fails first
+    st = lib.mlra_decode(ctypes.byref(_dims(**kw)), fake, fake, fake, fake, fake, fake, 0.1, 0.5,
+                         fake, fake, 1 << 30, None)
+    assert st == code
+
+
+def test_decode_rejects_misaligned_or_null_pointers():
+    lib = b.library()
+    ok = 1 << 20
+    args = [ok] * 6
+    for i in range(6):
+        bad = list(args)
+        bad[i] = ok + 2
+        st = lib.mlra_decode(ctypes.byref(_dims()), *bad, 0.1, 0.5, ok, ok, 1 << 30, None)
+        assert st == b.MLRA_ERR_INVALID_ARG
+    st = lib.mlra_decode(ctypes.byref(_dims()), *args, 0.1, 0.5, None, ok, 1 << 30, None)
+    assert st == b.MLRA_ERR_INVALID_ARG
+    st = lib.mlra_decode(ctypes.byref(_dims()), *args, float("nan"), 0.5, ok, ok, 1 << 30, None)
+    assert st == b.MLRA_ERR_INVALID_ARG
+    st = lib.mlra_decode(ctypes.byref(_dims()), *args, 0.1, 0.5, ok, None, 1 << 30, None)
+    assert st == b.MLRA_ERR_WORKSPACE
+    st = lib.mlra_decode(ctypes.byref(_dims()), *args, 0.1, 0.5, ok, ok + 16, 1 << 30, None)
+    assert st == b.MLRA_ERR_WORKSPACE
+
+
+def test_up_proj_rejects_bad_arguments():
+    lib = b.library()
+    ok = 1 << 20
+    assert lib.mlra_up_proj(0, 16, 4, 128, 128, ok, ok, ok, None) == b.MLRA_ERR_INVALID_ARG
+    assert lib.mlra_up_proj(16, 16, 4, 128, 128, ok + 8, ok, ok, None) == b.MLRA_ERR_INVALID_ARG
+    assert lib.mlra_up_proj(16, 16, 4, 128, 96, ok, ok, ok, None) == b.MLRA_ERR_UNSUPPORTED
+    assert lib.mlra_up_proj(16, 16, 3, 20, 128, ok, ok, ok, None) == b.MLRA_ERR_UNSUPPORTED
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 1, 1, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        b.mlra_decode(x, x[0], x, x[0], x[0, 0].int(), x[0, 0, 0].int(), 0.1, 0.5)
+
+
+@pytest.mark.parametrize("seqlens,ctas", [
+    ([8192] * 16, 148), ([1, 127, 128, 129, 0, 300], 7), ([131072] * 4, 148),
+    ([5], 148), ([0, 0], 4), (list(range(1, 2000, 37)), 148), ([128 * 1000 + 1, 3], 3),
+])
+def test_plan_model_covers_every_tile_once(seqlens, ctas):
+    P, maxp = 64, 4096
+    flat = plan_model.plan(seqlens, P, maxp, ctas)
+    tiles = [plan_model.seq_tiles(L, P, maxp) for L in seqlens]
+    total = sum(tiles)
+    covered = []
+    for c in range(ctas):
+        g0, g1, n0, n1 = flat[4 * c:4 * c + 4]
+        covered += list(range(g0, g1))
+        if g0 < g1:
+            assert 0 <= n0 <= n1 < len(seqlens)
+        else:
+            assert n0 == n1 == -1
+    assert covered == list(range(total))
+    # ranges differ in size by at most one chunk (the last non-empty one may be short)
+    sizes = [flat[4 * c + 1] - flat[4 * c] for c in range(ctas)]
+    assert max(sizes, default=0) - min([s for s in sizes if s] or [0]) <= max(sizes, default=0)
+    for n, t in enumerate(tiles):
+        splits, first = flat[4 * ctas + 2 * n:4 * ctas + 2 * n + 2]
+        if t == 0:
+            assert (splits, first) == (0, -1)
+        else:
+            owners = [c for c in range(ctas)
+                      if flat[4 * c] < flat[4 * c + 1] and flat[4 * c + 2] <= n <= flat[4 * c + 3]]
+            assert owners == list(range(first, first + splits))

@@ -1,0 +1,210 @@
+"""GPU path against the fp64 oracle, through the C ABI (needs a B200).
+
+Tolerance (bf16 inputs, fp32 accumulation, bf16 output): max-abs error
+<= 2e-2 and relative L2 error <= 5e-3 against the oracle.  Paging and index
+bookkeeping are bit-exact: page permutations give identical bits, length-1
+sequences return out_scale * c_b[0] exactly, the plan matches its CPU
+statement exactly.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from branch_latent_kv_b200 import binding as b
+from branch_latent_kv_b200.inputs import WORKLOADS, make_inputs
+from tests import plan_model
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS, REL_L2 = 2e-2, 5e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    torch.cuda.init()
+
+
+def _errors(gpu, ref, seq_ids=None):
+    g = gpu.detach().float().cpu().double().numpy()
+    if seq_ids is not None:
+        g, ref = g[seq_ids], ref[seq_ids]
+    diff = g - ref
+    return float(np.abs(diff).max()), float(np.linalg.norm(diff) / max(np.linalg.norm(ref), 1e-300))
+
+
+def _assert_close(gpu, ref, seq_ids=None, what=""):
+    max_abs, rel = _errors(gpu, ref, seq_ids)
+    assert max_abs <= MAX_ABS and rel <= REL_L2, f"{what}: max_abs={max_abs:.3e} rel_l2={rel:.3e}"
+    return max_abs, rel
+
+
+def _run(x, **kw):
+    return b.mlra_decode(x.q_lat, x.q_rope, x.latent_cache, x.rope_cache, x.block_table, x.seqlens,
+                         x.scale, x.out_scale, **kw)
+
+
+def _oracle(oracle_lib, x, seq_ids=None):
+    out, lse, status = oracle_lib.decode(x.q_lat.cpu(), x.q_rope.cpu(), x.latent_cache.cpu(),
+                                         x.rope_cache.cpu(), x.block_table.cpu(), x.seqlens.cpu(),
+                                         x.scale, x.out_scale, seq_ids=seq_ids)
+    return out, status
+
+
+def _score_gain(w, target_std):
+    """Query gain that makes the score standard deviation about target_std."""
+    return target_std / (w.scale * math.sqrt(1.0 / w.d_c + 1.0 / w.d_r))
+
+
+RAGGED = torch.tensor([1, 200, 777, 128, 129, 64, 1000, 255], dtype=torch.int32)
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+@pytest.mark.parametrize("peaked", [False, True])
+def test_small_cases_match_oracle(oracle_lib, name, peaked):
+    """Every workload's model shape on short ragged sequences (several tiles,
+    partial pages, NaN in every unused pool slot)."""
+    w = WORKLOADS[name]
+    n = min(w.batch, 4)
+    w = w.with_(batch=n, seqlen=None, seqlen_range=None, page_order="permuted")
+    seqlens = RAGGED[:n].clone()
+    if name == "tiny":
+        seqlens = torch.tensor([256], dtype=torch.int32)
+    gain = _score_gain(w, 4.0) if peaked else 1.0
+    x = make_inputs(w, seed=3, q_gain=gain, slack_pages=5, nan_fill_unused=True,
+                    seqlens=seqlens).to("cuda")
+    out = _run(x)
+    ref, status = _oracle(oracle_lib, x)
+    assert status == 0
+    assert torch.isfinite(out.float()).all()
+    _assert_close(out, ref, what=f"{name} peaked={peaked}")
+
+
+def test_tiny_workload_exact_recipe(oracle_lib):
+    x = make_inputs(WORKLOADS["tiny"]).to("cuda")
+    out = _run(x)
+    ref, status = _oracle(oracle_lib, x)
+    assert status == 0
+    _assert_close(out, ref, what="tiny")
+
+
+@pytest.mark.parametrize("name,samples", [
+    ("decode_2p9b", [0, 15]), ("long_context", [2]), ("ragged", [0, 17, 63]),
+    ("mla_equal_bytes", [5]), ("mlra4_equal_bytes", [31]), ("tp_shard", [0, 9]),
+])
+def test_full_size_sampled_sequences(oracle_lib, name, samples):
+    """Full-size workloads in the launch configuration the benchmark times;
+    the oracle checks sampled sequences."""
+    w = WORKLOADS[name]
+    x = make_inputs(w, device="cuda")
+    out = _run(x)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
+    ref, status = _oracle(oracle_lib, x, seq_ids=samples)
+    assert status == 0
+    _assert_close(out, ref, seq_ids=samples, what=name)
+
+
+def test_length_one_is_bit_exact():
+    w = WORKLOADS["decode_2p9b"].with_(batch=6, seqlen=1, page_order="permuted")
+    x = make_inputs(w, seed=5, q_gain=40.0, slack_pages=3, nan_fill_unused=True).to("cuda")
+    out = _run(x)
+    pages = x.block_table[:, 0].long()
+    want = (x.latent_cache[pages, 0].float() * x.out_scale).to(torch.bfloat16)  # [N, B, d_c]
+    assert torch.equal(out, want[:, None].expand_as(out))
+
+
+def test_page_permutation_gives_identical_bits():
+    w = WORKLOADS["decode_2p9b"].with_(batch=5, seqlen=None)
+    seqlens = torch.tensor([3000, 1, 640, 129, 2049], dtype=torch.int32)
+    x = make_inputs(w, seed=9, seqlens=seqlens, slack_pages=7).to("cuda")
+    perm = torch.randperm(x.latent_cache.shape[0], generator=torch.Generator().manual_seed(1)).cuda()
+    lat2 = torch.empty_like(x.latent_cache)
+    rope2 = torch.empty_like(x.rope_cache)
+    lat2[perm] = x.latent_cache
+    rope2[perm] = x.rope_cache
+    bt2 = torch.where(x.block_table >= 0, perm[x.block_table.long().clamp(min=0)].int(), x.block_table)
+    out1 = _run(x)
+    out2 = b.mlra_decode(x.q_lat, x.q_rope, lat2, rope2, bt2.contiguous(), x.seqlens, x.scale,
+                         x.out_scale)
+    assert torch.equal(out1, out2)
+
+
+def test_repeat_calls_are_deterministic():
+    x = make_inputs(WORKLOADS["ragged"].with_(batch=8), seed=2, device="cuda")
+    a = _run(x).clone()
+    for _ in range(3):
+        assert torch.equal(_run(x), a)
+
+
+def test_invalid_sequences_are_zeroed_and_reported(oracle_lib):
+    w = WORKLOADS["decode_2p9b"].with_(batch=4, seqlen=None)
+    seqlens = torch.tensor([500, 700, 900, 300], dtype=torch.int32)
+    x = make_inputs(w, seed=4, seqlens=seqlens).to("cuda")
+    ws = torch.zeros(b.mlra_decode_workspace_bytes(b.decode_dims(x.q_lat, x.q_rope, x.latent_cache,
+                                                                 x.block_table)),
+                     dtype=torch.uint8, device="cuda")
+    ref, _ = _oracle(oracle_lib, x)
+    bad_len = x.seqlens.clone()
+    bad_len[1] = 0
+    out = b.mlra_decode(x.q_lat, x.q_rope, x.latent_cache, x.rope_cache, x.block_table, bad_len,
+                        x.scale, x.out_scale, workspace=ws)
+    assert b.mlra_read_device_error(ws) == b.MLRA_ERR_DEVICE_BAD_SEQLEN
+    assert (out[1].float() == 0).all()
+    _assert_close(out, ref, seq_ids=[0, 2, 3], what="others unaffected")
+    assert b.mlra_read_device_error(ws) == b.MLRA_OK  # reading cleared it
+
+    bad_page = x.block_table.clone()
+    bad_page[2, 3] = x.latent_cache.shape[0]
+    out = b.mlra_decode(x.q_lat, x.q_rope, x.latent_cache, x.rope_cache, bad_page, x.seqlens,
+                        x.scale, x.out_scale, workspace=ws)
+    assert b.mlra_read_device_error(ws) == b.MLRA_ERR_DEVICE_BAD_INDEX
+    assert (out[2].float() == 0).all()
+    _assert_close(out, ref, seq_ids=[0, 1, 3], what="others unaffected")
+
+    too_long = x.seqlens.clone()
+    too_long[3] = x.block_table.shape[1] * w.page_size + 1
+    b.mlra_decode(x.q_lat, x.q_rope, x.latent_cache, x.rope_cache, x.block_table, too_long,
+                  x.scale, x.out_scale, workspace=ws)
+    assert b.mlra_read_device_error(ws) == b.MLRA_ERR_DEVICE_BAD_SEQLEN
+
+
+@pytest.mark.parametrize("seqlens,ctas", [
+    ([8192] * 16, 148), ([1, 127, 128, 129, 0, 300], 7), ([131072] * 4, 148), ([5], 148),
+    (list(range(1, 5000, 97)), 148), ([0, 3, 0], 2),
+])
+def test_plan_is_bit_exact(seqlens, ctas):
+    P, maxp = 64, 2048
+    sl = torch.tensor(seqlens, dtype=torch.int32, device="cuda")
+    got = b.mlra_decode_plan(sl, P, maxp, ctas).cpu().tolist()
+    assert got == plan_model.plan(seqlens, P, maxp, ctas)
+
+
+def test_up_proj_matches_oracle(oracle_lib):
+    w = WORKLOADS["decode_2p9b"]
+    x = make_inputs(w.with_(seqlen=300), seed=6).to("cuda")
+    out_lat = _run(x)
+    y = b.mlra_up_proj(out_lat, x.w_uv)
+    y_ref = oracle_lib.up_proj(out_lat.cpu(), x.w_uv.cpu(), w.d_h)
+    g = y.float().cpu().double().numpy()
+    assert np.abs(g - y_ref).max() <= MAX_ABS
+    assert np.linalg.norm(g - y_ref) / np.linalg.norm(y_ref) <= REL_L2
+    # end to end: fp64 decode -> fp64 up-projection
+    ref_lat, _ = _oracle(oracle_lib, x)
+    y_ref2 = oracle_lib.up_proj(ref_lat, x.w_uv.cpu(), w.d_h)
+    assert np.linalg.norm(g - y_ref2) / np.linalg.norm(y_ref2) <= REL_L2
+
+
+@pytest.mark.parametrize("batch", [1, 5, 16, 33, 300])
+def test_up_proj_batches(oracle_lib, batch):
+    torch.manual_seed(batch)
+    H, B, d_c, d_h = 16, 4, 128, 128
+    out_lat = (torch.randn(batch, H, B, d_c) / 10).to(torch.bfloat16).cuda()
+    w_uv = (torch.randn(B, d_c, H * d_h) / math.sqrt(B * d_c)).to(torch.bfloat16).cuda()
+    y = b.mlra_up_proj(out_lat, w_uv)
+    y_ref = oracle_lib.up_proj(out_lat.cpu(), w_uv.cpu(), d_h)
+    g = y.float().cpu().double().numpy()
+    assert np.linalg.norm(g - y_ref) / np.linalg.norm(y_ref) <= REL_L2
