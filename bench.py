@@ -48,7 +48,8 @@ FALLBACK_HBM_GBS = 6650.0
 # hash of the kernel sources it was taken on.  Reported as null whenever the
 # kernel sources differ from the captured ones.
 TRAFFIC_CAPTURE = {"sources_sha1": None, "bytes_per_launch": None}
-KERNEL_SOURCES = ["branch_latent_kv_b200/csrc/decode_simt.cu", "branch_latent_kv_b200/csrc/common.cuh"]
+KERNEL_SOURCES = ["branch_latent_kv_b200/csrc/decode_tc.cu", "branch_latent_kv_b200/csrc/sm100.cuh",
+                  "branch_latent_kv_b200/csrc/common.cuh"]
 
 
 def kernel_sources_sha1() -> str:

@@ -63,6 +63,8 @@ def library() -> ctypes.CDLL:
             lib.mlra_decode.argtypes = [dp, vp, vp, vp, vp, vp, vp, ctypes.c_float, ctypes.c_float,
                                         vp, vp, sz, vp]
             lib.mlra_decode.restype = ctypes.c_int
+            lib.mlra_decode_simt.argtypes = lib.mlra_decode.argtypes
+            lib.mlra_decode_simt.restype = ctypes.c_int
             lib.mlra_up_proj.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp]
             lib.mlra_up_proj.restype = ctypes.c_int
             lib.mlra_read_device_error.argtypes = [vp, vp]
@@ -134,14 +136,8 @@ def workspace_for(dims: mlra_dims, device: torch.device) -> torch.Tensor:
     return ws
 
 
-def mlra_decode(q_lat, q_rope, latent_cache, rope_cache, block_table, seqlens, scale, out_scale,
-                out=None, workspace=None, stream=None) -> torch.Tensor:
-    """MLRA decode attention (see mlra_decode in include/mlra.h).
-
-    q_lat bf16 [N,H,B,d_c], q_rope bf16 [N,H,d_r], latent_cache bf16
-    [pages,P,B,d_c], rope_cache bf16 [pages,P,d_r], block_table int32
-    [N,max_pages], seqlens int32 [N]; returns out bf16 [N,H,B,d_c].
-    """
+def _decode(entry, q_lat, q_rope, latent_cache, rope_cache, block_table, seqlens, scale, out_scale,
+            out=None, workspace=None, stream=None) -> torch.Tensor:
     dev = q_lat.device
     if dev.type != "cuda":
         raise ValueError("mlra_decode runs on CUDA tensors only")
@@ -165,13 +161,32 @@ def mlra_decode(q_lat, q_rope, latent_cache, rope_cache, block_table, seqlens, s
             raise ValueError("out must have the shape of q_lat")
     if workspace is None:
         workspace = workspace_for(dims, dev)
-    st = library().mlra_decode(ctypes.byref(dims), _ptr(q_lat), _ptr(q_rope), _ptr(latent_cache),
+    st = getattr(library(), entry)(ctypes.byref(dims), _ptr(q_lat), _ptr(q_rope), _ptr(latent_cache),
                                _ptr(rope_cache), _ptr(block_table), _ptr(seqlens), float(scale),
                                float(out_scale), _ptr(out), _ptr(workspace),
                                workspace.numel() * workspace.element_size(),
                                _stream_ptr(stream, dev))
-    _check(st, "mlra_decode")
+    _check(st, entry)
     return out
+
+
+def mlra_decode(q_lat, q_rope, latent_cache, rope_cache, block_table, seqlens, scale, out_scale,
+                out=None, workspace=None, stream=None) -> torch.Tensor:
+    """MLRA decode attention on the tensor cores (see mlra_decode in mlra.h).
+
+    q_lat bf16 [N,H,B,d_c], q_rope bf16 [N,H,d_r], latent_cache bf16
+    [pages,P,B,d_c], rope_cache bf16 [pages,P,d_r], block_table int32
+    [N,max_pages], seqlens int32 [N]; returns out bf16 [N,H,B,d_c].
+    """
+    return _decode("mlra_decode", q_lat, q_rope, latent_cache, rope_cache, block_table, seqlens,
+                   scale, out_scale, out, workspace, stream)
+
+
+def mlra_decode_simt(q_lat, q_rope, latent_cache, rope_cache, block_table, seqlens, scale,
+                     out_scale, out=None, workspace=None, stream=None) -> torch.Tensor:
+    """The same operation on the CUDA cores (see mlra_decode_simt in mlra.h)."""
+    return _decode("mlra_decode_simt", q_lat, q_rope, latent_cache, rope_cache, block_table,
+                   seqlens, scale, out_scale, out, workspace, stream)
 
 
 def mlra_up_proj(out_lat, w_uv, d_h: Optional[int] = None, y=None, stream=None) -> torch.Tensor:

@@ -15,7 +15,7 @@ bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr
 
 bool is_pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1)) == 0; }
 
-// Structural validity (INVALID_ARG) then kernel coverage (UNSUPPORTED).
+// Structural validity of the dimensions (INVALID_ARG).
 mlra_status check_dims(const mlra_dims* d) {
     if (d == nullptr) return MLRA_ERR_INVALID_ARG;
     if (d->batch < 1 || d->heads < 1 || d->branches < 1 || d->d_c < 1 || d->d_r < 1 ||
@@ -29,11 +29,23 @@ mlra_status check_dims(const mlra_dims* d) {
     // the plan counts 128-token tiles in int32
     if ((int64_t)d->batch * d->max_pages_per_seq * d->page_size / kTileTokens > (int64_t(1) << 30))
         return MLRA_ERR_INVALID_ARG;
-    if (d->heads > 16) return MLRA_ERR_UNSUPPORTED;
-    if (!is_pow2_in(d->d_c, 64, 512) || d->branches * d->d_c > 512) return MLRA_ERR_UNSUPPORTED;
-    if (d->d_r != 32 && d->d_r != 64) return MLRA_ERR_UNSUPPORTED;
+    if (d->batch > 65535) return MLRA_ERR_UNSUPPORTED;
+    return MLRA_OK;
+}
+
+// Shapes the tensor-core decode kernel implements.
+mlra_status check_tc_coverage(const mlra_dims* d) {
     if (!is_pow2_in(d->page_size, 16, 128)) return MLRA_ERR_UNSUPPORTED;
-    if (d->batch > 65535) return MLRA_ERR_UNSUPPORTED;  // combine grid.x limit is far above; keep a sane cap
+    if (!decode_tc_supported(d->branches, d->d_c, d->d_r, d->heads)) return MLRA_ERR_UNSUPPORTED;
+    return MLRA_OK;
+}
+
+// Shapes the CUDA-core decode kernel implements (its shared memory holds the
+// whole query block and a 32-token tile).
+mlra_status check_simt_coverage(const mlra_dims* d) {
+    if (d->d_c % 8 != 0 || d->d_r % 8 != 0 || d->heads > 64) return MLRA_ERR_UNSUPPORTED;
+    if ((int64_t)d->branches * d->d_c > 1024 || d->d_r > 256) return MLRA_ERR_UNSUPPORTED;
+    if (decode_simt_smem_bytes(d->heads, d->branches, d->d_c, d->d_r) > 232448) return MLRA_ERR_UNSUPPORTED;
     return MLRA_OK;
 }
 
@@ -50,23 +62,16 @@ int device_sm_count() {
 
 mlra_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MLRA_OK : MLRA_ERR_CUDA; }
 
-}  // namespace
+enum class Impl { kTensorCore, kSimt };
 
-extern "C" {
-
-size_t mlra_decode_workspace_bytes(const mlra_dims* dims, int32_t num_ctas) {
-    if (check_dims(dims) != MLRA_OK) return 0;
-    if (num_ctas <= 0) num_ctas = device_sm_count();
-    if (num_ctas <= 0) return 0;
-    return workspace_layout(dims->batch, dims->heads, dims->branches, dims->d_c, num_ctas).total;
-}
-
-mlra_status mlra_decode(const mlra_dims* dims, const void* q_lat, const void* q_rope,
+mlra_status decode_impl(Impl impl, const mlra_dims* dims, const void* q_lat, const void* q_rope,
                         const void* latent_cache, const void* rope_cache,
                         const int32_t* block_table, const int32_t* seqlens, float scale,
                         float out_scale, void* out, void* workspace, size_t workspace_bytes,
                         void* stream) {
-    const mlra_status s = check_dims(dims);
+    mlra_status s = check_dims(dims);
+    if (s != MLRA_OK) return s;
+    s = impl == Impl::kTensorCore ? check_tc_coverage(dims) : check_simt_coverage(dims);
     if (s != MLRA_OK) return s;
     if (!aligned16(q_lat) || !aligned16(q_rope) || !aligned16(latent_cache) ||
         !aligned16(rope_cache) || !aligned16(block_table) || !aligned16(seqlens) ||
@@ -106,9 +111,39 @@ mlra_status mlra_decode(const mlra_dims* dims, const void* q_lat, const void* q_
     a.out_scale = out_scale;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    mlra_status r = cuda_status(launch_decode_simt(a, st));
+    mlra_status r = cuda_status(impl == Impl::kTensorCore ? launch_decode_tc(a, st)
+                                                          : launch_decode_simt(a, st));
     if (r != MLRA_OK) return r;
     return cuda_status(launch_combine(a, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mlra_decode_workspace_bytes(const mlra_dims* dims, int32_t num_ctas) {
+    if (check_dims(dims) != MLRA_OK) return 0;
+    if (num_ctas <= 0) num_ctas = device_sm_count();
+    if (num_ctas <= 0) return 0;
+    return workspace_layout(dims->batch, dims->heads, dims->branches, dims->d_c, num_ctas).total;
+}
+
+mlra_status mlra_decode(const mlra_dims* dims, const void* q_lat, const void* q_rope,
+                        const void* latent_cache, const void* rope_cache,
+                        const int32_t* block_table, const int32_t* seqlens, float scale,
+                        float out_scale, void* out, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+    return decode_impl(Impl::kTensorCore, dims, q_lat, q_rope, latent_cache, rope_cache, block_table,
+                       seqlens, scale, out_scale, out, workspace, workspace_bytes, stream);
+}
+
+mlra_status mlra_decode_simt(const mlra_dims* dims, const void* q_lat, const void* q_rope,
+                             const void* latent_cache, const void* rope_cache,
+                             const int32_t* block_table, const int32_t* seqlens, float scale,
+                             float out_scale, void* out, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+    return decode_impl(Impl::kSimt, dims, q_lat, q_rope, latent_cache, rope_cache, block_table,
+                       seqlens, scale, out_scale, out, workspace, workspace_bytes, stream);
 }
 
 mlra_status mlra_up_proj(int32_t batch, int32_t heads, int32_t branches, int32_t d_c, int32_t d_h,

@@ -6,7 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/mlra.h"
+#include "mlra.h"
 
 namespace mlra {
 

@@ -1,0 +1,754 @@
+// decode_tc.cu -- split-KV MLRA decode on the sm_100a tensor cores.
+//
+// Method ("MLRA: Breaking the Sharding Bottleneck in Latent Attention",
+// wispaper.ai blog, section "The Core Insight: Sum of Branches, Not Sum of
+// Keys"): every latent branch b is attended independently,
+//   s_t = scale * (q_lat[h,b] . c_b[t] + q_rope[h] . k_r[t]),
+//   o[h,b] = sum_t softmax_t(s)_t c_b[t]       (values = the same latents),
+// with one RoPE key per token shared by all branches and heads.  The
+// decoding cost is the HBM -> SRAM movement of the cache at every step
+// (abstract of "Multi-Head Low-Rank Attention"), so the kernel streams each
+// token's latent and RoPE row through shared memory exactly once.
+//
+// Organisation (one persistent CTA per SM, 192 threads):
+//   warp 0     TMA producer: per 128-token tile, the RoPE tile and, per
+//              "pair" of 64-column chunks (128 latent columns), the paged
+//              latent rows (one 2-D box per page) into a ring of stages.
+//   warp 1     MMA issuer (one thread) and TMEM owner:
+//                S^T_b[t, h]  = C_b[t, :] . Q_b[h, :] + K_r[t, :] . Q_r[h, :]
+//                               M = 128 tokens, N = 16 heads, K = d_c + d_r
+//                O^T_b[k, h] += C_b[:, k]^T . P_b[:, h]
+//                               M = 128 latent columns, N = 16 heads, K = 128 tokens
+//              (the same shared-memory tile is the K-major A operand of the
+//              score MMA and the MN-major A operand of the output MMA).
+//   warps 2-5  softmax and epilogue: thread t owns token t of the tile (a
+//              TMEM lane); scores are base-2 logits; each (head, branch) has
+//              its own running max, rescaled only when a score exceeds it by
+//              more than 2^8 (then the exact column max is reduced and the
+//              TMEM accumulator is rescaled); P is written as bf16 to shared
+//              memory; at the end of a sequence's range the row sums are
+//              reduced and the normalised output (or a split partial with its
+//              log-sum-exp) is written.
+// Every wait is bounded: a wait that expires records
+// MLRA_ERR_DEVICE_TIMEOUT, and the CTA drains its copies and exits.
+#include <cudaTypedefs.h>
+
+#include <cstddef>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace mlra {
+namespace {
+
+using namespace sm100;
+
+constexpr int kHP = 16;             // heads padded to the MMA N
+constexpr int kT = kTileTokens;     // tokens per tile = MMA M
+constexpr int kThreads = 192;
+constexpr int kTmemCols = 128;
+constexpr float kRescaleLog2 = 8.0f;
+constexpr int kSmemLimit = 232448;  // max dynamic shared memory per CTA on sm_100
+
+template <int NB, int DC, int DR>
+struct Cfg {
+    static constexpr int W = NB * DC;                       // latent elements per token
+    static constexpr int NCHUNK = W / 64;                   // 64-column (128-byte) chunks
+    static constexpr int G = DC >= 128 ? 1 : 128 / DC;      // branches per step
+    static constexpr int PPS = DC >= 128 ? DC / 128 : 1;    // pairs per step
+    static constexpr int NSTEP = NB / G;                    // steps per tile
+    static constexpr int CHUNK_BYTES = kT * 128;            // 16 KB
+    static constexpr int PAIR_BYTES = 2 * CHUNK_BYTES;      // 32 KB
+    static constexpr int ROPE_ROW = DR * 2;                 // 128 or 64 bytes
+    static constexpr int ROPE_BYTES = kT * ROPE_ROW;
+    static constexpr int Q_CHUNK_BYTES = kHP * 128;         // [16 heads x 64 elements]
+    static constexpr int Q_BYTES = NCHUNK * Q_CHUNK_BYTES;
+    static constexpr int QR_BYTES = kHP * ROPE_ROW;                 // [16 heads x d_r]
+    static constexpr int QR_SPAN = (QR_BYTES + 1023) / 1024 * 1024;  // keeps the next region aligned
+    static constexpr int P_BRANCH_BYTES = kT * kHP * 2;     // 4 KB
+    static constexpr int P_BYTES = G * P_BRANCH_BYTES;
+    static constexpr int MISC_BYTES = 4096;
+    static constexpr int FIXED = 2 * ROPE_BYTES + Q_BYTES + QR_SPAN + 2 * P_BYTES + MISC_BYTES;
+    static constexpr int NSTAGE_FIT = (kSmemLimit - 1024 - FIXED) / PAIR_BYTES;
+    static constexpr int NSTAGE = NSTAGE_FIT > 8 ? 8 : NSTAGE_FIT;
+    // shared-memory offsets from a 1024-byte aligned base
+    static constexpr int OFF_PAIR = 0;
+    static constexpr int OFF_ROPE = OFF_PAIR + NSTAGE * PAIR_BYTES;
+    static constexpr int OFF_Q = OFF_ROPE + 2 * ROPE_BYTES;
+    static constexpr int OFF_QR = OFF_Q + Q_BYTES;
+    static constexpr int OFF_P = OFF_QR + QR_SPAN;
+    static constexpr int OFF_MISC = OFF_P + 2 * P_BYTES;
+    static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
+    // TMEM columns: O blocks first, then two S slots
+    static constexpr int O_BLOCKS = NSTEP * PPS * G;
+    static constexpr int S_COL0 = O_BLOCKS * kHP;
+    static constexpr int S_SLOT_COLS = G * kHP;
+    static_assert(NB % G == 0, "branches must fill whole steps");
+    static_assert(NSTAGE >= PPS, "a step's pairs must fit the stage ring");
+    // The score MMA of step s+1 is issued before the output MMA of step s
+    // (overlapping the softmax of s) only when both steps' pairs fit the ring.
+    static constexpr bool OVERLAP = 2 * PPS <= NSTAGE;
+    static_assert(S_COL0 + 2 * S_SLOT_COLS <= kTmemCols, "TMEM budget");
+    static_assert(SMEM_BYTES <= kSmemLimit, "shared-memory budget");
+    static_assert(OFF_QR + QR_BYTES <= OFF_P && OFF_Q + Q_BYTES <= OFF_QR && OFF_P + 2 * P_BYTES <= OFF_MISC,
+                  "shared-memory regions must not overlap");
+    static_assert(DR == 32 || DR == 64, "RoPE width");
+};
+
+// Barriers and scratch in the MISC region.
+template <int NSTAGE>
+struct Misc {
+    uint64_t pair_full[NSTAGE];
+    uint64_t pair_empty[NSTAGE];
+    uint64_t rope_full[2];
+    uint64_t rope_empty[2];
+    uint64_t s_full[2];
+    uint64_t p_full[2];
+    uint64_t o_done;    // one phase per output MMA step (rescale path: at most one outstanding)
+    uint64_t seg_done;  // one phase per sequence range: every output MMA of the range finished
+    uint64_t q_full;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    int plan[4];
+    float red_max[4][2 * kHP];
+    float red_sum[4][4 * kHP];
+    alignas(16) float m_run[8 * kHP];  // running max per (branch, head), base-2 logits; read as float4
+};
+
+static_assert(offsetof(Misc<5>, m_run) % 16 == 0 && offsetof(Misc<4>, m_run) % 16 == 0 &&
+              offsetof(Misc<6>, m_run) % 16 == 0, "float4 access to m_run");
+
+struct Maps {
+    CUtensorMap lat;
+    CUtensorMap rope;
+};
+
+template <int DR>
+__device__ __forceinline__ uint64_t rope_desc(uint32_t addr) {
+    return DR == 64 ? smem_desc(addr, 16, 1024, kLayoutSw128) : smem_desc(addr, 16, 512, kLayoutSw64);
+}
+
+// The sequence-range walk every role performs identically.
+__device__ __forceinline__ bool next_segment(const DecodeArgs& a, int& n, int first, int g0, int g1,
+                                             int& L, int& tiles, int& tb, int& te) {
+    while (n < a.batch && first < g1) {
+        L = __ldg(a.seqlens + n);
+        tiles = seq_tiles(L, a.page_size, a.max_pages);
+        if (tiles == 0) {
+            ++n;
+            continue;
+        }
+        tb = max(g0, first) - first;
+        te = min(g1, first + tiles) - first;
+        return true;
+    }
+    return false;
+}
+
+template <int NB, int DC, int DR>
+__global__ void __launch_bounds__(kThreads, 1)
+decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
+    using C = Cfg<NB, DC, DR>;
+    using M = Misc<C::NSTAGE>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    M& misc = *reinterpret_cast<M*>(sm + C::OFF_MISC);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int P = a.page_size;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::NSTAGE; ++i) {
+            mbar_init(&misc.pair_full[i], 1);
+            mbar_init(&misc.pair_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&misc.rope_full[i], 1);
+            mbar_init(&misc.rope_empty[i], 1);
+            mbar_init(&misc.s_full[i], 1);
+            mbar_init(&misc.p_full[i], 4);
+        }
+        mbar_init(&misc.o_done, 1);
+        mbar_init(&misc.seg_done, 1);
+        mbar_init(&misc.q_full, 4);
+        mbar_init(&misc.drain, 1);
+        misc.abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        const int total = warp_total_tiles(a.seqlens, a.batch, P, a.max_pages);
+        const int chunk = total > 0 ? ceil_div(total, a.num_ctas) : 0;
+        const int g0 = blockIdx.x * chunk;
+        int n0 = -1, f0 = 0;
+        if (g0 < total) warp_find_seq(a.seqlens, a.batch, P, a.max_pages, g0, &n0, &f0);
+        if (lane == 0) {
+            misc.plan[0] = total;
+            misc.plan[1] = chunk;
+            misc.plan[2] = n0;
+            misc.plan[3] = f0;
+        }
+        prefetch_tensormap(&maps.lat);
+        prefetch_tensormap(&maps.rope);
+    }
+    if (warp == 1) {
+        tmem_alloc(&misc.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const int total = misc.plan[0], chunk = misc.plan[1];
+    const int g0 = blockIdx.x * chunk, g1 = min(g0 + chunk, total);
+    const uint32_t tmem = misc.tmem_base;
+    volatile int* abort_flag = &misc.abort_flag;
+
+    if (g0 < g1) {
+        if (warp == 0) {
+            // ------------------------------------------------------------ producer
+            int n = misc.plan[2], first = misc.plan[3];
+            int L, tiles, tb, te;
+            uint32_t pc = 0, tc = 0;
+            bool ok = true;
+            while (ok && next_segment(a, n, first, g0, g1, L, tiles, tb, te)) {
+                const int32_t* bt = a.block_table + (size_t)n * a.max_pages;
+                int win_base = -(1 << 30), win_val = 0;
+                for (int j = tb; j < te && ok; ++j) {
+                    const int tok0 = j * kT;
+                    const int valid = min(kT, L - tok0);
+                    const int npages = ceil_div(valid, P);
+                    const int page0 = tok0 / P;
+                    if (page0 < win_base || page0 + npages > win_base + 32) {
+                        win_base = page0;
+                        const int idx = page0 + lane;
+                        const int v = idx < a.max_pages ? __ldg(bt + idx) : 0;
+                        win_val = (v >= 0 && v < a.num_pages) ? v : 0;  // bad entries are reported by the softmax warps
+                    }
+                    const int rslot = tc & 1;
+                    if (lane == 0) {
+                        ok = mbar_wait(&misc.rope_empty[rslot], ((tc >> 1) & 1) ^ 1);
+                        if (ok) mbar_arrive_expect_tx(&misc.rope_full[rslot], npages * P * C::ROPE_ROW);
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    for (int q = 0; q < npages; ++q) {
+                        const int page = __shfl_sync(0xffffffffu, win_val, page0 + q - win_base);
+                        if (lane == 0)
+                            tma_load_2d(sm + C::OFF_ROPE + rslot * C::ROPE_BYTES + q * P * C::ROPE_ROW,
+                                        &maps.rope, 0, page * P, &misc.rope_full[rslot]);
+                    }
+                    ++tc;
+                    for (int sp = 0; sp < C::NSTEP * C::PPS && ok; ++sp) {
+                        const int stage = pc % C::NSTAGE;
+                        if (lane == 0) {
+                            ok = mbar_wait(&misc.pair_empty[stage], ((pc / C::NSTAGE) & 1) ^ 1);
+                            if (ok) mbar_arrive_expect_tx(&misc.pair_full[stage], 2 * npages * P * 128);
+                        }
+                        ok = __shfl_sync(0xffffffffu, ok, 0);
+                        if (!ok) break;
+                        const int chunk0 = sp * 2;  // pairs are consecutive 128-column groups
+                        for (int q = 0; q < npages; ++q) {
+                            const int page = __shfl_sync(0xffffffffu, win_val, page0 + q - win_base);
+                            if (lane == 0) {
+                                uint8_t* dst = sm + C::OFF_PAIR + stage * C::PAIR_BYTES + q * P * 128;
+                                tma_load_2d(dst, &maps.lat, chunk0 * 64, page * P, &misc.pair_full[stage]);
+                                tma_load_2d(dst + C::CHUNK_BYTES, &maps.lat, chunk0 * 64 + 64, page * P,
+                                            &misc.pair_full[stage]);
+                            }
+                        }
+                        ++pc;
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok && !*abort_flag, 0);
+                }
+                first += tiles;
+                ++n;
+            }
+            if (!ok) {
+                if (lane == 0) {
+                    record_error(a.err, MLRA_ERR_DEVICE_TIMEOUT);
+                    *abort_flag = 1;
+                }
+            }
+            // drain: wait (bounded) for the copies issued last, so that no
+            // TMA write lands after this CTA has exited
+            if (lane == 0) {
+                for (uint32_t i = 0; i < (uint32_t)C::NSTAGE && i < pc; ++i) {
+                    const uint32_t k = pc - 1 - i;
+                    mbar_wait(&misc.pair_full[k % C::NSTAGE], (k / C::NSTAGE) & 1, 200000000ull);
+                }
+                for (uint32_t i = 0; i < 2 && i < tc; ++i) {
+                    const uint32_t k = tc - 1 - i;
+                    mbar_wait(&misc.rope_full[k & 1], (k >> 1) & 1, 200000000ull);
+                }
+            }
+        } else if (warp == 1) {
+            // ------------------------------------------------------------ MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t IDESC_S = idesc_bf16_f32(128, kHP, false, false);
+                constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, kHP, true, true);
+                const uint32_t sm_base = smem_u32(sm);
+                int n = misc.plan[2], first = misc.plan[3];
+                int L, tiles, tb, te;
+                uint32_t gs = 0, pc = 0, tc = 0, sc = 0;
+                bool ok = true;
+                bool have_prev = false;
+                uint32_t prev_gs = 0, prev_pc = 0;
+                int prev_st = 0;
+                bool prev_first = false;
+
+                auto issue_pv = [&](uint32_t pgs, int pst, uint32_t ppc, bool pfirst) -> bool {
+                    if (!mbar_wait(&misc.p_full[pgs & 1], (pgs >> 1) & 1)) return false;
+                    tc_fence_after();
+                    const uint32_t p_base = sm_base + C::OFF_P + (pgs & 1) * C::P_BYTES;
+#pragma unroll
+                    for (int p = 0; p < C::PPS; ++p) {
+                        const uint32_t a_base = sm_base + C::OFF_PAIR + ((ppc + p) % C::NSTAGE) * C::PAIR_BYTES;
+#pragma unroll
+                        for (int g = 0; g < C::G; ++g) {
+                            const uint32_t d = tmem + ((pst * C::PPS + p) * C::G + g) * kHP;
+#pragma unroll
+                            for (int kt = 0; kt < kT / 16; ++kt) {
+                                const uint64_t ad = smem_desc(a_base + kt * 2048, C::CHUNK_BYTES, 1024, kLayoutSw128);
+                                const uint64_t bd = smem_desc(p_base + g * C::P_BRANCH_BYTES + kt * 256, 128,
+                                                              2048, kLayoutNone);
+                                mma_bf16(d, ad, bd, IDESC_PV, (pfirst && kt == 0) ? 0u : 1u);
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int p = 0; p < C::PPS; ++p) mma_commit(&misc.pair_empty[(ppc + p) % C::NSTAGE]);
+                    mma_commit(&misc.o_done);
+                    return true;
+                };
+
+                while (ok && next_segment(a, n, first, g0, g1, L, tiles, tb, te)) {
+                    ok = mbar_wait(&misc.q_full, sc & 1);
+                    tc_fence_after();
+                    for (int j = tb; j < te && ok; ++j) {
+                        const int rslot = tc & 1;
+                        ok = mbar_wait(&misc.rope_full[rslot], (tc >> 1) & 1);
+                        const uint32_t rope_base = sm_base + C::OFF_ROPE + rslot * C::ROPE_BYTES;
+#pragma unroll 1
+                        for (int st = 0; st < C::NSTEP && ok; ++st) {
+                            for (int p = 0; p < C::PPS && ok; ++p)
+                                ok = mbar_wait(&misc.pair_full[(pc + p) % C::NSTAGE], ((pc + p) / C::NSTAGE) & 1);
+                            if (!ok) break;
+                            tc_fence_after();
+#pragma unroll
+                            for (int g = 0; g < C::G; ++g) {
+                                const int b = st * C::G + g;
+                                const uint32_t d = tmem + C::S_COL0 + (gs & 1) * C::S_SLOT_COLS + g * kHP;
+                                uint32_t acc = 0;
+#pragma unroll
+                                for (int c = 0; c < DC / 64; ++c) {
+                                    const int gc = b * (DC / 64) + c;          // chunk of the token row
+                                    const int pp = gc / 2 - st * C::PPS;        // pair within this step
+                                    const uint32_t a_base = sm_base + C::OFF_PAIR +
+                                                            ((pc + pp) % C::NSTAGE) * C::PAIR_BYTES +
+                                                            (gc & 1) * C::CHUNK_BYTES;
+                                    const uint32_t q_base = sm_base + C::OFF_Q + gc * C::Q_CHUNK_BYTES;
+#pragma unroll
+                                    for (int kk = 0; kk < 4; ++kk) {
+                                        mma_bf16(d, smem_desc(a_base + kk * 32, 16, 1024, kLayoutSw128),
+                                                 smem_desc(q_base + kk * 32, 16, 1024, kLayoutSw128), IDESC_S, acc);
+                                        acc = 1;
+                                    }
+                                }
+#pragma unroll
+                                for (int kk = 0; kk < DR / 16; ++kk)
+                                    mma_bf16(d, rope_desc<DR>(rope_base + kk * 32),
+                                             rope_desc<DR>(sm_base + C::OFF_QR + kk * 32), IDESC_S, 1u);
+                            }
+                            mma_commit(&misc.s_full[gs & 1]);
+                            if (st == C::NSTEP - 1) mma_commit(&misc.rope_empty[rslot]);
+                            if (C::OVERLAP) {
+                                if (have_prev) ok = issue_pv(prev_gs, prev_st, prev_pc, prev_first);
+                                have_prev = true;
+                                prev_gs = gs;
+                                prev_st = st;
+                                prev_pc = pc;
+                                prev_first = (j == tb);
+                            } else {
+                                ok = issue_pv(gs, st, pc, j == tb);
+                            }
+                            pc += C::PPS;
+                            ++gs;
+                        }
+                        ++tc;
+                        if (*abort_flag) ok = false;
+                    }
+                    if (ok && have_prev) ok = issue_pv(prev_gs, prev_st, prev_pc, prev_first);
+                    have_prev = false;
+                    if (ok) mma_commit(&misc.seg_done);
+                    ++sc;
+                    first += tiles;
+                    ++n;
+                }
+                if (!ok) {
+                    record_error(a.err, MLRA_ERR_DEVICE_TIMEOUT);
+                    *abort_flag = 1;
+                }
+                // drain: every MMA issued above completes before TMEM is freed
+                mma_commit(&misc.drain);
+                mbar_wait(&misc.drain, 0, 200000000ull);
+            }
+            __syncwarp();
+        } else {
+            // ------------------------------------------------------------ softmax + epilogue
+            const int quad = warp & 3;                 // TMEM lane quadrant of this warp
+            const int row = quad * 32 + lane;          // token (S) / latent row (O)
+            const int stid = threadIdx.x - 64;         // 0..127 within the group
+            const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+            const int H = a.heads;
+            int n = misc.plan[2], first = misc.plan[3];
+            int L, tiles, tb, te;
+            uint32_t gs = 0, sc = 0;
+            float l[NB][kHP];  // this thread's share of the softmax denominators
+            bool dead = false;
+
+            while (!dead && next_segment(a, n, first, g0, g1, L, tiles, tb, te)) {
+                // queries of sequence n -> shared memory (128-byte swizzled, K-major)
+                {
+                    const uint4* q_src = reinterpret_cast<const uint4*>(a.q_lat + (size_t)n * H * C::W);
+                    constexpr int UPR = C::W / 8;  // 16-byte units per head row
+                    for (int i = stid; i < kHP * UPR; i += 128) {
+                        const int h = i / UPR, rem = i % UPR, gc = rem / 8, u = rem % 8;
+                        uint4 v = make_uint4(0, 0, 0, 0);
+                        if (h < H) v = __ldg(q_src + (size_t)h * UPR + rem);
+                        *reinterpret_cast<uint4*>(sm + C::OFF_Q + gc * C::Q_CHUNK_BYTES + h * 128 +
+                                                  ((u ^ (h & 7)) << 4)) = v;
+                    }
+                    const uint4* qr_src = reinterpret_cast<const uint4*>(a.q_rope + (size_t)n * H * DR);
+                    constexpr int RU = DR / 8;
+                    for (int i = stid; i < kHP * RU; i += 128) {
+                        const int h = i / RU, u = i % RU;
+                        uint4 v = make_uint4(0, 0, 0, 0);
+                        if (h < H) v = __ldg(qr_src + (size_t)h * RU + u);
+                        const int sw = DR == 64 ? (u ^ (h & 7)) : (u ^ ((h >> 1) & 3));
+                        *reinterpret_cast<uint4*>(sm + C::OFF_QR + h * C::ROPE_ROW + (sw << 4)) = v;
+                    }
+                }
+                // block-table entries of this range must name real pages
+                bool bad = false;
+                {
+                    const int32_t* bt = a.block_table + (size_t)n * a.max_pages;
+                    const int p0 = tb * kT / P, p1 = ceil_div(min(te * kT, L), P);
+                    for (int i = p0 + stid; i < p1; i += 128) {
+                        const int v = __ldg(bt + i);
+                        bad |= (v < 0 || v >= a.num_pages);
+                    }
+                }
+                bad = named_bar_or<1, 128>(bad);
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&misc.q_full);
+#pragma unroll
+                for (int b = 0; b < NB; ++b)
+#pragma unroll
+                    for (int i = 0; i < kHP; ++i) l[b][i] = 0.f;
+                if (stid < NB * kHP) misc.m_run[stid] = -INFINITY;
+                named_bar_sync<1, 128>();
+
+                for (int j = tb; j < te && !dead; ++j) {
+                    const int valid = min(kT, L - j * kT);
+                    const bool masked = row >= valid;
+#pragma unroll
+                    for (int st = 0; st < C::NSTEP; ++st) {
+                        const bool ok = mbar_wait(&misc.s_full[gs & 1], (gs >> 1) & 1);
+                        tc_fence_after();
+                        float x[C::G][kHP];
+#pragma unroll
+                        for (int g = 0; g < C::G; ++g)
+                            tmem_ld16(tmem + lane_off + C::S_COL0 + (gs & 1) * C::S_SLOT_COLS + g * kHP, x[g]);
+                        tmem_wait_ld();
+                        float m[C::G][kHP];
+#pragma unroll
+                        for (int g = 0; g < C::G; ++g)
+#pragma unroll
+                            for (int i = 0; i < kHP; i += 4) {
+                                const float4 v = *reinterpret_cast<const float4*>(&misc.m_run[(st * C::G + g) * kHP + i]);
+                                m[g][i] = v.x;
+                                m[g][i + 1] = v.y;
+                                m[g][i + 2] = v.z;
+                                m[g][i + 3] = v.w;
+                            }
+                        bool need = false;
+#pragma unroll
+                        for (int g = 0; g < C::G; ++g) {
+#pragma unroll
+                            for (int i = 0; i < kHP; ++i) {
+                                x[g][i] = masked ? -INFINITY : x[g][i] * a.scale_log2;
+                                need |= x[g][i] > m[g][i] + kRescaleLog2;
+                            }
+                        }
+                        if (named_bar_or<1, 128>(need || !ok)) {
+                            if (named_bar_or<1, 128>(!ok)) {
+                                dead = true;
+                                break;
+                            }
+                            // exact column max over the tile's 128 tokens
+#pragma unroll
+                            for (int g = 0; g < C::G; ++g)
+#pragma unroll
+                                for (int i = 0; i < kHP; ++i) {
+                                    float v = x[g][i];
+#pragma unroll
+                                    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+                                    if (lane == 0) misc.red_max[quad][g * kHP + i] = v;
+                                }
+                            named_bar_sync<1, 128>();
+                            float alpha[C::G][kHP];
+#pragma unroll
+                            for (int g = 0; g < C::G; ++g) {
+                                const int b = st * C::G + g;
+#pragma unroll
+                                for (int i = 0; i < kHP; ++i) {
+                                    const float tmax = fmaxf(fmaxf(misc.red_max[0][g * kHP + i], misc.red_max[1][g * kHP + i]),
+                                                             fmaxf(misc.red_max[2][g * kHP + i], misc.red_max[3][g * kHP + i]));
+                                    const float mnew = fmaxf(m[g][i], tmax);
+                                    alpha[g][i] = exp2f(m[g][i] - mnew);
+                                    m[g][i] = mnew;
+                                    l[b][i] *= alpha[g][i];
+                                }
+                            }
+                            // every thread read the old maxima before the barrier above; the
+                            // barrier below publishes the new ones (and frees red_max)
+                            if (stid == 0) {
+#pragma unroll
+                                for (int g = 0; g < C::G; ++g)
+#pragma unroll
+                                    for (int i = 0; i < kHP; ++i) misc.m_run[(st * C::G + g) * kHP + i] = m[g][i];
+                            }
+                            named_bar_sync<1, 128>();
+                            if (j > tb) {
+                                // O holds earlier tiles of this range: rescale it once the
+                                // previous output MMA has finished
+                                const bool ok2 = mbar_wait(&misc.o_done, (gs - 1) & 1);
+                                if (named_bar_or<1, 128>(!ok2)) {
+                                    dead = true;
+                                    break;
+                                }
+                                tc_fence_after();
+#pragma unroll
+                                for (int p = 0; p < C::PPS; ++p)
+#pragma unroll
+                                    for (int g = 0; g < C::G; ++g) {
+                                        const uint32_t col = ((st * C::PPS + p) * C::G + g) * kHP;
+                                        float o[kHP];
+                                        tmem_ld16(tmem + lane_off + col, o);
+                                        tmem_wait_ld();
+#pragma unroll
+                                        for (int i = 0; i < kHP; ++i) o[i] *= alpha[g][i];
+                                        tmem_st16(tmem + lane_off + col, o);
+                                    }
+                                tmem_wait_st();
+                            }
+                        }
+                        // probabilities -> bf16 P (MN-major, 8x8 core matrices)
+                        uint8_t* p_slot = sm + C::OFF_P + (gs & 1) * C::P_BYTES;
+#pragma unroll
+                        for (int g = 0; g < C::G; ++g) {
+                            const int b = st * C::G + g;
+                            uint32_t packed[kHP / 2];
+#pragma unroll
+                            for (int i = 0; i < kHP; i += 2) {
+                                const float p0 = exp2f(x[g][i] - m[g][i]);
+                                const float p1 = exp2f(x[g][i + 1] - m[g][i + 1]);
+                                l[b][i] += p0;
+                                l[b][i + 1] += p1;
+                                __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
+                                packed[i / 2] = *reinterpret_cast<uint32_t*>(&pr);
+                            }
+                            uint8_t* dst = p_slot + g * C::P_BRANCH_BYTES + (row >> 3) * 128 + (row & 7) * 16;
+                            *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                            *reinterpret_cast<uint4*>(dst + 2048) = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                        }
+                        // rows past the end of the sequence (stale or poisoned data)
+                        // become zero before the output MMA reads them
+                        if (masked) {
+#pragma unroll
+                            for (int p = 0; p < C::PPS; ++p) {
+                                uint8_t* pair = sm + C::OFF_PAIR + ((gs * C::PPS + p) % C::NSTAGE) * C::PAIR_BYTES;
+#pragma unroll
+                                for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+                                    for (int u = 0; u < 8; ++u)
+                                        *reinterpret_cast<uint4*>(pair + h2 * C::CHUNK_BYTES + row * 128 + u * 16) =
+                                            make_uint4(0, 0, 0, 0);
+                            }
+                        }
+                        fence_proxy_async_smem();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&misc.p_full[gs & 1]);
+                        ++gs;
+                    }
+                }
+                if (dead) break;
+
+                // ---------------------------------------------------- epilogue
+                // (two output MMAs may still be in flight here, so o_done's parity
+                // cannot tell them apart: wait for the range's own barrier)
+                const bool ok = mbar_wait(&misc.seg_done, sc & 1);
+                if (named_bar_or<1, 128>(!ok)) {
+                    dead = true;
+                    break;
+                }
+                tc_fence_after();
+                // row sums over all tokens of the range
+#pragma unroll
+                for (int b = 0; b < NB; ++b)
+#pragma unroll
+                    for (int i = 0; i < kHP; ++i) {
+                        float v = l[b][i];
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                        l[b][i] = v;
+                    }
+                // reduce across the four warps, NB*16 values at a time in chunks of 64
+#pragma unroll
+                for (int b0 = 0; b0 < NB; b0 += 4) {
+                    if (lane == 0) {
+#pragma unroll
+                        for (int b = b0; b < b0 + 4 && b < NB; ++b)
+#pragma unroll
+                            for (int i = 0; i < kHP; ++i) misc.red_sum[quad][(b - b0) * kHP + i] = l[b][i];
+                    }
+                    named_bar_sync<1, 128>();
+#pragma unroll
+                    for (int b = b0; b < b0 + 4 && b < NB; ++b)
+#pragma unroll
+                        for (int i = 0; i < kHP; ++i) {
+                            const int k = (b - b0) * kHP + i;
+                            l[b][i] = misc.red_sum[0][k] + misc.red_sum[1][k] + misc.red_sum[2][k] + misc.red_sum[3][k];
+                        }
+                    named_bar_sync<1, 128>();
+                }
+                const int first_cta = first / chunk, last_cta = (first + tiles - 1) / chunk;
+                const bool single = first_cta == last_cta;
+                const size_t slot = (size_t)blockIdx.x + n;
+#pragma unroll
+                for (int st = 0; st < C::NSTEP; ++st)
+#pragma unroll
+                    for (int p = 0; p < C::PPS; ++p)
+#pragma unroll
+                        for (int g = 0; g < C::G; ++g) {
+                            const int colw = (st * C::PPS + p) * 128 + row;  // latent column of the token row
+                            const int b = colw / DC, k = colw % DC;
+                            float o[kHP];
+                            tmem_ld16(tmem + lane_off + ((st * C::PPS + p) * C::G + g) * kHP, o);
+                            tmem_wait_ld();
+                            if (b != st * C::G + g) continue;  // rows of the other branch of a pair
+#pragma unroll
+                            for (int i = 0; i < kHP; ++i) {
+                                if (i >= H) break;
+                                const float v = bad ? 0.f : o[i] / l[st * C::G + g][i];
+                                if (single)
+                                    a.out[(((size_t)n * H + i) * NB + b) * DC + k] = to_bf16(v * a.out_scale);
+                                else
+                                    a.o_part[((slot * NB + b) * H + i) * DC + k] = v;
+                            }
+                        }
+                if (!single) {
+#pragma unroll
+                    for (int b = 0; b < NB; ++b)
+#pragma unroll
+                        for (int i = 0; i < kHP; ++i)
+                            if (stid == b * kHP + i && i < H)
+                                a.lse_part[(slot * NB + b) * H + i] =
+                                    bad ? bad_split_marker() : misc.m_run[b * kHP + i] + log2f(l[b][i]);
+                }
+                if (bad && stid == 0) record_error(a.err, MLRA_ERR_DEVICE_BAD_INDEX);
+                tc_fence_before();
+                ++sc;
+                first += tiles;
+                ++n;
+            }
+            if (dead && stid == 0) {
+                record_error(a.err, MLRA_ERR_DEVICE_TIMEOUT);
+                *abort_flag = 1;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+bool encode_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
+               uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {inner * 2};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int NB, int DC, int DR>
+cudaError_t launch_cfg(const DecodeArgs& a, cudaStream_t stream) {
+    using C = Cfg<NB, DC, DR>;
+    Maps maps;
+    const uint64_t rows = (uint64_t)a.num_pages * a.page_size;
+    const uint32_t box_rows = (uint32_t)a.page_size;
+    if (!encode_2d(&maps.lat, a.latent, (uint64_t)C::W, rows, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&maps.rope, a.rope, (uint64_t)DR, rows, DR, box_rows,
+                   DR == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+        return cudaErrorInvalidValue;
+    auto kernel = decode_tc_kernel<NB, DC, DR>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    kernel<<<a.num_ctas, kThreads, C::SMEM_BYTES, stream>>>(maps, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool decode_tc_supported(int branches, int d_c, int d_r, int heads) {
+    if (heads > kHP || (d_r != 32 && d_r != 64)) return false;
+    switch (d_c) {
+        case 64: return branches == 2 || branches == 4;
+        case 128: return branches == 1 || branches == 2 || branches == 4;
+        case 256: return branches == 1 || branches == 2;
+        case 512: return branches == 1;
+    }
+    return false;
+}
+
+cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
+#define MLRA_TC_CASE(NB_, DC_)                                                          \
+    if (a.branches == NB_ && a.d_c == DC_)                                              \
+        return a.d_r == 64 ? launch_cfg<NB_, DC_, 64>(a, stream) : launch_cfg<NB_, DC_, 32>(a, stream);
+    MLRA_TC_CASE(2, 64)
+    MLRA_TC_CASE(4, 64)
+    MLRA_TC_CASE(1, 128)
+    MLRA_TC_CASE(2, 128)
+    MLRA_TC_CASE(4, 128)
+    MLRA_TC_CASE(1, 256)
+    MLRA_TC_CASE(2, 256)
+    MLRA_TC_CASE(1, 512)
+#undef MLRA_TC_CASE
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace mlra

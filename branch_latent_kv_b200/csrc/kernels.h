@@ -29,6 +29,10 @@ struct DecodeArgs {
 // Split-KV decode on CUDA cores (fp32 FMA).  Writes final outputs of
 // single-split sequences and partials of the others.
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream);
+
+// Split-KV decode on the tensor cores (tcgen05 + TMA); see decode_tc.cu.
+bool decode_tc_supported(int branches, int d_c, int d_r, int heads);
+cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);
 size_t decode_simt_smem_bytes(int heads, int branches, int d_c, int d_r);
 
 // Log-sum-exp merge of the partials, out_scale, bf16 cast; zeros and an error

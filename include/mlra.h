@@ -108,9 +108,11 @@ MLRA_API size_t mlra_decode_workspace_bytes(const mlra_dims* dims, int32_t num_c
  *   workspace    device buffer of >= mlra_decode_workspace_bytes(dims, 0)
  *                bytes, zeroed before its first use; one call at a time
  *
- * Supported shapes: heads <= 16, d_c in {64, 128, 256, 512} with
- * branches * d_c <= 512, d_r in {32, 64}, page_size in {16, 32, 64, 128}.
- * Other shapes return MLRA_ERR_UNSUPPORTED.
+ * Runs on the tensor cores (tcgen05, operands staged by TMA).  Supported
+ * shapes: heads <= 16; (branches, d_c) in {(2,64), (4,64), (1,128), (2,128),
+ * (4,128), (1,256), (2,256), (1,512)}; d_r in {32, 64}; page_size in
+ * {16, 32, 64, 128}.  Other shapes return MLRA_ERR_UNSUPPORTED
+ * (mlra_decode_simt covers more).
  * Returns MLRA_OK once the kernels are enqueued.
  */
 MLRA_API mlra_status mlra_decode(const mlra_dims* dims, const void* q_lat, const void* q_rope,
@@ -118,6 +120,20 @@ MLRA_API mlra_status mlra_decode(const mlra_dims* dims, const void* q_lat, const
                         const int32_t* block_table, const int32_t* seqlens, float scale,
                         float out_scale, void* out, void* workspace, size_t workspace_bytes,
                         void* stream);
+
+/*
+ * The same operation as mlra_decode, computed by a split-KV kernel on the
+ * CUDA cores (fp32 FMA) instead of the tensor cores: same arguments, same
+ * workspace, same outputs within the stated tolerance.  It covers more
+ * shapes (heads <= 64, d_c and d_r multiples of 8, branches * d_c <= 1024,
+ * any page size) at a fraction of the speed, and serves as an independent
+ * GPU statement of the kernel for cross-checks.
+ */
+MLRA_API mlra_status mlra_decode_simt(const mlra_dims* dims, const void* q_lat, const void* q_rope,
+                             const void* latent_cache, const void* rope_cache,
+                             const int32_t* block_table, const int32_t* seqlens, float scale,
+                             float out_scale, void* out, void* workspace, size_t workspace_bytes,
+                             void* stream);
 
 /*
  * Per-branch W_UV up-projection followed by the branch sum ("The Core

@@ -129,7 +129,10 @@ def decode(q_lat, q_rope, latent_cache, rope_cache, block_table, seqlens, scale,
 
 def up_proj(out_lat, w_uv, d_h, lib=None):
     """fp64 per-branch up-projection plus branch sum: y [N, H*d_h]."""
-    ol = np.ascontiguousarray(_as_input(out_lat, None)[0], dtype=np.float64)
+    ol, ol_kind = _as_input(out_lat, None)
+    if ol_kind == BF16:  # decode bf16 bit patterns to their (exact) values
+        ol = (ol.astype(np.uint32) << 16).view(np.float32)
+    ol = np.ascontiguousarray(ol, dtype=np.float64)
     w, kind = _as_input(w_uv, None)
     N, H, B, d_c = ol.shape
     if w.shape != (B, d_c, H * d_h):

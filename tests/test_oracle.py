@@ -292,3 +292,10 @@ def test_planted_mistakes_are_caught(tmp_path, name):
         except AssertionError:
             caught += 1
     assert caught >= 1, f"mutant {name} passed every pin"
+
+
+def test_up_proj_bf16_and_float64_inputs_agree(oracle_lib):
+    rng = np.random.default_rng(14)
+    out_lat = torch.from_numpy(bf16_exact((3, 2, 4, 8), rng)).to(torch.bfloat16)
+    w_uv = torch.from_numpy(bf16_exact((4, 8, 2 * 5), rng)).to(torch.bfloat16)
+    assert np.array_equal(oracle_lib.up_proj(out_lat, w_uv, 5), oracle_lib.up_proj(out_lat.double(), w_uv, 5))

@@ -42,9 +42,12 @@ def _assert_close(gpu, ref, seq_ids=None, what=""):
     return max_abs, rel
 
 
-def _run(x, **kw):
-    return b.mlra_decode(x.q_lat, x.q_rope, x.latent_cache, x.rope_cache, x.block_table, x.seqlens,
-                         x.scale, x.out_scale, **kw)
+IMPLS = {"tc": b.mlra_decode, "simt": b.mlra_decode_simt}
+
+
+def _run(x, impl="tc", **kw):
+    return IMPLS[impl](x.q_lat, x.q_rope, x.latent_cache, x.rope_cache, x.block_table, x.seqlens,
+                       x.scale, x.out_scale, **kw)
 
 
 def _oracle(oracle_lib, x, seq_ids=None):
@@ -62,9 +65,10 @@ def _score_gain(w, target_std):
 RAGGED = torch.tensor([1, 200, 777, 128, 129, 64, 1000, 255], dtype=torch.int32)
 
 
+@pytest.mark.parametrize("impl", sorted(IMPLS))
 @pytest.mark.parametrize("name", sorted(WORKLOADS))
 @pytest.mark.parametrize("peaked", [False, True])
-def test_small_cases_match_oracle(oracle_lib, name, peaked):
+def test_small_cases_match_oracle(oracle_lib, name, peaked, impl):
     """Every workload's model shape on short ragged sequences (several tiles,
     partial pages, NaN in every unused pool slot)."""
     w = WORKLOADS[name]
@@ -76,16 +80,17 @@ def test_small_cases_match_oracle(oracle_lib, name, peaked):
     gain = _score_gain(w, 4.0) if peaked else 1.0
     x = make_inputs(w, seed=3, q_gain=gain, slack_pages=5, nan_fill_unused=True,
                     seqlens=seqlens).to("cuda")
-    out = _run(x)
+    out = _run(x, impl)
     ref, status = _oracle(oracle_lib, x)
     assert status == 0
     assert torch.isfinite(out.float()).all()
-    _assert_close(out, ref, what=f"{name} peaked={peaked}")
+    _assert_close(out, ref, what=f"{name} peaked={peaked} {impl}")
 
 
-def test_tiny_workload_exact_recipe(oracle_lib):
+@pytest.mark.parametrize("impl", sorted(IMPLS))
+def test_tiny_workload_exact_recipe(oracle_lib, impl):
     x = make_inputs(WORKLOADS["tiny"]).to("cuda")
-    out = _run(x)
+    out = _run(x, impl)
     ref, status = _oracle(oracle_lib, x)
     assert status == 0
     _assert_close(out, ref, what="tiny")
@@ -108,10 +113,12 @@ def test_full_size_sampled_sequences(oracle_lib, name, samples):
     _assert_close(out, ref, seq_ids=samples, what=name)
 
 
-def test_length_one_is_bit_exact():
-    w = WORKLOADS["decode_2p9b"].with_(batch=6, seqlen=1, page_order="permuted")
+@pytest.mark.parametrize("impl", sorted(IMPLS))
+@pytest.mark.parametrize("name", ["decode_2p9b", "tiny", "mla_equal_bytes"])
+def test_length_one_is_bit_exact(impl, name):
+    w = WORKLOADS[name].with_(batch=6, seqlen=1, page_order="permuted")
     x = make_inputs(w, seed=5, q_gain=40.0, slack_pages=3, nan_fill_unused=True).to("cuda")
-    out = _run(x)
+    out = _run(x, impl)
     pages = x.block_table[:, 0].long()
     want = (x.latent_cache[pages, 0].float() * x.out_scale).to(torch.bfloat16)  # [N, B, d_c]
     assert torch.equal(out, want[:, None].expand_as(out))
@@ -131,6 +138,17 @@ def test_page_permutation_gives_identical_bits():
     out2 = b.mlra_decode(x.q_lat, x.q_rope, lat2, rope2, bt2.contiguous(), x.seqlens, x.scale,
                          x.out_scale)
     assert torch.equal(out1, out2)
+
+
+@pytest.mark.parametrize("name", ["decode_2p9b", "ragged", "mla_equal_bytes", "tp_shard"])
+def test_tensor_core_and_cuda_core_paths_agree(name):
+    """Two independent GPU statements of the kernel agree within the tolerance."""
+    w = WORKLOADS[name].with_(batch=6, seqlen=None, seqlen_range=None)
+    seqlens = torch.tensor([5000, 1, 777, 128, 4097, 2500], dtype=torch.int32)
+    x = make_inputs(w, seed=12, seqlens=seqlens, device="cuda")
+    a, c = _run(x, "tc"), _run(x, "simt")
+    ref = c.double().cpu().numpy()
+    _assert_close(a, ref, what=f"tc vs simt {name}")
 
 
 def test_repeat_calls_are_deterministic():
