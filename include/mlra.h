@@ -136,6 +136,37 @@ MLRA_API mlra_status mlra_decode_simt(const mlra_dims* dims, const void* q_lat, 
                              void* stream);
 
 /*
+ * mlra_decode for callers that cannot allocate device memory.  (An interface
+ * addition of this library; the pages describing the method have no
+ * counterpart.)  Some callers cannot call cudaMalloc or own a workspace:
+ * plugins that must not allocate from the host application's memory pools,
+ * runtimes that have handed all device memory to their own allocator, and
+ * serving loops that forbid allocation after start-up (cudaMalloc
+ * synchronises the device and can fail under memory pressure).  This variant takes no
+ * workspace: its scratch is a fixed 8 MiB array inside the library's device
+ * image, held on every GPU that loads the library until the process exits.
+ *   Arguments as mlra_decode, without workspace/workspace_bytes;
+ *   device_status  optional int32 in device memory (4-byte aligned, may be
+ *                  NULL): receives the call's device error code (0, or
+ *                  MLRA_ERR_DEVICE_*), stream-ordered after the kernels.
+ * Returns MLRA_ERR_WORKSPACE when the step needs more scratch than the
+ * 8 MiB array holds (mlra_decode_workspace_bytes(dims, 0) > 8 MiB; call
+ * mlra_decode with a workspace instead), otherwise what mlra_decode returns.
+ * It allocates and frees nothing.  All calls on a device share the array:
+ * calls that may overlap on the GPU race and corrupt each other's results,
+ * so order them on one stream.  The array keeps the last call's contents;
+ * the only part that must start at zero (the error word) starts zeroed and
+ * is cleared again at the end of every call.  The first call on each device
+ * looks up the array's address with that device current; make it before any
+ * stream capture starts.
+ */
+MLRA_API mlra_status mlra_decode_static_scratch(const mlra_dims* dims, const void* q_lat,
+                             const void* q_rope, const void* latent_cache,
+                             const void* rope_cache, const int32_t* block_table,
+                             const int32_t* seqlens, float scale, float out_scale, void* out,
+                             int32_t* device_status, void* stream);
+
+/*
  * Per-branch W_UV up-projection followed by the branch sum ("The Core
  * Insight" section: each branch is up-projected by its own matrix and the
  * branch outputs are summed at the end):
