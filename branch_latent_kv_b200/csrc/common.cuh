@@ -22,7 +22,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 // Workspace layout (byte offsets, each region 256-byte aligned):
 //   [0, 256)        int32 error word (first device-side error code, else 0)
 //   lse partials    fp32 [slots][branches][heads]      (log2 domain)
-//   o partials      fp32 [slots][branches][heads][d_c] (normalised per split)
+//   o partials      fp32 [slots][branches][d_c][16]    (normalised per split;
+//                   heads innermost, padded to 16: one 64-byte row per column)
 // slots = num_ctas + batch: the partial of CTA c for sequence n lives in slot
 // c + n (unique because CTA ranges are contiguous and ordered).
 // ---------------------------------------------------------------------------
@@ -40,9 +41,13 @@ __host__ __device__ inline WorkspaceLayout workspace_layout(int batch, int heads
     w.err_off = 0;
     w.lse_off = 256;
     w.o_off = align256(w.lse_off + sizeof(float) * (size_t)w.slots * branches * heads);
-    w.total = align256(w.o_off + sizeof(float) * (size_t)w.slots * branches * heads * d_c);
+    const size_t hp = heads <= 16 ? 16 : (size_t)heads;  // heads padded to 16 (more for the CUDA-core kernel)
+    w.total = align256(w.o_off + sizeof(float) * (size_t)w.slots * branches * d_c * hp);
     return w;
 }
+
+// Heads per partial row: 16 (or H when H > 16).
+__host__ __device__ inline int partial_heads(int heads) { return heads <= 16 ? 16 : heads; }
 
 // Marker stored in a partial's lse when the split met a bad block-table entry.
 __device__ __forceinline__ float bad_split_marker() { return __int_as_float(0x7f800000); }  // +inf

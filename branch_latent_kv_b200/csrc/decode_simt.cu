@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
             for (int e = tid; e < H * W; e += kThreads) {
                 const int h = e / W, rem = e % W, b = rem / d_c, k = rem % d_c;
                 const float v = bad ? 0.f : o_s[e] / l_s[h * B + b];
-                a.o_part[((slot * B + b) * H + h) * d_c + k] = v;
+                a.o_part[((slot * B + b) * d_c + k) * partial_heads(H) + h] = v;
             }
             for (int hb = tid; hb < HB; hb += kThreads) {
                 const int h = hb / B, b = hb % B;

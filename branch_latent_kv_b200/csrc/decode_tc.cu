@@ -47,7 +47,6 @@ using namespace sm100;
 constexpr int kHP = 16;             // heads padded to the MMA N
 constexpr int kT = kTileTokens;     // tokens per tile = MMA M
 constexpr int kThreads = 192;
-constexpr int kTmemCols = 128;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kSmemLimit = 232448;  // max dynamic shared memory per CTA on sm_100
 
@@ -80,16 +79,19 @@ struct Cfg {
     static constexpr int OFF_P = OFF_QR + QR_SPAN;
     static constexpr int OFF_MISC = OFF_P + 2 * P_BYTES;
     static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
-    // TMEM columns: O blocks first, then two S slots
+    // TMEM columns: O blocks first, then two S slots, then two slots of the
+    // RoPE score shared by all branches of a tile
     static constexpr int O_BLOCKS = NSTEP * PPS * G;
     static constexpr int S_COL0 = O_BLOCKS * kHP;
     static constexpr int S_SLOT_COLS = G * kHP;
+    static constexpr int R_COL0 = S_COL0 + 2 * S_SLOT_COLS;
+    static constexpr int TMEM_COLS = R_COL0 + 2 * kHP <= 128 ? 128 : 256;
     static_assert(NB % G == 0, "branches must fill whole steps");
     static_assert(NSTAGE >= PPS, "a step's pairs must fit the stage ring");
     // The score MMA of step s+1 is issued before the output MMA of step s
     // (overlapping the softmax of s) only when both steps' pairs fit the ring.
     static constexpr bool OVERLAP = 2 * PPS <= NSTAGE;
-    static_assert(S_COL0 + 2 * S_SLOT_COLS <= kTmemCols, "TMEM budget");
+    static_assert(R_COL0 + 2 * kHP <= TMEM_COLS, "TMEM budget");
     static_assert(SMEM_BYTES <= kSmemLimit, "shared-memory budget");
     static_assert(OFF_QR + QR_BYTES <= OFF_P && OFF_Q + Q_BYTES <= OFF_QR && OFF_P + 2 * P_BYTES <= OFF_MISC,
                   "shared-memory regions must not overlap");
@@ -115,6 +117,7 @@ struct Misc {
     float red_max[4][2 * kHP];
     float red_sum[4][4 * kHP];
     alignas(16) float m_run[8 * kHP];  // running max per (branch, head), base-2 logits; read as float4
+    float inv_l[8 * kHP];              // 1 / softmax denominator per (branch, head), epilogue only
 };
 
 static_assert(offsetof(Misc<5>, m_run) % 16 == 0 && offsetof(Misc<4>, m_run) % 16 == 0 &&
@@ -124,6 +127,65 @@ struct Maps {
     CUtensorMap lat;
     CUtensorMap rope;
 };
+
+// 2^x on the special-function unit (ex2.approx, flush-to-zero: results below
+// 2^-126 become 0, which only affects probabilities that are negligible).
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Max over the 32 lanes of a warp of each of 16 values, reduce-scattered:
+// the result for column c ends up in lanes 2c and 2c+1.  16 shuffles.
+__device__ __forceinline__ float warp_colmax16(const float (&v)[16], int lane) {
+    float a8[8], a4[4], a2[2];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {  // lanes with bit 4 keep columns 8..15
+        const bool hi = lane & 16;
+        const float keep = hi ? v[i + 8] : v[i], send = hi ? v[i] : v[i + 8];
+        a8[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 16));
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const bool hi = lane & 8;
+        const float keep = hi ? a8[i + 4] : a8[i], send = hi ? a8[i] : a8[i + 4];
+        a4[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const bool hi = lane & 4;
+        const float keep = hi ? a4[i + 2] : a4[i], send = hi ? a4[i] : a4[i + 2];
+        a2[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+    }
+    const bool hi = lane & 2;
+    const float keep = hi ? a2[1] : a2[0], send = hi ? a2[0] : a2[1];
+    const float a1 = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
+    return fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
+}
+
+// Sum over the 32 lanes of a warp of each of N values (N = 16, 32, 64, 128),
+// reduce-scattered: afterwards, for N >= 32, lane L holds in v[r]
+// (r < N/32) the warp total of value N/32*L + r; for N = 16, lanes 2c and
+// 2c+1 hold in v[0] the total of value c.  N - 1 + (N < 32) shuffles.
+template <int LIVE, int O, int N>
+__device__ __forceinline__ void warp_sum_scatter(float (&v)[N], int lane) {
+    if constexpr (O >= 1) {
+        if constexpr (LIVE >= 2) {
+            constexpr int H = LIVE / 2;
+#pragma unroll
+            for (int i = 0; i < H; ++i) {
+                const bool hi = lane & O;
+                const float keep = hi ? v[i + H] : v[i], send = hi ? v[i] : v[i + H];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+            }
+            warp_sum_scatter<H, O / 2, N>(v, lane);
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], O);
+            warp_sum_scatter<1, O / 2, N>(v, lane);
+        }
+    }
+}
 
 template <int DR>
 __device__ __forceinline__ uint64_t rope_desc(uint32_t addr) {
@@ -192,13 +254,14 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
         prefetch_tensormap(&maps.rope);
     }
     if (warp == 1) {
-        tmem_alloc(&misc.tmem_base, kTmemCols);
+        tmem_alloc(&misc.tmem_base, C::TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
 
+    launch_dependents();  // the combine kernel may be scheduled as CTAs retire
     const int total = misc.plan[0], chunk = misc.plan[1];
     const int g0 = blockIdx.x * chunk, g1 = min(g0 + chunk, total);
     const uint32_t tmem = misc.tmem_base;
@@ -284,113 +347,140 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
             }
         } else if (warp == 1) {
             // ------------------------------------------------------------ MMA issuer
-            if (lane == 0) {
+            // (the whole warp walks the schedule; the elected lane issues)
+            {
                 constexpr uint32_t IDESC_S = idesc_bf16_f32(128, kHP, false, false);
                 constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, kHP, true, true);
                 const uint32_t sm_base = smem_u32(sm);
+                // Descriptor bases; every operand below is a base plus a byte
+                // offset >> 4 (the start-address field never overflows: all
+                // addresses are below 256 KB).
+                const uint64_t dA_s = smem_desc(sm_base + C::OFF_PAIR, 16, 1024, kLayoutSw128);       // K-major
+                const uint64_t dA_pv = smem_desc(sm_base + C::OFF_PAIR, C::CHUNK_BYTES, 1024, kLayoutSw128);  // MN-major
+                const uint64_t dQ = smem_desc(sm_base + C::OFF_Q, 16, 1024, kLayoutSw128);
+                const uint64_t dQR = rope_desc<DR>(sm_base + C::OFF_QR);
+                const uint64_t dR = rope_desc<DR>(sm_base + C::OFF_ROPE);
+                const uint64_t dP = smem_desc(sm_base + C::OFF_P, 128, 2048, kLayoutNone);
                 int n = misc.plan[2], first = misc.plan[3];
                 int L, tiles, tb, te;
-                uint32_t gs = 0, pc = 0, tc = 0, sc = 0;
+                uint32_t gs = 0, tc = 0, sc = 0;
+                uint32_t stage = 0, phase = 0;  // ring position of the next pair to consume
                 bool ok = true;
                 bool have_prev = false;
-                uint32_t prev_gs = 0, prev_pc = 0;
+                uint32_t prev_gs = 0, prev_stage = 0;
                 int prev_st = 0;
                 bool prev_first = false;
 
-                auto issue_pv = [&](uint32_t pgs, int pst, uint32_t ppc, bool pfirst) -> bool {
-                    if (!mbar_wait(&misc.p_full[pgs & 1], (pgs >> 1) & 1)) return false;
+                auto issue_pv = [&](uint32_t pgs, int pst, uint32_t pstage, bool pfirst) -> bool {
+                    if (!mbar_wait_warp(&misc.p_full[pgs & 1], (pgs >> 1) & 1)) return false;
                     tc_fence_after();
-                    const uint32_t p_base = sm_base + C::OFF_P + (pgs & 1) * C::P_BYTES;
+                    const uint64_t b0 = dP + ((pgs & 1) * C::P_BYTES >> 4);
 #pragma unroll
                     for (int p = 0; p < C::PPS; ++p) {
-                        const uint32_t a_base = sm_base + C::OFF_PAIR + ((ppc + p) % C::NSTAGE) * C::PAIR_BYTES;
+                        uint32_t sp = pstage + p;
+                        if (sp >= (uint32_t)C::NSTAGE) sp -= C::NSTAGE;
+                        const uint64_t a0 = dA_pv + ((sp * C::PAIR_BYTES) >> 4);
 #pragma unroll
                         for (int g = 0; g < C::G; ++g) {
                             const uint32_t d = tmem + ((pst * C::PPS + p) * C::G + g) * kHP;
 #pragma unroll
-                            for (int kt = 0; kt < kT / 16; ++kt) {
-                                const uint64_t ad = smem_desc(a_base + kt * 2048, C::CHUNK_BYTES, 1024, kLayoutSw128);
-                                const uint64_t bd = smem_desc(p_base + g * C::P_BRANCH_BYTES + kt * 256, 128,
-                                                              2048, kLayoutNone);
-                                mma_bf16(d, ad, bd, IDESC_PV, (pfirst && kt == 0) ? 0u : 1u);
-                            }
+                            for (int kt = 0; kt < kT / 16; ++kt)
+                                if (elect_one())
+                                    mma_bf16(d, a0 + (kt * 2048 >> 4), b0 + ((g * C::P_BRANCH_BYTES + kt * 256) >> 4),
+                                             IDESC_PV, (pfirst && kt == 0) ? 0u : 1u);
                         }
                     }
 #pragma unroll
-                    for (int p = 0; p < C::PPS; ++p) mma_commit(&misc.pair_empty[(ppc + p) % C::NSTAGE]);
-                    mma_commit(&misc.o_done);
+                    for (int p = 0; p < C::PPS; ++p) {
+                        uint32_t sp = pstage + p;
+                        if (sp >= (uint32_t)C::NSTAGE) sp -= C::NSTAGE;
+                        if (elect_one()) mma_commit(&misc.pair_empty[sp]);
+                    }
+                    if (elect_one()) mma_commit(&misc.o_done);
+                    __syncwarp();
                     return true;
                 };
 
                 while (ok && next_segment(a, n, first, g0, g1, L, tiles, tb, te)) {
-                    ok = mbar_wait(&misc.q_full, sc & 1);
+                    ok = mbar_wait_warp(&misc.q_full, sc & 1);
                     tc_fence_after();
                     for (int j = tb; j < te && ok; ++j) {
                         const int rslot = tc & 1;
-                        ok = mbar_wait(&misc.rope_full[rslot], (tc >> 1) & 1);
-                        const uint32_t rope_base = sm_base + C::OFF_ROPE + rslot * C::ROPE_BYTES;
+                        ok = mbar_wait_warp(&misc.rope_full[rslot], (tc >> 1) & 1);
+                        const uint64_t dRs = dR + ((rslot * C::ROPE_BYTES) >> 4);
 #pragma unroll 1
                         for (int st = 0; st < C::NSTEP && ok; ++st) {
-                            for (int p = 0; p < C::PPS && ok; ++p)
-                                ok = mbar_wait(&misc.pair_full[(pc + p) % C::NSTAGE], ((pc + p) / C::NSTAGE) & 1);
+                            const uint32_t stage0 = stage;
+                            for (int p = 0; p < C::PPS && ok; ++p) {
+                                ok = mbar_wait_warp(&misc.pair_full[stage], phase);
+                                if (++stage == (uint32_t)C::NSTAGE) {
+                                    stage = 0;
+                                    phase ^= 1;
+                                }
+                            }
                             if (!ok) break;
                             tc_fence_after();
-#pragma unroll
-                            for (int g = 0; g < C::G; ++g) {
-                                const int b = st * C::G + g;
-                                const uint32_t d = tmem + C::S_COL0 + (gs & 1) * C::S_SLOT_COLS + g * kHP;
-                                uint32_t acc = 0;
-#pragma unroll
-                                for (int c = 0; c < DC / 64; ++c) {
-                                    const int gc = b * (DC / 64) + c;          // chunk of the token row
-                                    const int pp = gc / 2 - st * C::PPS;        // pair within this step
-                                    const uint32_t a_base = sm_base + C::OFF_PAIR +
-                                                            ((pc + pp) % C::NSTAGE) * C::PAIR_BYTES +
-                                                            (gc & 1) * C::CHUNK_BYTES;
-                                    const uint32_t q_base = sm_base + C::OFF_Q + gc * C::Q_CHUNK_BYTES;
-#pragma unroll
-                                    for (int kk = 0; kk < 4; ++kk) {
-                                        mma_bf16(d, smem_desc(a_base + kk * 32, 16, 1024, kLayoutSw128),
-                                                 smem_desc(q_base + kk * 32, 16, 1024, kLayoutSw128), IDESC_S, acc);
-                                        acc = 1;
-                                    }
-                                }
+                            if (st == 0) {
+                                // RoPE score of the tile, shared by every branch
+                                const uint32_t dRt = tmem + C::R_COL0 + (tc & 1) * kHP;
 #pragma unroll
                                 for (int kk = 0; kk < DR / 16; ++kk)
-                                    mma_bf16(d, rope_desc<DR>(rope_base + kk * 32),
-                                             rope_desc<DR>(sm_base + C::OFF_QR + kk * 32), IDESC_S, 1u);
+                                    if (elect_one()) mma_bf16(dRt, dRs + kk * 2, dQR + kk * 2, IDESC_S, kk ? 1u : 0u);
+                                if (elect_one()) mma_commit(&misc.rope_empty[rslot]);
+                                __syncwarp();
                             }
-                            mma_commit(&misc.s_full[gs & 1]);
-                            if (st == C::NSTEP - 1) mma_commit(&misc.rope_empty[rslot]);
+                            const uint32_t dS = tmem + C::S_COL0 + (gs & 1) * C::S_SLOT_COLS;
+                            // this step's branches start at chunk st*G*(DC/64) of the token row
+                            const uint64_t dQs = dQ + ((st * C::G * (DC / 64) * C::Q_CHUNK_BYTES) >> 4);
+#pragma unroll
+                            for (int g = 0; g < C::G; ++g) {
+#pragma unroll
+                                for (int c = 0; c < DC / 64; ++c) {
+                                    // chunk (g*(DC/64) + c) of this step: pair pp, half hf
+                                    const int lc = g * (DC / 64) + c;
+                                    const int pp = lc / 2, hf = lc % 2;
+                                    uint32_t sp = stage0 + pp;
+                                    if (sp >= (uint32_t)C::NSTAGE) sp -= C::NSTAGE;
+                                    const uint64_t a0 = dA_s + ((sp * C::PAIR_BYTES + hf * C::CHUNK_BYTES) >> 4);
+                                    const uint64_t q0 = dQs + ((lc * C::Q_CHUNK_BYTES) >> 4);
+#pragma unroll
+                                    for (int kk = 0; kk < 4; ++kk)
+                                        if (elect_one())
+                                            mma_bf16(dS + g * kHP, a0 + kk * 2, q0 + kk * 2, IDESC_S, (c | kk) ? 1u : 0u);
+                                }
+                            }
+                            if (elect_one()) mma_commit(&misc.s_full[gs & 1]);
+                            __syncwarp();
                             if (C::OVERLAP) {
-                                if (have_prev) ok = issue_pv(prev_gs, prev_st, prev_pc, prev_first);
+                                if (have_prev) ok = issue_pv(prev_gs, prev_st, prev_stage, prev_first);
                                 have_prev = true;
                                 prev_gs = gs;
                                 prev_st = st;
-                                prev_pc = pc;
+                                prev_stage = stage0;
                                 prev_first = (j == tb);
                             } else {
-                                ok = issue_pv(gs, st, pc, j == tb);
+                                ok = issue_pv(gs, st, stage0, j == tb);
                             }
-                            pc += C::PPS;
                             ++gs;
                         }
                         ++tc;
-                        if (*abort_flag) ok = false;
+                        if (__shfl_sync(0xffffffffu, *abort_flag, 0)) ok = false;
                     }
-                    if (ok && have_prev) ok = issue_pv(prev_gs, prev_st, prev_pc, prev_first);
+                    if (ok && have_prev) ok = issue_pv(prev_gs, prev_st, prev_stage, prev_first);
                     have_prev = false;
-                    if (ok) mma_commit(&misc.seg_done);
+                    if (ok && elect_one()) mma_commit(&misc.seg_done);
+                    __syncwarp();
                     ++sc;
                     first += tiles;
                     ++n;
                 }
-                if (!ok) {
+                if (!ok && lane == 0) {
                     record_error(a.err, MLRA_ERR_DEVICE_TIMEOUT);
                     *abort_flag = 1;
                 }
                 // drain: every MMA issued above completes before TMEM is freed
-                mma_commit(&misc.drain);
+                if (elect_one()) mma_commit(&misc.drain);
+                __syncwarp();
                 mbar_wait(&misc.drain, 0, 200000000ull);
             }
             __syncwarp();
@@ -403,8 +493,11 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
             const int H = a.heads;
             int n = misc.plan[2], first = misc.plan[3];
             int L, tiles, tb, te;
-            uint32_t gs = 0, sc = 0;
-            float l[NB][kHP];  // this thread's share of the softmax denominators
+            uint32_t gs = 0, sc = 0, tcnt = 0;  // steps, ranges, tiles so far
+            // This thread's share of the softmax denominators, one row per
+            // branch.  The step loop is not unrolled: after each step the rows
+            // rotate by G so that the current step's branches are rows 0..G-1.
+            float l[NB][kHP];
             bool dead = false;
 
             while (!dead && next_segment(a, n, first, g0, g1, L, tiles, tb, te)) {
@@ -439,7 +532,8 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                         bad |= (v < 0 || v >= a.num_pages);
                     }
                 }
-                bad = named_bar_or<1, 128>(bad);
+                if (stid < NB * kHP) misc.m_run[stid] = -INFINITY;
+                bad = named_bar_or<1, 128>(bad);  // also publishes m_run
                 fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
@@ -448,27 +542,28 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                 for (int b = 0; b < NB; ++b)
 #pragma unroll
                     for (int i = 0; i < kHP; ++i) l[b][i] = 0.f;
-                if (stid < NB * kHP) misc.m_run[stid] = -INFINITY;
-                named_bar_sync<1, 128>();
 
                 for (int j = tb; j < te && !dead; ++j) {
                     const int valid = min(kT, L - j * kT);
                     const bool masked = row >= valid;
-#pragma unroll
+                    float r[kHP];  // this token's RoPE score per head, shared by the tile's branches
+#pragma unroll 1
                     for (int st = 0; st < C::NSTEP; ++st) {
                         const bool ok = mbar_wait(&misc.s_full[gs & 1], (gs >> 1) & 1);
                         tc_fence_after();
                         float x[C::G][kHP];
+                        if (st == 0) tmem_ld16(tmem + lane_off + C::R_COL0 + (tcnt & 1) * kHP, r);
 #pragma unroll
                         for (int g = 0; g < C::G; ++g)
                             tmem_ld16(tmem + lane_off + C::S_COL0 + (gs & 1) * C::S_SLOT_COLS + g * kHP, x[g]);
                         tmem_wait_ld();
+                        float* m_step = &misc.m_run[st * C::G * kHP];
                         float m[C::G][kHP];
 #pragma unroll
                         for (int g = 0; g < C::G; ++g)
 #pragma unroll
                             for (int i = 0; i < kHP; i += 4) {
-                                const float4 v = *reinterpret_cast<const float4*>(&misc.m_run[(st * C::G + g) * kHP + i]);
+                                const float4 v = *reinterpret_cast<const float4*>(m_step + g * kHP + i);
                                 m[g][i] = v.x;
                                 m[g][i + 1] = v.y;
                                 m[g][i + 2] = v.z;
@@ -476,50 +571,44 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                             }
                         bool need = false;
 #pragma unroll
-                        for (int g = 0; g < C::G; ++g) {
+                        for (int g = 0; g < C::G; ++g)
 #pragma unroll
                             for (int i = 0; i < kHP; ++i) {
-                                x[g][i] = masked ? -INFINITY : x[g][i] * a.scale_log2;
+                                x[g][i] = masked ? -INFINITY : (x[g][i] + r[i]) * a.scale_log2;
                                 need |= x[g][i] > m[g][i] + kRescaleLog2;
                             }
-                        }
                         if (named_bar_or<1, 128>(need || !ok)) {
                             if (named_bar_or<1, 128>(!ok)) {
                                 dead = true;
                                 break;
                             }
-                            // exact column max over the tile's 128 tokens
+                            // exact column max over the tile's 128 tokens: a warp
+                            // reduce-scatter leaves column (lane >> 1) in each lane
 #pragma unroll
-                            for (int g = 0; g < C::G; ++g)
-#pragma unroll
-                                for (int i = 0; i < kHP; ++i) {
-                                    float v = x[g][i];
-#pragma unroll
-                                    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-                                    if (lane == 0) misc.red_max[quad][g * kHP + i] = v;
-                                }
+                            for (int g = 0; g < C::G; ++g) {
+                                const float v = warp_colmax16(x[g], lane);
+                                if ((lane & 1) == 0) misc.red_max[quad][g * kHP + (lane >> 1)] = v;
+                            }
                             named_bar_sync<1, 128>();
                             float alpha[C::G][kHP];
 #pragma unroll
-                            for (int g = 0; g < C::G; ++g) {
-                                const int b = st * C::G + g;
+                            for (int g = 0; g < C::G; ++g)
 #pragma unroll
                                 for (int i = 0; i < kHP; ++i) {
                                     const float tmax = fmaxf(fmaxf(misc.red_max[0][g * kHP + i], misc.red_max[1][g * kHP + i]),
                                                              fmaxf(misc.red_max[2][g * kHP + i], misc.red_max[3][g * kHP + i]));
                                     const float mnew = fmaxf(m[g][i], tmax);
-                                    alpha[g][i] = exp2f(m[g][i] - mnew);
+                                    alpha[g][i] = fast_exp2(m[g][i] - mnew);
                                     m[g][i] = mnew;
-                                    l[b][i] *= alpha[g][i];
+                                    l[g][i] *= alpha[g][i];
                                 }
-                            }
                             // every thread read the old maxima before the barrier above; the
                             // barrier below publishes the new ones (and frees red_max)
                             if (stid == 0) {
 #pragma unroll
                                 for (int g = 0; g < C::G; ++g)
 #pragma unroll
-                                    for (int i = 0; i < kHP; ++i) misc.m_run[(st * C::G + g) * kHP + i] = m[g][i];
+                                    for (int i = 0; i < kHP; ++i) m_step[g * kHP + i] = m[g][i];
                             }
                             named_bar_sync<1, 128>();
                             if (j > tb) {
@@ -550,14 +639,13 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                         uint8_t* p_slot = sm + C::OFF_P + (gs & 1) * C::P_BYTES;
 #pragma unroll
                         for (int g = 0; g < C::G; ++g) {
-                            const int b = st * C::G + g;
                             uint32_t packed[kHP / 2];
 #pragma unroll
                             for (int i = 0; i < kHP; i += 2) {
-                                const float p0 = exp2f(x[g][i] - m[g][i]);
-                                const float p1 = exp2f(x[g][i + 1] - m[g][i + 1]);
-                                l[b][i] += p0;
-                                l[b][i + 1] += p1;
+                                const float p0 = fast_exp2(x[g][i] - m[g][i]);
+                                const float p1 = fast_exp2(x[g][i + 1] - m[g][i + 1]);
+                                l[g][i] += p0;
+                                l[g][i + 1] += p1;
                                 __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
                                 packed[i / 2] = *reinterpret_cast<uint32_t*>(&pr);
                             }
@@ -583,8 +671,22 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&misc.p_full[gs & 1]);
+                        // rotate the denominator rows: the next step's branches first
+#pragma unroll
+                        for (int r = 0; r < C::G; ++r) {
+                            float t[kHP];
+#pragma unroll
+                            for (int i = 0; i < kHP; ++i) t[i] = l[0][i];
+#pragma unroll
+                            for (int b = 0; b + 1 < NB; ++b)
+#pragma unroll
+                                for (int i = 0; i < kHP; ++i) l[b][i] = l[b + 1][i];
+#pragma unroll
+                            for (int i = 0; i < kHP; ++i) l[NB - 1][i] = t[i];
+                        }
                         ++gs;
                     }
+                    ++tcnt;
                 }
                 if (dead) break;
 
@@ -597,71 +699,68 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                     break;
                 }
                 tc_fence_after();
-                // row sums over all tokens of the range
-#pragma unroll
-                for (int b = 0; b < NB; ++b)
-#pragma unroll
-                    for (int i = 0; i < kHP; ++i) {
-                        float v = l[b][i];
-#pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                        l[b][i] = v;
-                    }
-                // reduce across the four warps, NB*16 values at a time in chunks of 64
-#pragma unroll
-                for (int b0 = 0; b0 < NB; b0 += 4) {
-                    if (lane == 0) {
-#pragma unroll
-                        for (int b = b0; b < b0 + 4 && b < NB; ++b)
-#pragma unroll
-                            for (int i = 0; i < kHP; ++i) misc.red_sum[quad][(b - b0) * kHP + i] = l[b][i];
-                    }
-                    named_bar_sync<1, 128>();
-#pragma unroll
-                    for (int b = b0; b < b0 + 4 && b < NB; ++b)
-#pragma unroll
-                        for (int i = 0; i < kHP; ++i) {
-                            const int k = (b - b0) * kHP + i;
-                            l[b][i] = misc.red_sum[0][k] + misc.red_sum[1][k] + misc.red_sum[2][k] + misc.red_sum[3][k];
-                        }
-                    named_bar_sync<1, 128>();
-                }
-                const int first_cta = first / chunk, last_cta = (first + tiles - 1) / chunk;
-                const bool single = first_cta == last_cta;
-                const size_t slot = (size_t)blockIdx.x + n;
-#pragma unroll
-                for (int st = 0; st < C::NSTEP; ++st)
-#pragma unroll
-                    for (int p = 0; p < C::PPS; ++p)
-#pragma unroll
-                        for (int g = 0; g < C::G; ++g) {
-                            const int colw = (st * C::PPS + p) * 128 + row;  // latent column of the token row
-                            const int b = colw / DC, k = colw % DC;
-                            float o[kHP];
-                            tmem_ld16(tmem + lane_off + ((st * C::PPS + p) * C::G + g) * kHP, o);
-                            tmem_wait_ld();
-                            if (b != st * C::G + g) continue;  // rows of the other branch of a pair
-#pragma unroll
-                            for (int i = 0; i < kHP; ++i) {
-                                if (i >= H) break;
-                                const float v = bad ? 0.f : o[i] / l[st * C::G + g][i];
-                                if (single)
-                                    a.out[(((size_t)n * H + i) * NB + b) * DC + k] = to_bf16(v * a.out_scale);
-                                else
-                                    a.o_part[((slot * NB + b) * H + i) * DC + k] = v;
-                            }
-                        }
-                if (!single) {
+                // denominators: warp reduce-scatter, then the four warps through shared memory
+                {
+                    constexpr int NV = NB * kHP;
+                    float f[NV];
 #pragma unroll
                     for (int b = 0; b < NB; ++b)
 #pragma unroll
+                        for (int i = 0; i < kHP; ++i) f[b * kHP + i] = l[b][i];
+                    warp_sum_scatter<NV, 16, NV>(f, lane);
+                    if constexpr (NV >= 32) {
+#pragma unroll
+                        for (int r = 0; r < NV / 32; ++r) misc.red_sum[quad][(NV / 32) * lane + r] = f[r];
+                    } else {
+                        if ((lane & 1) == 0) misc.red_sum[quad][lane >> 1] = f[0];
+                    }
+                }
+                named_bar_sync<1, 128>();
+                const int first_cta = first / chunk, last_cta = (first + tiles - 1) / chunk;
+                const bool single = first_cta == last_cta;
+                const size_t slot = (size_t)blockIdx.x + n;
+                if (stid < NB * kHP) {
+                    const float lt = misc.red_sum[0][stid] + misc.red_sum[1][stid] + misc.red_sum[2][stid] +
+                                     misc.red_sum[3][stid];
+                    misc.inv_l[stid] = 1.0f / lt;
+                    const int b = stid / kHP, i = stid % kHP;
+                    if (!single && i < H)
+                        a.lse_part[(slot * NB + b) * H + i] = bad ? bad_split_marker() : misc.m_run[stid] + __log2f(lt);
+                }
+                named_bar_sync<1, 128>();
+                // outputs: a block of TMEM holds 128 latent rows x 16 heads of one
+                // branch (or two branches of 64 rows when DC = 64)
+                constexpr int WIDTH = DC >= 128 ? 128 : DC;  // valid rows per block
+#pragma unroll 1
+                for (int blk = 0; blk < C::O_BLOCKS; ++blk) {
+                    const int g = blk % C::G, sp = blk / C::G;       // sp = st * PPS + p
+                    const int st = sp / C::PPS;
+                    const int b = st * C::G + g;
+                    const int row0 = C::G == 1 ? 0 : g * WIDTH;      // first valid row of the block
+                    const int k = (sp * 128 + row0) % DC + (row - row0);  // latent column of this row
+                    const bool mine = row >= row0 && row < row0 + WIDTH;
+                    float o[kHP];
+                    tmem_ld16(tmem + lane_off + blk * kHP, o);
+                    tmem_wait_ld();
+                    if (!mine) continue;
+                    const float* inv = &misc.inv_l[b * kHP];
+#pragma unroll
+                    for (int i = 0; i < kHP; ++i) o[i] = bad ? 0.f : o[i] * inv[i];
+                    if (single) {
+                        __nv_bfloat16* dst = a.out + ((size_t)n * H * NB + b) * DC + k;
+#pragma unroll
                         for (int i = 0; i < kHP; ++i)
-                            if (stid == b * kHP + i && i < H)
-                                a.lse_part[(slot * NB + b) * H + i] =
-                                    bad ? bad_split_marker() : misc.m_run[b * kHP + i] + log2f(l[b][i]);
+                            if (i < H) dst[(size_t)i * NB * DC] = to_bf16(o[i] * a.out_scale);
+                    } else {
+                        // partial layout [slot][branch][k][16 heads]: 64 contiguous bytes per row
+                        float4* dst = reinterpret_cast<float4*>(a.o_part + (((slot * NB + b) * DC + k) * kHP));
+#pragma unroll
+                        for (int i = 0; i < kHP; i += 4) dst[i / 4] = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+                    }
                 }
                 if (bad && stid == 0) record_error(a.err, MLRA_ERR_DEVICE_BAD_INDEX);
                 tc_fence_before();
+                named_bar_sync<1, 128>();  // inv_l and red_sum are reused by the next range
                 ++sc;
                 first += tiles;
                 ++n;
@@ -676,7 +775,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+    if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 // ------------------------------------------------------------------ host side

@@ -1,45 +1,188 @@
-// up_proj.cu -- per-branch W_UV up-projection and branch sum.
+// up_proj.cu -- per-branch W_UV up-projection and branch sum on tcgen05.
 //
 //   y[n, h*d_h + j] = sum_b sum_k out_lat[n,h,b,k] * w_uv[b][k][h*d_h + j]
 //
 // ("The Core Insight" section of the wispaper.ai MLRA blog page: every
 // branch is up-projected by its own matrix and the branch outputs are summed
-// at the end.)  The branch sum is the K reduction over K = branches * d_c.
-// One CTA per (head, group of 8 sequences); thread j owns output column j,
-// so the W_UV reads of a warp are contiguous.
+// at the end.)  The branch sum is the K reduction over K = branches * d_c:
+// for head h the product is one GEMM of W_h^T [d_h x K] by X_h^T [K x N].
+//
+// A cluster of KS CTAs per (head, tile of up to 64 sequences) splits K; each
+// CTA multiplies its K range, swap-AB so that the 128 output columns of a
+// head are the MMA's M:
+//   D[j, n] = sum_K W[K][h*d_h + j] * X[n][h][K]
+//   A = W slice, MN-major (j contiguous), 128-byte swizzle, two 64-column boxes
+//   B = X slice, K-major (K contiguous), 128-byte swizzle, rows past the
+//       batch are zero-filled by TMA
+// Every 64-wide K chunk of a CTA's range is loaded at once, each on its own
+// mbarrier, so the MMAs start as chunks land.  The KS fp32 partial products
+// are summed through distributed shared memory: each CTA stages its
+// [128 x nt] partial, then CTA r of the cluster adds up columns
+// [r*nt/KS, (r+1)*nt/KS) from all KS CTAs and writes them as bf16.
+// Rows j >= d_h (d_h = 64) are computed from neighbouring columns or TMA
+// zero fill and discarded.
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace mlra {
 namespace {
 
-constexpr int kSeqPerCta = 8;
+using namespace sm100;
 
-__global__ void up_proj_simt_kernel(int batch, int heads, int K, int d_h,
-                                    const __nv_bfloat16* __restrict__ out_lat,
-                                    const __nv_bfloat16* __restrict__ w_uv,
-                                    __nv_bfloat16* __restrict__ y) {
-    extern __shared__ float ol[];  // [kSeqPerCta][K]
-    const int h = blockIdx.x, n0 = blockIdx.y * kSeqPerCta, j = threadIdx.x;
-    for (int i = threadIdx.x; i < kSeqPerCta * K; i += blockDim.x) {
-        const int nn = i / K, kk = i % K, n = n0 + nn;
-        ol[i] = n < batch ? __bfloat162float(out_lat[((size_t)n * heads + h) * K + kk]) : 0.f;
+constexpr int kThreads = 128;
+constexpr int kMaxChunks = 8;      // K <= 512
+constexpr int kMaxNT = 64;         // sequences per CTA
+constexpr int kWChunkBytes = 2 * 64 * 128;  // two 64-column boxes of 64 K rows: 16 KB
+
+struct UpMaps {
+    CUtensorMap w;  // w_uv as [K rows][H*d_h columns]
+    CUtensorMap x;  // out_lat as [N rows][H*K columns]
+};
+
+struct UpSmem {
+    uint64_t full[kMaxChunks];
+    uint64_t mma_done;
+    uint32_t tmem_base;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+up_proj_tc_kernel(const __grid_constant__ UpMaps maps, int batch, int heads, int K, int d_h, int nt, int ks,
+                  __nv_bfloat16* __restrict__ y) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int cpc = K / 64 / ks;                 // K chunks of this CTA
+    const int x_chunk_bytes = nt * 128;
+    uint8_t* w_s = sm;                           // cpc x 16 KB
+    uint8_t* x_s = sm + cpc * kWChunkBytes;      // cpc x nt*128 B
+    UpSmem& ms = *reinterpret_cast<UpSmem*>(x_s + cpc * x_chunk_bytes);
+    float* part = reinterpret_cast<float*>(sm);  // [128][nt] fp32 partial, reuses the operand buffers
+    const uint32_t rank = cluster_ctarank();
+    const int h = blockIdx.x / ks, n0 = blockIdx.y * nt;
+    const int c_first = (int)rank * cpc;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t tmem_cols = nt <= 32 ? 32 : 64;
+
+    if (threadIdx.x == 0) {
+        for (int c = 0; c < cpc; ++c) mbar_init(&ms.full[c], 1);
+        mbar_init(&ms.mma_done, 1);
+        fence_barrier_init();
     }
+    if (warp == 1) {
+        tmem_alloc(&ms.tmem_base, tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
-    float acc[kSeqPerCta];
-#pragma unroll
-    for (int nn = 0; nn < kSeqPerCta; ++nn) acc[nn] = 0.f;
-    const size_t width = (size_t)heads * d_h;
-    for (int kk = 0; kk < K; ++kk) {
-        const float w = __bfloat162float(w_uv[kk * width + (size_t)h * d_h + j]);
-#pragma unroll
-        for (int nn = 0; nn < kSeqPerCta; ++nn) acc[nn] = fmaf(ol[nn * K + kk], w, acc[nn]);
+    tc_fence_after();
+    const uint32_t tmem = ms.tmem_base;
+
+    launch_dependents();
+    if (warp == 0 && elect_one()) {
+        prefetch_tensormap(&maps.w);
+        prefetch_tensormap(&maps.x);
+        // W_UV does not depend on the preceding kernels: load it first, then
+        // wait for the grid that writes out_lat (programmatic dependent launch)
+        for (int c = 0; c < cpc; ++c) {
+            const int kc = c_first + c;
+            mbar_arrive_expect_tx(&ms.full[c], kWChunkBytes + x_chunk_bytes);
+            tma_load_2d(w_s + c * kWChunkBytes, &maps.w, h * d_h, kc * 64, &ms.full[c]);
+            tma_load_2d(w_s + c * kWChunkBytes + kWChunkBytes / 2, &maps.w, h * d_h + 64, kc * 64, &ms.full[c]);
+        }
+        wait_prerequisite_grid();
+        for (int c = 0; c < cpc; ++c)
+            tma_load_2d(x_s + c * x_chunk_bytes, &maps.x, h * K + (c_first + c) * 64, n0, &ms.full[c]);
     }
+    if (warp == 1) {
+        bool ok = true;
+        const uint32_t idesc = idesc_bf16_f32(128, nt, true, false);
+        const uint64_t dW = smem_desc(smem_u32(w_s), kWChunkBytes / 2, 1024, kLayoutSw128);  // MN-major
+        const uint64_t dX = smem_desc(smem_u32(x_s), 16, 1024, kLayoutSw128);               // K-major
+        for (int c = 0; c < cpc && ok; ++c) {
+            ok = mbar_wait_warp(&ms.full[c], 0);
+            tc_fence_after();
 #pragma unroll
-    for (int nn = 0; nn < kSeqPerCta; ++nn) {
-        const int n = n0 + nn;
-        if (n < batch) y[(size_t)n * width + (size_t)h * d_h + j] = to_bf16(acc[nn]);
+            for (int kk = 0; kk < 4; ++kk)
+                if (ok && elect_one())
+                    mma_bf16(tmem, dW + ((c * kWChunkBytes + kk * 2048) >> 4),
+                             dX + ((c * x_chunk_bytes + kk * 32) >> 4), idesc, (c | kk) ? 1u : 0u);
+            __syncwarp();
+        }
+        if (elect_one()) mma_commit(&ms.mma_done);
+        __syncwarp();
     }
+    // every copy has landed once the MMAs that read it are done; the wait
+    // below also covers the case where an MMA wait gave up (bounded)
+    const bool done = mbar_wait(&ms.mma_done, 0);
+    if (warp == 0 && lane == 0)
+        for (int c = 0; c < cpc; ++c) mbar_wait(&ms.full[c], 0, 200000000ull);
+    __syncthreads();
+    tc_fence_after();
+    // stage this CTA's partial: thread j writes row j (nt fp32)
+    const int j = warp * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    for (int c0 = 0; c0 < nt; c0 += 16) {
+        float v[16];
+        tmem_ld16(tmem + lane_off + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4*>(part + j * nt + c0 + i) =
+                done ? make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    tc_fence_before();
+    cluster_sync();  // every CTA's partial is staged
+    // CTA `rank` sums columns [n_lo, n_hi) over the cluster
+    const int per = nt / ks;
+    const int n_lo = (int)rank * per, n_hi = n_lo + per;
+    const uint32_t part_addr = smem_u32(part);
+    if (j < d_h) {
+        for (int nn = n_lo; nn < n_hi; nn += 4) {
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int r = 0; r < ks; ++r) {
+                const float4 v = ld_shared_cluster_f4(map_shared_rank(part_addr + (j * nt + nn) * 4, r));
+                acc.x += v.x;
+                acc.y += v.y;
+                acc.z += v.z;
+                acc.w += v.w;
+            }
+            const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int n = n0 + nn + i;
+                if (n < batch) y[(size_t)n * heads * d_h + (size_t)h * d_h + j] = to_bf16(vals[i]);
+            }
+        }
+    }
+    cluster_sync();  // no CTA leaves while another still reads its shared memory
+    if (warp == 1) tmem_dealloc(tmem, tmem_cols);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+bool encode(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
+            uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {inner * 2};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -48,10 +191,37 @@ cudaError_t launch_up_proj(int batch, int heads, int branches, int d_c, int d_h,
                            const __nv_bfloat16* out_lat, const __nv_bfloat16* w_uv,
                            __nv_bfloat16* y, cudaStream_t stream) {
     const int K = branches * d_c;
-    dim3 grid(heads, ceil_div(batch, kSeqPerCta));
-    up_proj_simt_kernel<<<grid, d_h, sizeof(float) * kSeqPerCta * K, stream>>>(batch, heads, K, d_h,
-                                                                             out_lat, w_uv, y);
-    return cudaGetLastError();
+    if (K % 64 != 0 || K / 64 > kMaxChunks) return cudaErrorInvalidValue;
+    const int nchunk = K / 64;
+    const int ks = nchunk % 4 == 0 ? 4 : (nchunk % 2 == 0 ? 2 : 1);  // CTAs splitting K (cluster size)
+    // sequences per CTA: a multiple of 16 (MMA N) and of 4 * ks, at most 64
+    const int nt = batch >= kMaxNT ? kMaxNT : ceil_div(batch, 16) * 16;
+    UpMaps maps;
+    if (!encode(&maps.w, w_uv, (uint64_t)heads * d_h, (uint64_t)K, 64, 64) ||
+        !encode(&maps.x, out_lat, (uint64_t)heads * K, (uint64_t)batch, 64, (uint32_t)nt))
+        return cudaErrorInvalidValue;
+    const int cpc = nchunk / ks;
+    size_t smem = (size_t)cpc * (kWChunkBytes + nt * 128) + sizeof(UpSmem) + 64;
+    const size_t part_bytes = (size_t)128 * nt * 4;
+    if (smem < part_bytes) smem = part_bytes + 64;  // the partial reuses the operand buffers
+    smem += 1024;
+    cudaError_t e = cudaFuncSetAttribute(up_proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(heads * ks, ceil_div(batch, nt));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = ks;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, up_proj_tc_kernel, maps, batch, heads, K, d_h, nt, ks, y);
 }
 
 }  // namespace mlra
