@@ -26,9 +26,8 @@ mlra_status check_dims(const mlra_dims* d) {
     if ((int64_t)d->num_pages * d->page_size > INT32_MAX) return MLRA_ERR_INVALID_ARG;
     if ((int64_t)d->max_pages_per_seq * d->page_size > INT32_MAX) return MLRA_ERR_INVALID_ARG;
     if ((int64_t)d->batch * d->max_pages_per_seq > INT32_MAX) return MLRA_ERR_INVALID_ARG;
-    // the plan counts 128-token tiles in int32
-    if ((int64_t)d->batch * d->max_pages_per_seq * d->page_size / kTileTokens > (int64_t(1) << 30))
-        return MLRA_ERR_INVALID_ARG;
+    // the plan counts cost units in int32
+    if (!plan_fits_int32(d->batch, d->page_size, d->max_pages_per_seq)) return MLRA_ERR_INVALID_ARG;
     if (d->batch > 65535) return MLRA_ERR_UNSUPPORTED;
     return MLRA_OK;
 }
@@ -191,6 +190,7 @@ mlra_status mlra_decode_plan(int32_t batch, int32_t page_size, int32_t max_pages
     if (batch < 1 || page_size < 1 || max_pages_per_seq < 1 || num_ctas < 1) return MLRA_ERR_INVALID_ARG;
     if (!aligned16(seqlens) || !aligned16(plan_out)) return MLRA_ERR_INVALID_ARG;
     if ((int64_t)max_pages_per_seq * page_size > INT32_MAX) return MLRA_ERR_INVALID_ARG;
+    if (!plan_fits_int32(batch, page_size, max_pages_per_seq)) return MLRA_ERR_INVALID_ARG;
     return cuda_status(launch_plan_dump(batch, page_size, max_pages_per_seq, seqlens, num_ctas,
                                         plan_out, static_cast<cudaStream_t>(stream)));
 }

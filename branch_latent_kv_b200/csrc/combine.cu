@@ -40,11 +40,9 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(DecodeArgs a) {
         const int tiles = seq_tiles(Ln, a.page_size, a.max_pages);
         int c0 = 0, c1 = -1;
         if (tiles > 0) {
-            const int total = warp_total_tiles(a.seqlens, a.batch, a.page_size, a.max_pages);
-            const int chunk = ceil_div(total, a.num_ctas);
-            const int first = warp_seq_first_tile(a.seqlens, n, a.page_size, a.max_pages);
-            c0 = first / chunk;
-            c1 = (first + tiles - 1) / chunk;
+            const int cum = warp_cost_prefix(a.seqlens, n, a.page_size, a.max_pages);
+            const int total = cum + warp_cost_prefix(a.seqlens + n, a.batch - n, a.page_size, a.max_pages);
+            seq_owners(cum, tiles, plan_chunk(total, a.num_ctas), &c0, &c1);
         }
         if (tid == 0) {
             info[0] = tiles;

@@ -58,10 +58,22 @@ __device__ __forceinline__ void record_error(int* err, int code) {
 
 // ---------------------------------------------------------------------------
 // Split-KV plan.  Sequence n owns tiles_n = ceil(L_n / 128) tiles, or none if
-// L_n is invalid.  The concatenated tile list is cut into num_ctas contiguous
-// ranges of chunk = ceil(total / num_ctas) tiles.  Every kernel recomputes
-// this from seqlens with the warp routines below (no plan buffer).
+// L_n is invalid.  Work is counted in cost units: a tile costs kTileCost, and
+// every sequence adds kSeqCost after its last tile for the per-segment work
+// (query load, first-tile setup, epilogue) that a CTA pays each time its range
+// enters a new sequence.  Sequence n occupies the cost interval
+// [cum_n, cum_n + cost_n), cost_n = kTileCost * tiles_n + kSeqCost, and its
+// tile t starts at cum_n + kTileCost * t.  With
+//   chunk = max(ceil(total_cost / num_ctas), kTileCost)
+// CTA c owns the tiles whose start lies in [c * chunk, (c + 1) * chunk).
+// Ranges are contiguous in the tile list, and because chunk >= kTileCost
+// every CTA between the first and the last owner of a sequence owns at least
+// one of its tiles.  Every kernel recomputes this from seqlens with the warp
+// routines below (no plan buffer).
 // ---------------------------------------------------------------------------
+constexpr int kTileCost = 8;
+constexpr int kSeqCost = 8;
+
 __device__ __forceinline__ bool seqlen_valid(int L, int page_size, int max_pages) {
     return L >= 1 && (long long)L <= (long long)max_pages * page_size;
 }
@@ -70,54 +82,75 @@ __device__ __forceinline__ int seq_tiles(int L, int page_size, int max_pages) {
     return seqlen_valid(L, page_size, max_pages) ? (L + kTileTokens - 1) / kTileTokens : 0;
 }
 
-// Whole warp: total number of tiles.
-__device__ inline int warp_total_tiles(const int32_t* seqlens, int batch, int P, int max_pages) {
+__device__ __forceinline__ int seq_cost(int L, int page_size, int max_pages) {
+    const int t = seq_tiles(L, page_size, max_pages);
+    return t > 0 ? t * kTileCost + kSeqCost : 0;
+}
+
+__host__ __device__ __forceinline__ int plan_chunk(int total_cost, int num_ctas) {
+    const int c = (total_cost + num_ctas - 1) / num_ctas;
+    return c > kTileCost ? c : kTileCost;
+}
+
+// First tile of a sequence (cost start cum, `tiles` tiles) that starts at or
+// after position A; `tiles` if none does.
+__device__ __forceinline__ int first_tile_at(int cum, int tiles, int A) {
+    if (A <= cum) return 0;
+    const int t = (A - cum + kTileCost - 1) / kTileCost;
+    return t < tiles ? t : tiles;
+}
+
+// Whole warp: sum of the costs of sequences [0, n).
+__device__ inline int warp_cost_prefix(const int32_t* seqlens, int n, int P, int max_pages) {
     const int lane = threadIdx.x & 31;
     int sum = 0;
-    for (int n = lane; n < batch; n += 32) sum += seq_tiles(__ldg(seqlens + n), P, max_pages);
+    for (int m = lane; m < n; m += 32) sum += seq_cost(__ldg(seqlens + m), P, max_pages);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     return sum;
 }
 
-// Whole warp: first global tile of sequence n (sum of tiles of sequences < n).
-__device__ inline int warp_seq_first_tile(const int32_t* seqlens, int n, int P, int max_pages) {
-    const int lane = threadIdx.x & 31;
-    int sum = 0;
-    for (int m = lane; m < n; m += 32) sum += seq_tiles(__ldg(seqlens + m), P, max_pages);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    return sum;
-}
-
-// Whole warp: the sequence whose tile range contains global tile g (g < total)
-// and that sequence's first global tile.
+// Whole warp: the first sequence with a tile starting at or after position A,
+// and its cost start (batch and the total cost if there is none).
 __device__ inline void warp_find_seq(const int32_t* seqlens, int batch, int P, int max_pages,
-                                     int g, int* seq_out, int* first_out) {
+                                     int A, int* seq_out, int* cum_out) {
     const int lane = threadIdx.x & 31;
     int base_cum = 0;
     for (int base = 0; base < batch; base += 32) {
         const int n = base + lane;
-        const int t = n < batch ? seq_tiles(__ldg(seqlens + n), P, max_pages) : 0;
-        int incl = t;
+        const int c = n < batch ? seq_cost(__ldg(seqlens + n), P, max_pages) : 0;
+        int incl = c;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int v = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += v;
         }
-        const int excl = incl - t;
-        const unsigned hit = __ballot_sync(0xffffffffu, t > 0 && base_cum + excl <= g &&
-                                                            g < base_cum + incl);
+        const int excl = incl - c;
+        // last tile start = cum + cost - kSeqCost - kTileCost
+        const unsigned hit = __ballot_sync(0xffffffffu,
+                                           c > 0 && base_cum + incl - kSeqCost - kTileCost >= A);
         if (hit) {
             const int src = __ffs(hit) - 1;
             *seq_out = base + src;
-            *first_out = __shfl_sync(0xffffffffu, base_cum + excl, src);
+            *cum_out = __shfl_sync(0xffffffffu, base_cum + excl, src);
             return;
         }
         base_cum += __shfl_sync(0xffffffffu, incl, 31);
     }
-    *seq_out = -1;
-    *first_out = base_cum;
+    *seq_out = batch;
+    *cum_out = base_cum;
+}
+
+// The plan's cost positions are int32: the largest possible total must fit.
+inline bool plan_fits_int32(long long batch, long long page_size, long long max_pages) {
+    const long long tiles_per_seq = (max_pages * page_size + kTileTokens - 1) / kTileTokens;
+    return batch * (tiles_per_seq * kTileCost + kSeqCost) <= (1LL << 30);
+}
+
+// CTAs owning the first and the last tile of a sequence (tiles > 0).
+__device__ __forceinline__ void seq_owners(int cum, int tiles, int chunk, int* c0, int* c1) {
+    *c0 = cum / chunk;
+    *c1 = (cum + (tiles - 1) * kTileCost) / chunk;
 }
 
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }

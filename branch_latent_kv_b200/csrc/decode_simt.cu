@@ -45,7 +45,7 @@ __device__ inline float bf16_at(const __nv_bfloat16* p, size_t i) { return __bfl
 
 __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
     extern __shared__ float sm[];
-    __shared__ int plan[4];  // total, chunk, first sequence, its first tile
+    __shared__ int plan[4];  // chunk, first sequence, its cost start
     __shared__ int seg_bad;
 
     const int H = a.heads, B = a.branches, d_c = a.d_c, d_r = a.d_r, P = a.page_size;
@@ -64,25 +64,27 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
     const int cta = blockIdx.x;
 
     if (tid < 32) {
-        const int total = warp_total_tiles(a.seqlens, a.batch, P, a.max_pages);
-        const int chunk = ceil_div(total, a.num_ctas);
-        const int g0 = cta * chunk;
-        int n0 = -1, f0 = 0;
-        if (g0 < total) warp_find_seq(a.seqlens, a.batch, P, a.max_pages, g0, &n0, &f0);
-        if (tid == 0) { plan[0] = total; plan[1] = chunk; plan[2] = n0; plan[3] = f0; }
+        const int total = warp_cost_prefix(a.seqlens, a.batch, P, a.max_pages);
+        const int chunk = plan_chunk(total, a.num_ctas);
+        int n0 = a.batch, cum0 = total;
+        if ((long long)cta * chunk < total)
+            warp_find_seq(a.seqlens, a.batch, P, a.max_pages, cta * chunk, &n0, &cum0);
+        if (tid == 0) { plan[0] = chunk; plan[1] = n0; plan[2] = cum0; }
     }
     __syncthreads();
-    const int total = plan[0], chunk = plan[1];
-    const int g0 = cta * chunk, g1 = min(g0 + chunk, total);
-    if (g0 >= g1) return;
+    const int chunk = plan[0];
+    const int A0 = cta * chunk, A1 = A0 + chunk;  // this CTA's cost window
 
-    int n = plan[2], first = plan[3];
-    while (n < a.batch && first < g1) {
+    int n = plan[1], cum = plan[2];
+    for (; n < a.batch && cum < A1; ++n) {
         const int Ln = __ldg(a.seqlens + n);
         const int tiles = seq_tiles(Ln, P, a.max_pages);
-        if (tiles == 0) { ++n; continue; }
-        const int tb = max(g0, first) - first;
-        const int te = min(g1, first + tiles) - first;
+        if (tiles == 0) continue;
+        const int cum_n = cum;
+        cum += seq_cost(Ln, P, a.max_pages);
+        const int tb = first_tile_at(cum_n, tiles, A0);
+        const int te = first_tile_at(cum_n, tiles, A1);
+        if (tb >= te) continue;
         const int tok_begin = tb * kTileTokens;
         const int tok_end = min(te * kTileTokens, Ln);
         const int32_t* bt = a.block_table + (size_t)n * a.max_pages;
@@ -180,7 +182,8 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
         }
 
         // epilogue: final output of a single-split sequence, else a partial
-        const int first_cta = first / chunk, last_cta = (first + tiles - 1) / chunk;
+        int first_cta, last_cta;
+        seq_owners(cum_n, tiles, chunk, &first_cta, &last_cta);
         const bool bad = seg_bad != 0;
         if (bad && tid == 0) record_error(a.err, MLRA_ERR_DEVICE_BAD_INDEX);
         if (first_cta == last_cta) {
@@ -203,8 +206,6 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
             }
         }
         __syncthreads();
-        first += tiles;
-        ++n;
     }
 }
 

@@ -54,9 +54,16 @@ template <int NB, int DC, int DR>
 struct Cfg {
     static constexpr int W = NB * DC;                       // latent elements per token
     static constexpr int NCHUNK = W / 64;                   // 64-column (128-byte) chunks
-    static constexpr int G = DC >= 128 ? 1 : 128 / DC;      // branches per step
-    static constexpr int PPS = DC >= 128 ? DC / 128 : 1;    // pairs per step
-    static constexpr int NSTEP = NB / G;                    // steps per tile
+    // A step is the unit of the MMA <-> softmax pipeline: SBR branches whose
+    // latents are PPS "pairs" (128 latent columns each); a pair holds BPP
+    // branches (two when DC = 64).
+    // one pair per step: the ring must hold two steps in flight plus the
+    // copies ahead of them, so steps stay as small as the pair layout allows
+    static constexpr int SBR = DC >= 128 ? 1 : 128 / DC;           // branches per step
+    static constexpr int BPP = DC >= 128 ? 1 : 128 / DC;            // branches per pair
+    static constexpr int PPS = SBR * DC / 128 > 0 ? SBR * DC / 128 : 1;  // pairs per step
+    static constexpr int NPAIR = W / 128;                           // pairs per tile
+    static constexpr int NSTEP = NB / SBR;                          // steps per tile
     static constexpr int CHUNK_BYTES = kT * 128;            // 16 KB
     static constexpr int PAIR_BYTES = 2 * CHUNK_BYTES;      // 32 KB
     static constexpr int ROPE_ROW = DR * 2;                 // 128 or 64 bytes
@@ -66,27 +73,28 @@ struct Cfg {
     static constexpr int QR_BYTES = kHP * ROPE_ROW;                 // [16 heads x d_r]
     static constexpr int QR_SPAN = (QR_BYTES + 1023) / 1024 * 1024;  // keeps the next region aligned
     static constexpr int P_BRANCH_BYTES = kT * kHP * 2;     // 4 KB
-    static constexpr int P_BYTES = G * P_BRANCH_BYTES;
+    static constexpr int P_BYTES = SBR * P_BRANCH_BYTES;   // one P slot (a step)
     static constexpr int MISC_BYTES = 4096;
-    static constexpr int FIXED = 2 * ROPE_BYTES + Q_BYTES + QR_SPAN + 2 * P_BYTES + MISC_BYTES;
+    static constexpr int FIXED = ROPE_BYTES + Q_BYTES + QR_SPAN + 2 * P_BYTES + MISC_BYTES;
     static constexpr int NSTAGE_FIT = (kSmemLimit - 1024 - FIXED) / PAIR_BYTES;
     static constexpr int NSTAGE = NSTAGE_FIT > 8 ? 8 : NSTAGE_FIT;
     // shared-memory offsets from a 1024-byte aligned base
     static constexpr int OFF_PAIR = 0;
     static constexpr int OFF_ROPE = OFF_PAIR + NSTAGE * PAIR_BYTES;
-    static constexpr int OFF_Q = OFF_ROPE + 2 * ROPE_BYTES;
+    static constexpr int OFF_Q = OFF_ROPE + ROPE_BYTES;  // one RoPE tile: its only reader runs at step 0
     static constexpr int OFF_QR = OFF_Q + Q_BYTES;
     static constexpr int OFF_P = OFF_QR + QR_SPAN;
     static constexpr int OFF_MISC = OFF_P + 2 * P_BYTES;
     static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
     // TMEM columns: O blocks first, then two S slots, then two slots of the
     // RoPE score shared by all branches of a tile
-    static constexpr int O_BLOCKS = NSTEP * PPS * G;
+    static constexpr int O_BLOCKS = NPAIR * BPP;
     static constexpr int S_COL0 = O_BLOCKS * kHP;
-    static constexpr int S_SLOT_COLS = G * kHP;
+    static constexpr int S_SLOT_COLS = SBR * kHP;
     static constexpr int R_COL0 = S_COL0 + 2 * S_SLOT_COLS;
     static constexpr int TMEM_COLS = R_COL0 + 2 * kHP <= 128 ? 128 : 256;
-    static_assert(NB % G == 0, "branches must fill whole steps");
+    static_assert(NB % SBR == 0 && (SBR * DC) % 128 == 0, "branches must fill whole steps and pairs");
+    static_assert(NSTEP * PPS == NPAIR, "step / pair bookkeeping");
     static_assert(NSTAGE >= PPS, "a step's pairs must fit the stage ring");
     // The score MMA of step s+1 is issued before the output MMA of step s
     // (overlapping the softmax of s) only when both steps' pairs fit the ring.
@@ -192,21 +200,28 @@ __device__ __forceinline__ uint64_t rope_desc(uint32_t addr) {
     return DR == 64 ? smem_desc(addr, 16, 1024, kLayoutSw128) : smem_desc(addr, 16, 512, kLayoutSw64);
 }
 
-// The sequence-range walk every role performs identically.
-__device__ __forceinline__ bool next_segment(const DecodeArgs& a, int& n, int first, int g0, int g1,
+// The sequence walk every role performs identically: the next sequence n
+// (cost start cum) with tiles [tb, te) in this CTA's cost window [A0, A1).
+// The caller advances past it with finish_segment.
+__device__ __forceinline__ bool next_segment(const DecodeArgs& a, int& n, int& cum, int A0, int A1,
                                              int& L, int& tiles, int& tb, int& te) {
-    while (n < a.batch && first < g1) {
+    while (n < a.batch && cum < A1) {
         L = __ldg(a.seqlens + n);
         tiles = seq_tiles(L, a.page_size, a.max_pages);
-        if (tiles == 0) {
-            ++n;
-            continue;
+        if (tiles > 0) {
+            tb = first_tile_at(cum, tiles, A0);
+            te = first_tile_at(cum, tiles, A1);
+            if (tb < te) return true;
+            cum += tiles * kTileCost + kSeqCost;
         }
-        tb = max(g0, first) - first;
-        te = min(g1, first + tiles) - first;
-        return true;
+        ++n;
     }
     return false;
+}
+
+__device__ __forceinline__ void finish_segment(int& n, int& cum, int tiles) {
+    cum += tiles * kTileCost + kSeqCost;
+    ++n;
 }
 
 template <int NB, int DC, int DR>
@@ -239,16 +254,15 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
         fence_barrier_init();
     }
     if (warp == 0) {
-        const int total = warp_total_tiles(a.seqlens, a.batch, P, a.max_pages);
-        const int chunk = total > 0 ? ceil_div(total, a.num_ctas) : 0;
-        const int g0 = blockIdx.x * chunk;
-        int n0 = -1, f0 = 0;
-        if (g0 < total) warp_find_seq(a.seqlens, a.batch, P, a.max_pages, g0, &n0, &f0);
+        const int total = warp_cost_prefix(a.seqlens, a.batch, P, a.max_pages);
+        const int chunk = plan_chunk(total, a.num_ctas);
+        int n0 = a.batch, cum0 = total;
+        if ((long long)blockIdx.x * chunk < total)
+            warp_find_seq(a.seqlens, a.batch, P, a.max_pages, blockIdx.x * chunk, &n0, &cum0);
         if (lane == 0) {
-            misc.plan[0] = total;
             misc.plan[1] = chunk;
             misc.plan[2] = n0;
-            misc.plan[3] = f0;
+            misc.plan[3] = cum0;
         }
         prefetch_tensormap(&maps.lat);
         prefetch_tensormap(&maps.rope);
@@ -262,19 +276,19 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
     tc_fence_after();
 
     launch_dependents();  // the combine kernel may be scheduled as CTAs retire
-    const int total = misc.plan[0], chunk = misc.plan[1];
-    const int g0 = blockIdx.x * chunk, g1 = min(g0 + chunk, total);
+    const int chunk = misc.plan[1];
+    const int A0 = blockIdx.x * chunk, A1 = A0 + chunk;  // this CTA's cost window
     const uint32_t tmem = misc.tmem_base;
     volatile int* abort_flag = &misc.abort_flag;
 
-    if (g0 < g1) {
+    if (misc.plan[2] < a.batch) {
         if (warp == 0) {
             // ------------------------------------------------------------ producer
-            int n = misc.plan[2], first = misc.plan[3];
+            int n = misc.plan[2], cum = misc.plan[3];
             int L, tiles, tb, te;
             uint32_t pc = 0, tc = 0;
             bool ok = true;
-            while (ok && next_segment(a, n, first, g0, g1, L, tiles, tb, te)) {
+            while (ok && next_segment(a, n, cum, A0, A1, L, tiles, tb, te)) {
                 const int32_t* bt = a.block_table + (size_t)n * a.max_pages;
                 int win_base = -(1 << 30), win_val = 0;
                 for (int j = tb; j < te && ok; ++j) {
@@ -288,18 +302,17 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                         const int v = idx < a.max_pages ? __ldg(bt + idx) : 0;
                         win_val = (v >= 0 && v < a.num_pages) ? v : 0;  // bad entries are reported by the softmax warps
                     }
-                    const int rslot = tc & 1;
                     if (lane == 0) {
-                        ok = mbar_wait(&misc.rope_empty[rslot], ((tc >> 1) & 1) ^ 1);
-                        if (ok) mbar_arrive_expect_tx(&misc.rope_full[rslot], npages * P * C::ROPE_ROW);
+                        ok = mbar_wait(&misc.rope_empty[0], (tc & 1) ^ 1);
+                        if (ok) mbar_arrive_expect_tx(&misc.rope_full[0], npages * P * C::ROPE_ROW);
                     }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
                     for (int q = 0; q < npages; ++q) {
                         const int page = __shfl_sync(0xffffffffu, win_val, page0 + q - win_base);
                         if (lane == 0)
-                            tma_load_2d(sm + C::OFF_ROPE + rslot * C::ROPE_BYTES + q * P * C::ROPE_ROW,
-                                        &maps.rope, 0, page * P, &misc.rope_full[rslot]);
+                            tma_load_2d(sm + C::OFF_ROPE + q * P * C::ROPE_ROW, &maps.rope, 0, page * P,
+                                        &misc.rope_full[0]);
                     }
                     ++tc;
                     for (int sp = 0; sp < C::NSTEP * C::PPS && ok; ++sp) {
@@ -324,8 +337,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                     }
                     ok = __shfl_sync(0xffffffffu, ok && !*abort_flag, 0);
                 }
-                first += tiles;
-                ++n;
+                finish_segment(n, cum, tiles);
             }
             if (!ok) {
                 if (lane == 0) {
@@ -340,10 +352,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                     const uint32_t k = pc - 1 - i;
                     mbar_wait(&misc.pair_full[k % C::NSTAGE], (k / C::NSTAGE) & 1, 200000000ull);
                 }
-                for (uint32_t i = 0; i < 2 && i < tc; ++i) {
-                    const uint32_t k = tc - 1 - i;
-                    mbar_wait(&misc.rope_full[k & 1], (k >> 1) & 1, 200000000ull);
-                }
+                if (tc > 0) mbar_wait(&misc.rope_full[0], (tc - 1) & 1, 200000000ull);
             }
         } else if (warp == 1) {
             // ------------------------------------------------------------ MMA issuer
@@ -361,7 +370,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                 const uint64_t dQR = rope_desc<DR>(sm_base + C::OFF_QR);
                 const uint64_t dR = rope_desc<DR>(sm_base + C::OFF_ROPE);
                 const uint64_t dP = smem_desc(sm_base + C::OFF_P, 128, 2048, kLayoutNone);
-                int n = misc.plan[2], first = misc.plan[3];
+                int n = misc.plan[2], cum = misc.plan[3];
                 int L, tiles, tb, te;
                 uint32_t gs = 0, tc = 0, sc = 0;
                 uint32_t stage = 0, phase = 0;  // ring position of the next pair to consume
@@ -381,12 +390,15 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                         if (sp >= (uint32_t)C::NSTAGE) sp -= C::NSTAGE;
                         const uint64_t a0 = dA_pv + ((sp * C::PAIR_BYTES) >> 4);
 #pragma unroll
-                        for (int g = 0; g < C::G; ++g) {
-                            const uint32_t d = tmem + ((pst * C::PPS + p) * C::G + g) * kHP;
+                        for (int g2 = 0; g2 < C::BPP; ++g2) {
+                            // branch of the step whose P multiplies this pair (rows of the
+                            // other branch of a shared pair are discarded later)
+                            const int gl = DC >= 128 ? p * 128 / DC : p * C::BPP + g2;
+                            const uint32_t d = tmem + ((pst * C::PPS + p) * C::BPP + g2) * kHP;
 #pragma unroll
                             for (int kt = 0; kt < kT / 16; ++kt)
                                 if (elect_one())
-                                    mma_bf16(d, a0 + (kt * 2048 >> 4), b0 + ((g * C::P_BRANCH_BYTES + kt * 256) >> 4),
+                                    mma_bf16(d, a0 + (kt * 2048 >> 4), b0 + ((gl * C::P_BRANCH_BYTES + kt * 256) >> 4),
                                              IDESC_PV, (pfirst && kt == 0) ? 0u : 1u);
                         }
                     }
@@ -401,13 +413,12 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                     return true;
                 };
 
-                while (ok && next_segment(a, n, first, g0, g1, L, tiles, tb, te)) {
+                while (ok && next_segment(a, n, cum, A0, A1, L, tiles, tb, te)) {
                     ok = mbar_wait_warp(&misc.q_full, sc & 1);
                     tc_fence_after();
                     for (int j = tb; j < te && ok; ++j) {
-                        const int rslot = tc & 1;
-                        ok = mbar_wait_warp(&misc.rope_full[rslot], (tc >> 1) & 1);
-                        const uint64_t dRs = dR + ((rslot * C::ROPE_BYTES) >> 4);
+                        ok = mbar_wait_warp(&misc.rope_full[0], tc & 1);
+                        const uint64_t dRs = dR;
 #pragma unroll 1
                         for (int st = 0; st < C::NSTEP && ok; ++st) {
                             const uint32_t stage0 = stage;
@@ -426,14 +437,14 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
 #pragma unroll
                                 for (int kk = 0; kk < DR / 16; ++kk)
                                     if (elect_one()) mma_bf16(dRt, dRs + kk * 2, dQR + kk * 2, IDESC_S, kk ? 1u : 0u);
-                                if (elect_one()) mma_commit(&misc.rope_empty[rslot]);
+                                if (elect_one()) mma_commit(&misc.rope_empty[0]);
                                 __syncwarp();
                             }
                             const uint32_t dS = tmem + C::S_COL0 + (gs & 1) * C::S_SLOT_COLS;
                             // this step's branches start at chunk st*G*(DC/64) of the token row
-                            const uint64_t dQs = dQ + ((st * C::G * (DC / 64) * C::Q_CHUNK_BYTES) >> 4);
+                            const uint64_t dQs = dQ + ((st * C::SBR * (DC / 64) * C::Q_CHUNK_BYTES) >> 4);
 #pragma unroll
-                            for (int g = 0; g < C::G; ++g) {
+                            for (int g = 0; g < C::SBR; ++g) {
 #pragma unroll
                                 for (int c = 0; c < DC / 64; ++c) {
                                     // chunk (g*(DC/64) + c) of this step: pair pp, half hf
@@ -471,8 +482,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                     if (ok && elect_one()) mma_commit(&misc.seg_done);
                     __syncwarp();
                     ++sc;
-                    first += tiles;
-                    ++n;
+                    finish_segment(n, cum, tiles);
                 }
                 if (!ok && lane == 0) {
                     record_error(a.err, MLRA_ERR_DEVICE_TIMEOUT);
@@ -491,7 +501,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
             const int stid = threadIdx.x - 64;         // 0..127 within the group
             const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
             const int H = a.heads;
-            int n = misc.plan[2], first = misc.plan[3];
+            int n = misc.plan[2], cum = misc.plan[3];
             int L, tiles, tb, te;
             uint32_t gs = 0, sc = 0, tcnt = 0;  // steps, ranges, tiles so far
             // This thread's share of the softmax denominators, one row per
@@ -500,7 +510,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
             float l[NB][kHP];
             bool dead = false;
 
-            while (!dead && next_segment(a, n, first, g0, g1, L, tiles, tb, te)) {
+            while (!dead && next_segment(a, n, cum, A0, A1, L, tiles, tb, te)) {
                 // queries of sequence n -> shared memory (128-byte swizzled, K-major)
                 {
                     const uint4* q_src = reinterpret_cast<const uint4*>(a.q_lat + (size_t)n * H * C::W);
@@ -532,8 +542,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                         bad |= (v < 0 || v >= a.num_pages);
                     }
                 }
-                if (stid < NB * kHP) misc.m_run[stid] = -INFINITY;
-                bad = named_bar_or<1, 128>(bad);  // also publishes m_run
+                bad = named_bar_or<1, 128>(bad);
                 fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
@@ -551,16 +560,32 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                     for (int st = 0; st < C::NSTEP; ++st) {
                         const bool ok = mbar_wait(&misc.s_full[gs & 1], (gs >> 1) & 1);
                         tc_fence_after();
-                        float x[C::G][kHP];
+                        float x[C::SBR][kHP];
                         if (st == 0) tmem_ld16(tmem + lane_off + C::R_COL0 + (tcnt & 1) * kHP, r);
 #pragma unroll
-                        for (int g = 0; g < C::G; ++g)
+                        for (int g = 0; g < C::SBR; ++g)
                             tmem_ld16(tmem + lane_off + C::S_COL0 + (gs & 1) * C::S_SLOT_COLS + g * kHP, x[g]);
                         tmem_wait_ld();
-                        float* m_step = &misc.m_run[st * C::G * kHP];
-                        float m[C::G][kHP];
 #pragma unroll
-                        for (int g = 0; g < C::G; ++g)
+                        for (int g = 0; g < C::SBR; ++g)
+#pragma unroll
+                            for (int i = 0; i < kHP; ++i)
+                                x[g][i] = masked ? -INFINITY : (x[g][i] + r[i]) * a.scale_log2;
+                        float* m_step = &misc.m_run[st * C::SBR * kHP];
+                        if (j == tb) {
+                            // first tile of the range: token 0 (always valid) sets the
+                            // reference maxima; larger scores take the exact path below
+                            if (stid == 0) {
+#pragma unroll
+                                for (int g = 0; g < C::SBR; ++g)
+#pragma unroll
+                                    for (int i = 0; i < kHP; ++i) m_step[g * kHP + i] = x[g][i];
+                            }
+                            named_bar_sync<1, 128>();
+                        }
+                        float m[C::SBR][kHP];
+#pragma unroll
+                        for (int g = 0; g < C::SBR; ++g)
 #pragma unroll
                             for (int i = 0; i < kHP; i += 4) {
                                 const float4 v = *reinterpret_cast<const float4*>(m_step + g * kHP + i);
@@ -571,12 +596,9 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                             }
                         bool need = false;
 #pragma unroll
-                        for (int g = 0; g < C::G; ++g)
+                        for (int g = 0; g < C::SBR; ++g)
 #pragma unroll
-                            for (int i = 0; i < kHP; ++i) {
-                                x[g][i] = masked ? -INFINITY : (x[g][i] + r[i]) * a.scale_log2;
-                                need |= x[g][i] > m[g][i] + kRescaleLog2;
-                            }
+                            for (int i = 0; i < kHP; ++i) need |= x[g][i] > m[g][i] + kRescaleLog2;
                         if (named_bar_or<1, 128>(need || !ok)) {
                             if (named_bar_or<1, 128>(!ok)) {
                                 dead = true;
@@ -585,14 +607,14 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                             // exact column max over the tile's 128 tokens: a warp
                             // reduce-scatter leaves column (lane >> 1) in each lane
 #pragma unroll
-                            for (int g = 0; g < C::G; ++g) {
+                            for (int g = 0; g < C::SBR; ++g) {
                                 const float v = warp_colmax16(x[g], lane);
                                 if ((lane & 1) == 0) misc.red_max[quad][g * kHP + (lane >> 1)] = v;
                             }
                             named_bar_sync<1, 128>();
-                            float alpha[C::G][kHP];
+                            float alpha[C::SBR][kHP];
 #pragma unroll
-                            for (int g = 0; g < C::G; ++g)
+                            for (int g = 0; g < C::SBR; ++g)
 #pragma unroll
                                 for (int i = 0; i < kHP; ++i) {
                                     const float tmax = fmaxf(fmaxf(misc.red_max[0][g * kHP + i], misc.red_max[1][g * kHP + i]),
@@ -606,7 +628,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                             // barrier below publishes the new ones (and frees red_max)
                             if (stid == 0) {
 #pragma unroll
-                                for (int g = 0; g < C::G; ++g)
+                                for (int g = 0; g < C::SBR; ++g)
 #pragma unroll
                                     for (int i = 0; i < kHP; ++i) m_step[g * kHP + i] = m[g][i];
                             }
@@ -623,13 +645,14 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
 #pragma unroll
                                 for (int p = 0; p < C::PPS; ++p)
 #pragma unroll
-                                    for (int g = 0; g < C::G; ++g) {
-                                        const uint32_t col = ((st * C::PPS + p) * C::G + g) * kHP;
+                                    for (int g2 = 0; g2 < C::BPP; ++g2) {
+                                        const int gl = DC >= 128 ? p * 128 / DC : p * C::BPP + g2;
+                                        const uint32_t col = ((st * C::PPS + p) * C::BPP + g2) * kHP;
                                         float o[kHP];
                                         tmem_ld16(tmem + lane_off + col, o);
                                         tmem_wait_ld();
 #pragma unroll
-                                        for (int i = 0; i < kHP; ++i) o[i] *= alpha[g][i];
+                                        for (int i = 0; i < kHP; ++i) o[i] *= alpha[gl][i];
                                         tmem_st16(tmem + lane_off + col, o);
                                     }
                                 tmem_wait_st();
@@ -638,7 +661,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                         // probabilities -> bf16 P (MN-major, 8x8 core matrices)
                         uint8_t* p_slot = sm + C::OFF_P + (gs & 1) * C::P_BYTES;
 #pragma unroll
-                        for (int g = 0; g < C::G; ++g) {
+                        for (int g = 0; g < C::SBR; ++g) {
                             uint32_t packed[kHP / 2];
 #pragma unroll
                             for (int i = 0; i < kHP; i += 2) {
@@ -673,7 +696,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                         if (lane == 0) mbar_arrive(&misc.p_full[gs & 1]);
                         // rotate the denominator rows: the next step's branches first
 #pragma unroll
-                        for (int r = 0; r < C::G; ++r) {
+                        for (int r = 0; r < C::SBR; ++r) {
                             float t[kHP];
 #pragma unroll
                             for (int i = 0; i < kHP; ++i) t[i] = l[0][i];
@@ -691,15 +714,9 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                 if (dead) break;
 
                 // ---------------------------------------------------- epilogue
-                // (two output MMAs may still be in flight here, so o_done's parity
-                // cannot tell them apart: wait for the range's own barrier)
-                const bool ok = mbar_wait(&misc.seg_done, sc & 1);
-                if (named_bar_or<1, 128>(!ok)) {
-                    dead = true;
-                    break;
-                }
-                tc_fence_after();
-                // denominators: warp reduce-scatter, then the four warps through shared memory
+                // denominators (final once the last probabilities are written):
+                // warp reduce-scatter, then the four warps through shared memory,
+                // while the range's last output MMA may still run
                 {
                     constexpr int NV = NB * kHP;
                     float f[NV];
@@ -716,7 +733,8 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                     }
                 }
                 named_bar_sync<1, 128>();
-                const int first_cta = first / chunk, last_cta = (first + tiles - 1) / chunk;
+                int first_cta, last_cta;
+                seq_owners(cum, tiles, chunk, &first_cta, &last_cta);
                 const bool single = first_cta == last_cta;
                 const size_t slot = (size_t)blockIdx.x + n;
                 if (stid < NB * kHP) {
@@ -727,43 +745,54 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                     if (!single && i < H)
                         a.lse_part[(slot * NB + b) * H + i] = bad ? bad_split_marker() : misc.m_run[stid] + __log2f(lt);
                 }
-                named_bar_sync<1, 128>();
+                // the range's own barrier: two output MMAs may be in flight, so
+                // o_done's parity cannot tell them apart (the barrier below also
+                // publishes inv_l)
+                {
+                    const bool ok = mbar_wait(&misc.seg_done, sc & 1);
+                    if (named_bar_or<1, 128>(!ok)) {
+                        dead = true;
+                        break;
+                    }
+                }
+                tc_fence_after();
                 // outputs: a block of TMEM holds 128 latent rows x 16 heads of one
-                // branch (or two branches of 64 rows when DC = 64)
+                // branch (or two branches of 64 rows when DC = 64); all blocks are
+                // read before a single wait
                 constexpr int WIDTH = DC >= 128 ? 128 : DC;  // valid rows per block
-#pragma unroll 1
+                float o[C::O_BLOCKS][kHP];
+#pragma unroll
+                for (int blk = 0; blk < C::O_BLOCKS; ++blk) tmem_ld16(tmem + lane_off + blk * kHP, o[blk]);
+                tmem_wait_ld();
+#pragma unroll
                 for (int blk = 0; blk < C::O_BLOCKS; ++blk) {
-                    const int g = blk % C::G, sp = blk / C::G;       // sp = st * PPS + p
-                    const int st = sp / C::PPS;
-                    const int b = st * C::G + g;
-                    const int row0 = C::G == 1 ? 0 : g * WIDTH;      // first valid row of the block
-                    const int k = (sp * 128 + row0) % DC + (row - row0);  // latent column of this row
+                    const int g2 = blk % C::BPP, gp = blk / C::BPP;  // pair of the tile, branch in it
+                    const int row0 = g2 * WIDTH;                     // first valid row of the block
+                    const int b = (gp * 128 + row0) / DC;            // branch of the block
+                    const int k = (gp * 128 + row0) % DC + (row - row0);  // latent column of this row
                     const bool mine = row >= row0 && row < row0 + WIDTH;
-                    float o[kHP];
-                    tmem_ld16(tmem + lane_off + blk * kHP, o);
-                    tmem_wait_ld();
                     if (!mine) continue;
                     const float* inv = &misc.inv_l[b * kHP];
 #pragma unroll
-                    for (int i = 0; i < kHP; ++i) o[i] = bad ? 0.f : o[i] * inv[i];
+                    for (int i = 0; i < kHP; ++i) o[blk][i] = bad ? 0.f : o[blk][i] * inv[i];
                     if (single) {
                         __nv_bfloat16* dst = a.out + ((size_t)n * H * NB + b) * DC + k;
 #pragma unroll
                         for (int i = 0; i < kHP; ++i)
-                            if (i < H) dst[(size_t)i * NB * DC] = to_bf16(o[i] * a.out_scale);
+                            if (i < H) dst[(size_t)i * NB * DC] = to_bf16(o[blk][i] * a.out_scale);
                     } else {
                         // partial layout [slot][branch][k][16 heads]: 64 contiguous bytes per row
                         float4* dst = reinterpret_cast<float4*>(a.o_part + (((slot * NB + b) * DC + k) * kHP));
 #pragma unroll
-                        for (int i = 0; i < kHP; i += 4) dst[i / 4] = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+                        for (int i = 0; i < kHP; i += 4)
+                            dst[i / 4] = make_float4(o[blk][i], o[blk][i + 1], o[blk][i + 2], o[blk][i + 3]);
                     }
                 }
                 if (bad && stid == 0) record_error(a.err, MLRA_ERR_DEVICE_BAD_INDEX);
                 tc_fence_before();
                 named_bar_sync<1, 128>();  // inv_l and red_sum are reused by the next range
                 ++sc;
-                first += tiles;
-                ++n;
+                finish_segment(n, cum, tiles);
             }
             if (dead && stid == 0) {
                 record_error(a.err, MLRA_ERR_DEVICE_TIMEOUT);

@@ -194,11 +194,16 @@ MLRA_API const char* mlra_status_string(mlra_status status);
 /*
  * The split-KV work partition mlra_decode uses, written for inspection.
  * Sequence n has tiles_n = ceil(L_n / 128) token tiles (0 if L_n is
- * invalid); the concatenation of all tiles is cut into `num_ctas` contiguous
- * ranges of ceil(total / num_ctas) tiles, CTA c taking range c.
+ * invalid).  Work is counted in cost units: 8 per tile plus 8 per valid
+ * sequence, placed after its last tile, for the per-sequence setup and
+ * epilogue.  Sequence n spans [cum_n, cum_n + 8 * tiles_n + 8) and its tile t
+ * starts at cum_n + 8 * t; with chunk = max(ceil(total / num_ctas), 8), CTA c
+ * owns the tiles that start in [c * chunk, (c + 1) * chunk).  The ranges are
+ * contiguous in the list of all tiles.
  *   plan_out int32 device [num_ctas * 4 + batch * 2]:
- *     per CTA c:  first tile (global), end tile (global), first sequence,
- *                 last sequence touched (-1, -1 when the range is empty)
+ *     per CTA c:  first tile (global index), end tile (global), first
+ *                 sequence, last sequence touched (0, 0, -1, -1 when the
+ *                 CTA owns no tile)
  *     per seq n:  number of CTAs covering it (0 if invalid), first such CTA
  * Returns after enqueueing one small kernel.
  */

@@ -2,12 +2,18 @@
 for the bit-exact plan test).
 
 Sequence n has tiles_n = ceil(L_n / 128) tiles of 128 tokens, or none when
-L_n < 1 or L_n > max_pages_per_seq * page_size.  The concatenation of all
-tiles is cut into num_ctas contiguous ranges of ceil(total / num_ctas) tiles.
+L_n < 1 or L_n > max_pages_per_seq * page_size.  Each tile costs TILE_COST
+units and each valid sequence SEQ_COST more, placed after its last tile, so a
+CTA whose range enters a new sequence is given less token work.  Tile t of
+sequence n starts at cum_n + TILE_COST * t; with
+chunk = max(ceil(total / num_ctas), TILE_COST), CTA c owns the tiles that
+start in [c * chunk, (c + 1) * chunk).
 """
 from __future__ import annotations
 
 TILE = 128
+TILE_COST = 8
+SEQ_COST = 8
 
 
 def seq_tiles(L, page_size, max_pages):
@@ -16,32 +22,32 @@ def seq_tiles(L, page_size, max_pages):
     return -(-L // TILE)
 
 
+def owners(seqlens, page_size, max_pages, num_ctas):
+    """Owner CTA of every tile, as a list of (sequence, tile, cta)."""
+    tiles = [seq_tiles(int(L), page_size, max_pages) for L in seqlens]
+    total = sum(TILE_COST * t + SEQ_COST for t in tiles if t)
+    chunk = max(-(-total // num_ctas), TILE_COST)
+    out, cum = [], 0
+    for n, t in enumerate(tiles):
+        if not t:
+            continue
+        for i in range(t):
+            out.append((n, i, (cum + TILE_COST * i) // chunk))
+        cum += TILE_COST * t + SEQ_COST
+    return out
+
+
 def plan(seqlens, page_size, max_pages, num_ctas):
     """Returns the flat int list the library's plan dump writes."""
-    tiles = [seq_tiles(int(L), page_size, max_pages) for L in seqlens]
-    total = sum(tiles)
-    chunk = -(-total // num_ctas) if total > 0 else 0
-    firsts, acc = [], 0
-    for t in tiles:
-        firsts.append(acc)
-        acc += t
-
-    def seq_of(g):
-        for n, (f, t) in enumerate(zip(firsts, tiles)):
-            if t > 0 and f <= g < f + t:
-                return n
-        return -1
-
-    out = []
-    for c in range(num_ctas):
-        g0, g1 = c * chunk, min(c * chunk + chunk, total)
-        if g0 < g1:
-            out += [g0, g1, seq_of(g0), seq_of(g1 - 1)]
-        else:
-            out += [min(g0, total), max(g1, min(g0, total)), -1, -1]
-    for f, t in zip(firsts, tiles):
-        if t == 0:
-            out += [0, -1]
-        else:
-            out += [(f + t - 1) // chunk - f // chunk + 1, f // chunk]
+    own = owners(seqlens, page_size, max_pages, num_ctas)
+    per_cta = [[0, 0, -1, -1] for _ in range(num_ctas)]
+    for g, (n, _, c) in enumerate(own):
+        p = per_cta[c]
+        if p[2] < 0:
+            p[0], p[2] = g, n
+        p[1], p[3] = g + 1, n
+    out = [v for p in per_cta for v in p]
+    for n in range(len(seqlens)):
+        cs = sorted({c for m, _, c in own if m == n})
+        out += [len(cs), cs[0]] if cs else [0, -1]
     return out

@@ -116,6 +116,7 @@ def test_binding_refuses_cpu_tensors():
 @pytest.mark.parametrize("seqlens,ctas", [
     ([8192] * 16, 148), ([1, 127, 128, 129, 0, 300], 7), ([131072] * 4, 148),
     ([5], 148), ([0, 0], 4), (list(range(1, 2000, 37)), 148), ([128 * 1000 + 1, 3], 3),
+    ([128] * 300, 148), ([1, 1, 4096, 1, 1], 148), ([8192] * 16 + [0], 5),
 ])
 def test_plan_model_covers_every_tile_once(seqlens, ctas):
     P, maxp = 64, 4096
@@ -129,11 +130,17 @@ def test_plan_model_covers_every_tile_once(seqlens, ctas):
         if g0 < g1:
             assert 0 <= n0 <= n1 < len(seqlens)
         else:
-            assert n0 == n1 == -1
+            assert (g0, g1, n0, n1) == (0, 0, -1, -1)
     assert covered == list(range(total))
-    # ranges differ in size by at most one chunk (the last non-empty one may be short)
-    sizes = [flat[4 * c + 1] - flat[4 * c] for c in range(ctas)]
-    assert max(sizes, default=0) - min([s for s in sizes if s] or [0]) <= max(sizes, default=0)
+    # a CTA's tiles plus the per-sequence charge of each sequence it enters
+    # fit within one chunk of cost, up to one tile and one sequence charge
+    total_cost = sum(plan_model.TILE_COST * t + plan_model.SEQ_COST for t in tiles if t)
+    chunk = max(-(-total_cost // ctas), plan_model.TILE_COST)
+    for c in range(ctas):
+        g0, g1, n0, n1 = flat[4 * c:4 * c + 4]
+        if g0 < g1:
+            cost = plan_model.TILE_COST * (g1 - g0) + plan_model.SEQ_COST * (n1 - n0)
+            assert cost <= chunk + plan_model.TILE_COST + plan_model.SEQ_COST
     for n, t in enumerate(tiles):
         splits, first = flat[4 * ctas + 2 * n:4 * ctas + 2 * n + 2]
         if t == 0:
@@ -142,3 +149,16 @@ def test_plan_model_covers_every_tile_once(seqlens, ctas):
             owners = [c for c in range(ctas)
                       if flat[4 * c] < flat[4 * c + 1] and flat[4 * c + 2] <= n <= flat[4 * c + 3]]
             assert owners == list(range(first, first + splits))
+
+
+def test_plan_model_gives_sequence_crossing_ctas_fewer_tiles():
+    # 16 sequences of 64 tiles over 148 CTAs: a CTA whose range enters a
+    # second sequence pays that sequence's charge in tiles
+    flat = plan_model.plan([8192] * 16, 64, 128, 148)
+    one, two = [], []
+    for c in range(148):
+        g0, g1, n0, n1 = flat[4 * c:4 * c + 4]
+        if g0 < g1:
+            (two if n1 > n0 else one).append(g1 - g0)
+    assert two and max(two) < max(one)
+    assert sum(one) + sum(two) == 16 * 64
