@@ -28,7 +28,7 @@ mlra_status check_dims(const mlra_dims* d) {
     if ((int64_t)d->batch * d->max_pages_per_seq > INT32_MAX) return MLRA_ERR_INVALID_ARG;
     // the plan counts cost units in int32
     if (!plan_fits_int32(d->batch, d->page_size, d->max_pages_per_seq)) return MLRA_ERR_INVALID_ARG;
-    if (d->batch > 65535) return MLRA_ERR_UNSUPPORTED;
+    if (d->batch > kMaxBatch) return MLRA_ERR_UNSUPPORTED;
     return MLRA_OK;
 }
 
@@ -97,6 +97,7 @@ mlra_status decode_impl(Impl impl, const mlra_dims* dims, const void* q_lat, con
     a.err = reinterpret_cast<int*>(ws + wl.err_off);
     a.lse_part = reinterpret_cast<float*>(ws + wl.lse_off);
     a.o_part = reinterpret_cast<float*>(ws + wl.o_off);
+    a.seq_cnt = reinterpret_cast<int*>(ws + wl.cnt_off);
     a.batch = dims->batch;
     a.heads = dims->heads;
     a.branches = dims->branches;
@@ -110,8 +111,8 @@ mlra_status decode_impl(Impl impl, const mlra_dims* dims, const void* q_lat, con
     a.out_scale = out_scale;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    mlra_status r = cuda_status(impl == Impl::kTensorCore ? launch_decode_tc(a, st)
-                                                          : launch_decode_simt(a, st));
+    if (impl == Impl::kTensorCore) return cuda_status(launch_decode_tc(a, st));  // merges in-kernel
+    mlra_status r = cuda_status(launch_decode_simt(a, st));
     if (r != MLRA_OK) return r;
     return cuda_status(launch_combine(a, st));
 }

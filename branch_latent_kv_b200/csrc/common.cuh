@@ -28,18 +28,25 @@ constexpr float kLog2e = 1.4426950408889634f;
 // c + n (unique because CTA ranges are contiguous and ordered).
 // ---------------------------------------------------------------------------
 struct WorkspaceLayout {
-    size_t err_off, lse_off, o_off, total;
+    size_t err_off, lse_off, o_off, cnt_off, total;
     int slots;
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Largest batch the library accepts (int32 sequence ids, 16-bit grid rows).
+constexpr int kMaxBatch = 65535;
 
 __host__ __device__ inline WorkspaceLayout workspace_layout(int batch, int heads, int branches,
                                                             int d_c, int num_ctas) {
     WorkspaceLayout w;
     w.slots = num_ctas + batch;
     w.err_off = 0;
-    w.lse_off = 256;
+    // per-sequence split counters of the tensor-core kernel's merge, at a
+    // fixed place sized for the largest batch: calls with other dimensions
+    // that reuse the workspace find them where they left them (at zero)
+    w.cnt_off = 256;
+    w.lse_off = align256(w.cnt_off + sizeof(int) * (size_t)(kMaxBatch + 1));
     w.o_off = align256(w.lse_off + sizeof(float) * (size_t)w.slots * branches * heads);
     const size_t hp = heads <= 16 ? 16 : (size_t)heads;  // heads padded to 16 (more for the CUDA-core kernel)
     w.total = align256(w.o_off + sizeof(float) * (size_t)w.slots * branches * d_c * hp);

@@ -36,8 +36,9 @@ constexpr int kMaxDevices = 64;
 
 // The scratch.  In host code this name only stands for the symbol: its
 // device address comes from cudaGetSymbolAddress below.  Device memory of a
-// __device__ array starts zeroed, so the error word at its start is 0 before
-// the first call; each call clears it again after copying it out.
+// __device__ array starts zeroed, so the error word at its start and the
+// split counters are 0 before the first call; each call clears the error word
+// again after copying it out, and the decode kernel returns the counters to 0.
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 std::mutex g_setup_mutex;

@@ -10,17 +10,20 @@
 // (abstract of "Multi-Head Low-Rank Attention"), so the kernel streams each
 // token's latent and RoPE row through shared memory exactly once.
 //
-// Organisation (one persistent CTA per SM, 192 threads):
+// Organisation (one persistent CTA per SM, 224 threads):
 //   warp 0     TMA producer: per 128-token tile, the RoPE tile and, per
 //              "pair" of 64-column chunks (128 latent columns), the paged
 //              latent rows (one 2-D box per page) into a ring of stages.
-//   warp 1     MMA issuer (one thread) and TMEM owner:
+//   warp 1     score MMA issuer (one thread) and TMEM owner:
 //                S^T_b[t, h]  = C_b[t, :] . Q_b[h, :] + K_r[t, :] . Q_r[h, :]
 //                               M = 128 tokens, N = 16 heads, K = d_c + d_r
+//   warp 6     output MMA issuer (one thread):
 //                O^T_b[k, h] += C_b[:, k]^T . P_b[:, h]
 //                               M = 128 latent columns, N = 16 heads, K = 128 tokens
 //              (the same shared-memory tile is the K-major A operand of the
-//              score MMA and the MN-major A operand of the output MMA).
+//              score MMA and the MN-major A operand of the output MMA).  An
+//              MMA issue stalls the issuing warp for about one MMA's duration,
+//              so two issuers keep the tensor pipe busy while either waits.
 //   warps 2-5  softmax and epilogue: thread t owns token t of the tile (a
 //              TMEM lane); scores are base-2 logits; each (head, branch) has
 //              its own running max, rescaled only when a score exceeds it by
@@ -46,7 +49,7 @@ using namespace sm100;
 
 constexpr int kHP = 16;             // heads padded to the MMA N
 constexpr int kT = kTileTokens;     // tokens per tile = MMA M
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kSmemLimit = 232448;  // max dynamic shared memory per CTA on sm_100
 
@@ -75,15 +78,16 @@ struct Cfg {
     static constexpr int P_BRANCH_BYTES = kT * kHP * 2;     // 4 KB
     static constexpr int P_BYTES = SBR * P_BRANCH_BYTES;   // one P slot (a step)
     static constexpr int MISC_BYTES = 4096;
-    static constexpr int FIXED = ROPE_BYTES + Q_BYTES + QR_SPAN + 2 * P_BYTES + MISC_BYTES;
+    static constexpr int QSET_BYTES = Q_BYTES + QR_SPAN;  // one sequence's queries (two slots)
+    static constexpr int FIXED = ROPE_BYTES + 2 * QSET_BYTES + 2 * P_BYTES + MISC_BYTES;
     static constexpr int NSTAGE_FIT = (kSmemLimit - 1024 - FIXED) / PAIR_BYTES;
     static constexpr int NSTAGE = NSTAGE_FIT > 8 ? 8 : NSTAGE_FIT;
     // shared-memory offsets from a 1024-byte aligned base
     static constexpr int OFF_PAIR = 0;
     static constexpr int OFF_ROPE = OFF_PAIR + NSTAGE * PAIR_BYTES;
     static constexpr int OFF_Q = OFF_ROPE + ROPE_BYTES;  // one RoPE tile: its only reader runs at step 0
-    static constexpr int OFF_QR = OFF_Q + Q_BYTES;
-    static constexpr int OFF_P = OFF_QR + QR_SPAN;
+    static constexpr int OFF_QR = OFF_Q + Q_BYTES;       // slot s at + s * QSET_BYTES
+    static constexpr int OFF_P = OFF_Q + 2 * QSET_BYTES;
     static constexpr int OFF_MISC = OFF_P + 2 * P_BYTES;
     static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
     // TMEM columns: O blocks first, then two S slots, then two slots of the
@@ -96,12 +100,10 @@ struct Cfg {
     static_assert(NB % SBR == 0 && (SBR * DC) % 128 == 0, "branches must fill whole steps and pairs");
     static_assert(NSTEP * PPS == NPAIR, "step / pair bookkeeping");
     static_assert(NSTAGE >= PPS, "a step's pairs must fit the stage ring");
-    // The score MMA of step s+1 is issued before the output MMA of step s
-    // (overlapping the softmax of s) only when both steps' pairs fit the ring.
-    static constexpr bool OVERLAP = 2 * PPS <= NSTAGE;
     static_assert(R_COL0 + 2 * kHP <= TMEM_COLS, "TMEM budget");
     static_assert(SMEM_BYTES <= kSmemLimit, "shared-memory budget");
-    static_assert(OFF_QR + QR_BYTES <= OFF_P && OFF_Q + Q_BYTES <= OFF_QR && OFF_P + 2 * P_BYTES <= OFF_MISC,
+    static_assert(OFF_QR + QSET_BYTES + QR_BYTES <= OFF_P && OFF_Q + Q_BYTES <= OFF_QR &&
+                  OFF_P + 2 * P_BYTES <= OFF_MISC && QSET_BYTES % 1024 == 0,
                   "shared-memory regions must not overlap");
     static_assert(DR == 32 || DR == 64, "RoPE width");
 };
@@ -113,15 +115,18 @@ struct Misc {
     uint64_t pair_empty[NSTAGE];
     uint64_t rope_full[2];
     uint64_t rope_empty[2];
-    uint64_t s_full[2];
-    uint64_t p_full[2];
-    uint64_t o_done;    // one phase per output MMA step (rescale path: at most one outstanding)
-    uint64_t seg_done;  // one phase per sequence range: every output MMA of the range finished
-    uint64_t q_full;
-    uint64_t drain;
+    uint64_t s_full[2];   // step g in slot g & 1: its scores are in TMEM
+    uint64_t p_full[2];   // its probabilities are in shared memory
+    uint64_t p_empty[2];  // its output MMA finished (S and P slots free, O up to date)
+    uint64_t q_full[2];   // sequence range r in slot r & 1: its queries are in shared memory
+    uint64_t q_empty[2];  // its score MMAs finished
+    uint64_t drain[2];
     uint32_t tmem_base;
     int abort_flag;
     int plan[4];
+    int last_seg[3];  // this CTA's last sequence range: sequence, cost start, tiles (-1: none)
+    int merge_flag;   // merge: bit 0 a split met a bad page, bit 1 the wait expired
+    uint64_t merge_bar;  // merge: the bulk copies of the partial slices
     float red_max[4][2 * kHP];
     float red_sum[4][4 * kHP];
     alignas(16) float m_run[8 * kHP];  // running max per (branch, head), base-2 logits; read as float4
@@ -132,8 +137,10 @@ static_assert(offsetof(Misc<5>, m_run) % 16 == 0 && offsetof(Misc<4>, m_run) % 1
               offsetof(Misc<6>, m_run) % 16 == 0, "float4 access to m_run");
 
 struct Maps {
-    CUtensorMap lat;
-    CUtensorMap rope;
+    CUtensorMap lat;   // latent cache rows [pages * P][W]
+    CUtensorMap rope;  // RoPE cache rows [pages * P][d_r]
+    CUtensorMap q;     // q_lat [batch][H][W]: a 16-head box per 64 columns (heads >= H read as 0)
+    CUtensorMap qr;    // q_rope [batch][H][d_r]
 };
 
 // 2^x on the special-function unit (ex2.approx, flush-to-zero: results below
@@ -202,11 +209,17 @@ __device__ __forceinline__ uint64_t rope_desc(uint32_t addr) {
 
 // The sequence walk every role performs identically: the next sequence n
 // (cost start cum) with tiles [tb, te) in this CTA's cost window [A0, A1).
-// The caller advances past it with finish_segment.
+// next_len holds seqlens[n], loaded one range ahead (first_len starts it).
+// The caller advances past the range with finish_segment.
+__device__ __forceinline__ int first_len(const DecodeArgs& a, int n) {
+    return n < a.batch ? __ldg(a.seqlens + n) : 0;
+}
+
 __device__ __forceinline__ bool next_segment(const DecodeArgs& a, int& n, int& cum, int A0, int A1,
-                                             int& L, int& tiles, int& tb, int& te) {
+                                             int& L, int& tiles, int& tb, int& te, int& next_len) {
     while (n < a.batch && cum < A1) {
-        L = __ldg(a.seqlens + n);
+        L = next_len;
+        next_len = n + 1 < a.batch ? __ldg(a.seqlens + n + 1) : 0;
         tiles = seq_tiles(L, a.page_size, a.max_pages);
         if (tiles > 0) {
             tb = first_tile_at(cum, tiles, A0);
@@ -224,9 +237,165 @@ __device__ __forceinline__ void finish_segment(int& n, int& cum, int tiles) {
     ++n;
 }
 
+// End of the kernel, all threads: the merge of split sequences and the
+// outputs of sequences with an invalid length.
+//
+// Sequence n with S > 1 splits (CTAs c0..c1) is merged by the CTAs whose
+// range ends in it: c0..c1-1 always, c1 when n is also its last sequence.
+// Each such CTA waits until all S splits have counted their partials into
+// seq_cnt[n], then combines rows [i R / G, (i+1) R / G) of the R = NB * DC
+// (branch, latent column) rows, i = c - c0, G the group size:
+//   o = out_scale * sum_s w_s o_s / sum_s w_s,  w_s = 2^(lse_s - max_s lse_s)
+// per (branch, head) -- the log-sum-exp merge of independent softmax
+// partitions.  The last of the S + G counts returns seq_cnt[n] to zero.
+template <int NB, int DC>
+__device__ __forceinline__ void merge_tail(const DecodeArgs& a, int n, int cum, int tiles, int chunk,
+                                        float* w_s, int* flag, uint64_t* bar) {
+    constexpr int HB = NB * kHP;  // (branch, head) weights per split
+    constexpr int R = NB * DC;    // (branch, latent column) rows
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int H = a.heads;
+
+    // invalid lengths: zeros and an error code, sequence m by CTA m mod grid
+    const int next_len = (n >= 0 && n + 1 < a.batch) ? __ldg(a.seqlens + n + 1) : 0;
+    for (int m = blockIdx.x; m < a.batch; m += a.num_ctas) {
+        if (seq_tiles(__ldg(a.seqlens + m), a.page_size, a.max_pages) > 0) continue;
+        __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(a.out + (size_t)m * H * R);
+        for (int e = tid; e < H * R / 2; e += kThreads) dst[e] = __floats2bfloat162_rn(0.f, 0.f);
+        if (tid == 0) record_error(a.err, MLRA_ERR_DEVICE_BAD_SEQLEN);
+    }
+    if (n < 0) return;
+    int c0, c1;
+    seq_owners(cum, tiles, chunk, &c0, &c1);
+    const int S = c1 - c0 + 1;
+    if (S == 1) return;  // written by the epilogue
+    // c1 belongs to the group when no later tile is its own: the next valid
+    // sequence starts at cum + cost_n, owned by c1 or a later CTA
+    bool c1_member = true;
+    for (int m = n + 1; m < a.batch; ++m) {
+        const int Lm = m == n + 1 ? next_len : __ldg(a.seqlens + m);
+        if (seq_tiles(Lm, a.page_size, a.max_pages) == 0) continue;
+        c1_member = (cum + tiles * kTileCost + kSeqCost) / chunk != c1;
+        break;
+    }
+    const int G = c1_member ? S : S - 1;
+    const int gi = blockIdx.x - c0;  // 0 <= gi < G: n is this CTA's last sequence
+    // this CTA's rows; a work item is (row, head quad), quads fastest so that
+    // each split's loads are contiguous 16-byte units
+    const int r0 = (int)((long long)gi * R / G), r1 = (int)((long long)(gi + 1) * R / G);
+    // wait until every split of n has counted its partials
+    if (tid == 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire_gpu(a.seq_cnt + n) < S) {
+            if (globaltimer_ns() - t0 > 2000000000ull) {
+                *flag = 2;
+                record_error(a.err, MLRA_ERR_DEVICE_TIMEOUT);
+                break;
+            }
+            __nanosleep(32);
+        }
+    }
+    __syncthreads();
+    if (*flag & 2) return;
+
+    // this CTA's row slice of every split's partial -> shared memory by bulk
+    // copies (rows are contiguous within a slot), in flight while the weights
+    // are formed
+    const int rows = r1 - r0;
+    float* part_s = w_s + S * HB;  // [S][rows][16 heads]
+    if (warp == 0 && rows > 0) {
+        const uint32_t slice = (uint32_t)rows * kHP * 4;
+        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)S * slice);
+        __syncwarp();
+        for (int sp = lane; sp < S; sp += 32)
+            bulk_load(part_s + (size_t)sp * rows * kHP,
+                      a.o_part + ((size_t)(c0 + n + sp) * R + r0) * kHP, slice, bar);
+    }
+    // log-sum-exps -> shared memory, eight independent loads per thread at a time
+    const float* lse = a.lse_part;
+    for (int e0 = tid; e0 < S * HB; e0 += 8 * kThreads) {
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = e0 + j * kThreads, sp = e / HB, bh = e % HB, b = bh / kHP, h = bh % kHP;
+            v[j] = (e < S * HB && h < H) ? __ldcg(lse + ((size_t)(c0 + sp + n) * NB + b) * H + h) : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (e0 + j * kThreads < S * HB) w_s[e0 + j * kThreads] = v[j];
+    }
+    __syncthreads();
+    // weights out_scale * 2^(lse - max) / sum per (branch, head): eight lanes
+    // per (branch, head), the splits strided over them
+    {
+        const int sub = lane & 7;
+        for (int bh = warp * 4 + (lane >> 3); bh < HB; bh += (kThreads / 32) * 4) {
+            float mx = -INFINITY;
+            bool bad = false;
+            for (int sp = sub; sp < S; sp += 8) {
+                const float l = w_s[sp * HB + bh];
+                if (l == bad_split_marker()) bad = true; else mx = fmaxf(mx, l);
+            }
+#pragma unroll
+            for (int o = 4; o > 0; o >>= 1) {
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                bad |= __shfl_xor_sync(0xffffffffu, (int)bad, o) != 0;
+            }
+            float sum = 0.f;
+            for (int sp = sub; sp < S; sp += 8) {
+                const float w = bad ? 0.f : exp2f(w_s[sp * HB + bh] - mx);
+                w_s[sp * HB + bh] = w;
+                sum += w;
+            }
+#pragma unroll
+            for (int o = 4; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            if (bad) {
+                if (sub == 0 && bh % kHP < H) atomicOr(flag, 1);
+            } else {
+                const float norm = a.out_scale / sum;
+                for (int sp = sub; sp < S; sp += 8) w_s[sp * HB + bh] *= norm;
+            }
+        }
+    }
+    __syncthreads();
+    const bool bad = *flag & 1;
+    if (bad && tid == 0) record_error(a.err, MLRA_ERR_DEVICE_BAD_INDEX);
+    if (rows > 0 && !mbar_wait(bar, 0, 200000000ull)) {
+        if (tid == 0) record_error(a.err, MLRA_ERR_DEVICE_TIMEOUT);
+        return;
+    }
+
+    // items (row, head quad), quads fastest: conflict-free 16-byte reads
+    for (int e = tid; e < rows * 4; e += kThreads) {
+        const int lr = e / 4, q = e % 4, row = r0 + lr;
+        const int b = row / DC, k = row % DC;
+        const float* w = w_s + b * kHP + 4 * q;
+        const float* src = part_s + lr * kHP + 4 * q;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+        for (int sp = 0; sp < S; ++sp) {
+            const float4 v = *reinterpret_cast<const float4*>(src + (size_t)sp * rows * kHP);
+            const float4 wv = *reinterpret_cast<const float4*>(w + sp * HB);
+            acc.x = fmaf(wv.x, v.x, acc.x);
+            acc.y = fmaf(wv.y, v.y, acc.y);
+            acc.z = fmaf(wv.z, v.z, acc.z);
+            acc.w = fmaf(wv.w, v.w, acc.w);
+        }
+        if (bad) acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        __nv_bfloat16* dst = a.out + ((size_t)n * H * NB + b) * DC + k;
+        const float v4[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (4 * q + j < H) dst[(size_t)(4 * q + j) * NB * DC] = to_bf16(v4[j]);
+    }
+    __syncthreads();
+    // the last of the S arrivals and G departures resets the counter
+    if (tid == 0 && atomicAdd(a.seq_cnt + n, 1) == S + G - 1) a.seq_cnt[n] = 0;
+}
+
 template <int NB, int DC, int DR>
 __global__ void __launch_bounds__(kThreads, 1)
-decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
+decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ DecodeArgs a) {
     using C = Cfg<NB, DC, DR>;
     using M = Misc<C::NSTAGE>;
     extern __shared__ uint8_t smem_raw[];
@@ -245,12 +414,17 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
             mbar_init(&misc.rope_empty[i], 1);
             mbar_init(&misc.s_full[i], 1);
             mbar_init(&misc.p_full[i], 4);
+            mbar_init(&misc.p_empty[i], 1);
+            mbar_init(&misc.drain[i], 1);
         }
-        mbar_init(&misc.o_done, 1);
-        mbar_init(&misc.seg_done, 1);
-        mbar_init(&misc.q_full, 4);
-        mbar_init(&misc.drain, 1);
+        mbar_init(&misc.q_full[0], 1);
+        mbar_init(&misc.q_full[1], 1);
+        mbar_init(&misc.q_empty[0], 1);
+        mbar_init(&misc.q_empty[1], 1);
+        mbar_init(&misc.merge_bar, 1);
         misc.abort_flag = 0;
+        misc.last_seg[0] = -1;
+        misc.merge_flag = 0;
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -266,6 +440,8 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
         }
         prefetch_tensormap(&maps.lat);
         prefetch_tensormap(&maps.rope);
+        prefetch_tensormap(&maps.q);
+        prefetch_tensormap(&maps.qr);
     }
     if (warp == 1) {
         tmem_alloc(&misc.tmem_base, C::TMEM_COLS);
@@ -284,11 +460,27 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
     if (misc.plan[2] < a.batch) {
         if (warp == 0) {
             // ------------------------------------------------------------ producer
-            int n = misc.plan[2], cum = misc.plan[3];
+            int n = misc.plan[2], cum = misc.plan[3], next_len = first_len(a, n);
             int L, tiles, tb, te;
-            uint32_t pc = 0, tc = 0;
+            uint32_t pc = 0, tc = 0, sc = 0;
             bool ok = true;
-            while (ok && next_segment(a, n, cum, A0, A1, L, tiles, tb, te)) {
+            while (ok && next_segment(a, n, cum, A0, A1, L, tiles, tb, te, next_len)) {
+                // the sequence's queries into slot sc & 1, once the range two
+                // before has finished its score MMAs
+                if (lane == 0) {
+                    if (sc >= 2) ok = mbar_wait(&misc.q_empty[sc & 1], ((sc >> 1) - 1) & 1);
+                    if (ok) {
+                        uint64_t* qb = &misc.q_full[sc & 1];
+                        uint8_t* qd = sm + C::OFF_Q + (sc & 1) * C::QSET_BYTES;
+                        mbar_arrive_expect_tx(qb, C::Q_BYTES + C::QR_BYTES);
+                        for (int c = 0; c < C::NCHUNK; ++c)
+                            tma_load_3d(qd + c * C::Q_CHUNK_BYTES, &maps.q, c * 64, 0, n, qb);
+                        tma_load_3d(qd + C::Q_BYTES, &maps.qr, 0, 0, n, qb);
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                ++sc;
                 const int32_t* bt = a.block_table + (size_t)n * a.max_pages;
                 int win_base = -(1 << 30), win_val = 0;
                 for (int j = tb; j < te && ok; ++j) {
@@ -353,146 +545,160 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                     mbar_wait(&misc.pair_full[k % C::NSTAGE], (k / C::NSTAGE) & 1, 200000000ull);
                 }
                 if (tc > 0) mbar_wait(&misc.rope_full[0], (tc - 1) & 1, 200000000ull);
+                for (uint32_t i = 0; i < 2u && i < sc; ++i) {
+                    const uint32_t k = sc - 1 - i;
+                    mbar_wait(&misc.q_full[k & 1], (k >> 1) & 1, 200000000ull);
+                }
             }
         } else if (warp == 1) {
-            // ------------------------------------------------------------ MMA issuer
+            // ------------------------------------------------------------ score MMA issuer
             // (the whole warp walks the schedule; the elected lane issues)
-            {
-                constexpr uint32_t IDESC_S = idesc_bf16_f32(128, kHP, false, false);
-                constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, kHP, true, true);
-                const uint32_t sm_base = smem_u32(sm);
-                // Descriptor bases; every operand below is a base plus a byte
-                // offset >> 4 (the start-address field never overflows: all
-                // addresses are below 256 KB).
-                const uint64_t dA_s = smem_desc(sm_base + C::OFF_PAIR, 16, 1024, kLayoutSw128);       // K-major
-                const uint64_t dA_pv = smem_desc(sm_base + C::OFF_PAIR, C::CHUNK_BYTES, 1024, kLayoutSw128);  // MN-major
-                const uint64_t dQ = smem_desc(sm_base + C::OFF_Q, 16, 1024, kLayoutSw128);
-                const uint64_t dQR = rope_desc<DR>(sm_base + C::OFF_QR);
-                const uint64_t dR = rope_desc<DR>(sm_base + C::OFF_ROPE);
-                const uint64_t dP = smem_desc(sm_base + C::OFF_P, 128, 2048, kLayoutNone);
-                int n = misc.plan[2], cum = misc.plan[3];
-                int L, tiles, tb, te;
-                uint32_t gs = 0, tc = 0, sc = 0;
-                uint32_t stage = 0, phase = 0;  // ring position of the next pair to consume
-                bool ok = true;
-                bool have_prev = false;
-                uint32_t prev_gs = 0, prev_stage = 0;
-                int prev_st = 0;
-                bool prev_first = false;
-
-                auto issue_pv = [&](uint32_t pgs, int pst, uint32_t pstage, bool pfirst) -> bool {
-                    if (!mbar_wait_warp(&misc.p_full[pgs & 1], (pgs >> 1) & 1)) return false;
-                    tc_fence_after();
-                    const uint64_t b0 = dP + ((pgs & 1) * C::P_BYTES >> 4);
-#pragma unroll
-                    for (int p = 0; p < C::PPS; ++p) {
-                        uint32_t sp = pstage + p;
-                        if (sp >= (uint32_t)C::NSTAGE) sp -= C::NSTAGE;
-                        const uint64_t a0 = dA_pv + ((sp * C::PAIR_BYTES) >> 4);
-#pragma unroll
-                        for (int g2 = 0; g2 < C::BPP; ++g2) {
-                            // branch of the step whose P multiplies this pair (rows of the
-                            // other branch of a shared pair are discarded later)
-                            const int gl = DC >= 128 ? p * 128 / DC : p * C::BPP + g2;
-                            const uint32_t d = tmem + ((pst * C::PPS + p) * C::BPP + g2) * kHP;
-#pragma unroll
-                            for (int kt = 0; kt < kT / 16; ++kt)
-                                if (elect_one())
-                                    mma_bf16(d, a0 + (kt * 2048 >> 4), b0 + ((gl * C::P_BRANCH_BYTES + kt * 256) >> 4),
-                                             IDESC_PV, (pfirst && kt == 0) ? 0u : 1u);
-                        }
-                    }
-#pragma unroll
-                    for (int p = 0; p < C::PPS; ++p) {
-                        uint32_t sp = pstage + p;
-                        if (sp >= (uint32_t)C::NSTAGE) sp -= C::NSTAGE;
-                        if (elect_one()) mma_commit(&misc.pair_empty[sp]);
-                    }
-                    if (elect_one()) mma_commit(&misc.o_done);
-                    __syncwarp();
-                    return true;
-                };
-
-                while (ok && next_segment(a, n, cum, A0, A1, L, tiles, tb, te)) {
-                    ok = mbar_wait_warp(&misc.q_full, sc & 1);
-                    tc_fence_after();
-                    for (int j = tb; j < te && ok; ++j) {
-                        ok = mbar_wait_warp(&misc.rope_full[0], tc & 1);
-                        const uint64_t dRs = dR;
+            constexpr uint32_t IDESC_S = idesc_bf16_f32(128, kHP, false, false);
+            const uint32_t sm_base = smem_u32(sm);
+            // Descriptor bases; every operand below is a base plus a byte
+            // offset >> 4 (the start-address field never overflows: all
+            // addresses are below 256 KB).
+            const uint64_t dA_s = smem_desc(sm_base + C::OFF_PAIR, 16, 1024, kLayoutSw128);  // K-major
+            const uint64_t dQ = smem_desc(sm_base + C::OFF_Q, 16, 1024, kLayoutSw128);
+            const uint64_t dQR = rope_desc<DR>(sm_base + C::OFF_QR);
+            const uint64_t dR = rope_desc<DR>(sm_base + C::OFF_ROPE);
+            int n = misc.plan[2], cum = misc.plan[3], next_len = first_len(a, n);
+            int L, tiles, tb, te;
+            uint32_t gs = 0, tc = 0, sc = 0;
+            uint32_t stage = 0, phase = 0;  // ring position of the next pair to consume
+            bool ok = true;
+            while (ok && next_segment(a, n, cum, A0, A1, L, tiles, tb, te, next_len)) {
+                ok = mbar_wait_warp(&misc.q_full[sc & 1], (sc >> 1) & 1);
+                tc_fence_after();
+                const uint32_t qoff = ((sc & 1) * C::QSET_BYTES) >> 4;  // descriptor offset of the slot
+                for (int j = tb; j < te && ok; ++j) {
+                    ok = mbar_wait_warp(&misc.rope_full[0], tc & 1);
 #pragma unroll 1
-                        for (int st = 0; st < C::NSTEP && ok; ++st) {
-                            const uint32_t stage0 = stage;
-                            for (int p = 0; p < C::PPS && ok; ++p) {
-                                ok = mbar_wait_warp(&misc.pair_full[stage], phase);
-                                if (++stage == (uint32_t)C::NSTAGE) {
-                                    stage = 0;
-                                    phase ^= 1;
-                                }
+                    for (int st = 0; st < C::NSTEP && ok; ++st) {
+                        const uint32_t stage0 = stage;
+                        for (int p = 0; p < C::PPS && ok; ++p) {
+                            ok = mbar_wait_warp(&misc.pair_full[stage], phase);
+                            if (++stage == (uint32_t)C::NSTAGE) {
+                                stage = 0;
+                                phase ^= 1;
                             }
-                            if (!ok) break;
-                            tc_fence_after();
-                            if (st == 0) {
-                                // RoPE score of the tile, shared by every branch
-                                const uint32_t dRt = tmem + C::R_COL0 + (tc & 1) * kHP;
-#pragma unroll
-                                for (int kk = 0; kk < DR / 16; ++kk)
-                                    if (elect_one()) mma_bf16(dRt, dRs + kk * 2, dQR + kk * 2, IDESC_S, kk ? 1u : 0u);
-                                if (elect_one()) mma_commit(&misc.rope_empty[0]);
-                                __syncwarp();
-                            }
-                            const uint32_t dS = tmem + C::S_COL0 + (gs & 1) * C::S_SLOT_COLS;
-                            // this step's branches start at chunk st*G*(DC/64) of the token row
-                            const uint64_t dQs = dQ + ((st * C::SBR * (DC / 64) * C::Q_CHUNK_BYTES) >> 4);
-#pragma unroll
-                            for (int g = 0; g < C::SBR; ++g) {
-#pragma unroll
-                                for (int c = 0; c < DC / 64; ++c) {
-                                    // chunk (g*(DC/64) + c) of this step: pair pp, half hf
-                                    const int lc = g * (DC / 64) + c;
-                                    const int pp = lc / 2, hf = lc % 2;
-                                    uint32_t sp = stage0 + pp;
-                                    if (sp >= (uint32_t)C::NSTAGE) sp -= C::NSTAGE;
-                                    const uint64_t a0 = dA_s + ((sp * C::PAIR_BYTES + hf * C::CHUNK_BYTES) >> 4);
-                                    const uint64_t q0 = dQs + ((lc * C::Q_CHUNK_BYTES) >> 4);
-#pragma unroll
-                                    for (int kk = 0; kk < 4; ++kk)
-                                        if (elect_one())
-                                            mma_bf16(dS + g * kHP, a0 + kk * 2, q0 + kk * 2, IDESC_S, (c | kk) ? 1u : 0u);
-                                }
-                            }
-                            if (elect_one()) mma_commit(&misc.s_full[gs & 1]);
-                            __syncwarp();
-                            if (C::OVERLAP) {
-                                if (have_prev) ok = issue_pv(prev_gs, prev_st, prev_stage, prev_first);
-                                have_prev = true;
-                                prev_gs = gs;
-                                prev_st = st;
-                                prev_stage = stage0;
-                                prev_first = (j == tb);
-                            } else {
-                                ok = issue_pv(gs, st, stage0, j == tb);
-                            }
-                            ++gs;
                         }
-                        ++tc;
-                        if (__shfl_sync(0xffffffffu, *abort_flag, 0)) ok = false;
+                        // the S slot (and the P slot the softmax fills next) of
+                        // this step is free once the output MMA of step gs-2 is done
+                        if (ok && gs >= 2) ok = mbar_wait_warp(&misc.p_empty[gs & 1], ((gs >> 1) - 1) & 1);
+                        if (!ok) break;
+                        tc_fence_after();
+                        if (st == 0) {
+                            // RoPE score of the tile, shared by every branch
+                            const uint32_t dRt = tmem + C::R_COL0 + (tc & 1) * kHP;
+#pragma unroll
+                            for (int kk = 0; kk < DR / 16; ++kk)
+                                if (elect_one()) mma_bf16(dRt, dR + kk * 2, dQR + qoff + kk * 2, IDESC_S, kk ? 1u : 0u);
+                            if (elect_one()) mma_commit(&misc.rope_empty[0]);
+                            __syncwarp();
+                        }
+                        const uint32_t dS = tmem + C::S_COL0 + (gs & 1) * C::S_SLOT_COLS;
+                        // this step's branches start at chunk st*SBR*(DC/64) of the token row
+                        const uint64_t dQs = dQ + qoff + ((st * C::SBR * (DC / 64) * C::Q_CHUNK_BYTES) >> 4);
+#pragma unroll
+                        for (int g = 0; g < C::SBR; ++g) {
+#pragma unroll
+                            for (int c = 0; c < DC / 64; ++c) {
+                                // chunk (g*(DC/64) + c) of this step: pair pp, half hf
+                                const int lc = g * (DC / 64) + c;
+                                const int pp = lc / 2, hf = lc % 2;
+                                uint32_t sp = stage0 + pp;
+                                if (sp >= (uint32_t)C::NSTAGE) sp -= C::NSTAGE;
+                                const uint64_t a0 = dA_s + ((sp * C::PAIR_BYTES + hf * C::CHUNK_BYTES) >> 4);
+                                const uint64_t q0 = dQs + ((lc * C::Q_CHUNK_BYTES) >> 4);
+#pragma unroll
+                                for (int kk = 0; kk < 4; ++kk)
+                                    if (elect_one())
+                                        mma_bf16(dS + g * kHP, a0 + kk * 2, q0 + kk * 2, IDESC_S, (c | kk) ? 1u : 0u);
+                            }
+                        }
+                        if (elect_one()) mma_commit(&misc.s_full[gs & 1]);
+                        __syncwarp();
+                        ++gs;
                     }
-                    if (ok && have_prev) ok = issue_pv(prev_gs, prev_st, prev_stage, prev_first);
-                    have_prev = false;
-                    if (ok && elect_one()) mma_commit(&misc.seg_done);
-                    __syncwarp();
-                    ++sc;
-                    finish_segment(n, cum, tiles);
+                    ++tc;
+                    if (__shfl_sync(0xffffffffu, *abort_flag, 0)) ok = false;
                 }
-                if (!ok && lane == 0) {
-                    record_error(a.err, MLRA_ERR_DEVICE_TIMEOUT);
-                    *abort_flag = 1;
-                }
-                // drain: every MMA issued above completes before TMEM is freed
-                if (elect_one()) mma_commit(&misc.drain);
+                // the queries' slot is free once this range's score MMAs finish
+                if (ok && elect_one()) mma_commit(&misc.q_empty[sc & 1]);
                 __syncwarp();
-                mbar_wait(&misc.drain, 0, 200000000ull);
+                ++sc;
+                finish_segment(n, cum, tiles);
             }
+            if (!ok && lane == 0) {
+                record_error(a.err, MLRA_ERR_DEVICE_TIMEOUT);
+                *abort_flag = 1;
+            }
+            // drain: every MMA issued above completes before TMEM is freed
+            if (elect_one()) mma_commit(&misc.drain[0]);
+            __syncwarp();
+            mbar_wait(&misc.drain[0], 0, 200000000ull);
+            __syncwarp();
+        } else if (warp == 6) {
+            // ------------------------------------------------------------ output MMA issuer
+            constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, kHP, true, true);
+            const uint32_t sm_base = smem_u32(sm);
+            const uint64_t dA_pv = smem_desc(sm_base + C::OFF_PAIR, C::CHUNK_BYTES, 1024, kLayoutSw128);  // MN-major
+            const uint64_t dP = smem_desc(sm_base + C::OFF_P, 128, 2048, kLayoutNone);
+            int n = misc.plan[2], cum = misc.plan[3], next_len = first_len(a, n);
+            int L, tiles, tb, te;
+            uint32_t gs = 0;
+            uint32_t stage = 0;  // ring position of the step's first pair
+            bool ok = true;
+            while (ok && next_segment(a, n, cum, A0, A1, L, tiles, tb, te, next_len)) {
+                for (int j = tb; j < te && ok; ++j) {
+#pragma unroll 1
+                    for (int st = 0; st < C::NSTEP; ++st) {
+                        ok = mbar_wait_warp(&misc.p_full[gs & 1], (gs >> 1) & 1);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint64_t b0 = dP + ((gs & 1) * C::P_BYTES >> 4);
+#pragma unroll
+                        for (int p = 0; p < C::PPS; ++p) {
+                            uint32_t sp = stage + p;
+                            if (sp >= (uint32_t)C::NSTAGE) sp -= C::NSTAGE;
+                            const uint64_t a0 = dA_pv + ((sp * C::PAIR_BYTES) >> 4);
+#pragma unroll
+                            for (int g2 = 0; g2 < C::BPP; ++g2) {
+                                // branch of the step whose P multiplies this pair (rows of the
+                                // other branch of a shared pair are discarded later)
+                                const int gl = DC >= 128 ? p * 128 / DC : p * C::BPP + g2;
+                                const uint32_t d = tmem + ((st * C::PPS + p) * C::BPP + g2) * kHP;
+#pragma unroll
+                                for (int kt = 0; kt < kT / 16; ++kt)
+                                    if (elect_one())
+                                        mma_bf16(d, a0 + (kt * 2048 >> 4), b0 + ((gl * C::P_BRANCH_BYTES + kt * 256) >> 4),
+                                                 IDESC_PV, (j == tb && kt == 0) ? 0u : 1u);
+                            }
+                        }
+#pragma unroll
+                        for (int p = 0; p < C::PPS; ++p) {
+                            uint32_t sp = stage + p;
+                            if (sp >= (uint32_t)C::NSTAGE) sp -= C::NSTAGE;
+                            if (elect_one()) mma_commit(&misc.pair_empty[sp]);
+                        }
+                        if (elect_one()) mma_commit(&misc.p_empty[gs & 1]);
+                        __syncwarp();
+                        stage += C::PPS;
+                        if (stage >= (uint32_t)C::NSTAGE) stage -= C::NSTAGE;
+                        ++gs;
+                    }
+                    if (__shfl_sync(0xffffffffu, *abort_flag, 0)) ok = false;
+                }
+                finish_segment(n, cum, tiles);
+            }
+            if (!ok && lane == 0) {
+                record_error(a.err, MLRA_ERR_DEVICE_TIMEOUT);
+                *abort_flag = 1;
+            }
+            if (elect_one()) mma_commit(&misc.drain[1]);
+            __syncwarp();
+            mbar_wait(&misc.drain[1], 0, 200000000ull);
             __syncwarp();
         } else {
             // ------------------------------------------------------------ softmax + epilogue
@@ -501,7 +707,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
             const int stid = threadIdx.x - 64;         // 0..127 within the group
             const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
             const int H = a.heads;
-            int n = misc.plan[2], cum = misc.plan[3];
+            int n = misc.plan[2], cum = misc.plan[3], next_len = first_len(a, n);
             int L, tiles, tb, te;
             uint32_t gs = 0, sc = 0, tcnt = 0;  // steps, ranges, tiles so far
             // This thread's share of the softmax denominators, one row per
@@ -509,44 +715,14 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
             // rotate by G so that the current step's branches are rows 0..G-1.
             float l[NB][kHP];
             bool dead = false;
+            int pend_a = -1, pend_b = -1;  // split ranges not yet counted (thread stid 0)
 
-            while (!dead && next_segment(a, n, cum, A0, A1, L, tiles, tb, te)) {
-                // queries of sequence n -> shared memory (128-byte swizzled, K-major)
-                {
-                    const uint4* q_src = reinterpret_cast<const uint4*>(a.q_lat + (size_t)n * H * C::W);
-                    constexpr int UPR = C::W / 8;  // 16-byte units per head row
-                    for (int i = stid; i < kHP * UPR; i += 128) {
-                        const int h = i / UPR, rem = i % UPR, gc = rem / 8, u = rem % 8;
-                        uint4 v = make_uint4(0, 0, 0, 0);
-                        if (h < H) v = __ldg(q_src + (size_t)h * UPR + rem);
-                        *reinterpret_cast<uint4*>(sm + C::OFF_Q + gc * C::Q_CHUNK_BYTES + h * 128 +
-                                                  ((u ^ (h & 7)) << 4)) = v;
-                    }
-                    const uint4* qr_src = reinterpret_cast<const uint4*>(a.q_rope + (size_t)n * H * DR);
-                    constexpr int RU = DR / 8;
-                    for (int i = stid; i < kHP * RU; i += 128) {
-                        const int h = i / RU, u = i % RU;
-                        uint4 v = make_uint4(0, 0, 0, 0);
-                        if (h < H) v = __ldg(qr_src + (size_t)h * RU + u);
-                        const int sw = DR == 64 ? (u ^ (h & 7)) : (u ^ ((h >> 1) & 3));
-                        *reinterpret_cast<uint4*>(sm + C::OFF_QR + h * C::ROPE_ROW + (sw << 4)) = v;
-                    }
-                }
-                // block-table entries of this range must name real pages
+            while (!dead && next_segment(a, n, cum, A0, A1, L, tiles, tb, te, next_len)) {
+                // block-table entries of the range must name real pages: each
+                // thread checks its own token's page once per tile (the load is
+                // issued at the tile's start and consumed at its end)
                 bool bad = false;
-                {
-                    const int32_t* bt = a.block_table + (size_t)n * a.max_pages;
-                    const int p0 = tb * kT / P, p1 = ceil_div(min(te * kT, L), P);
-                    for (int i = p0 + stid; i < p1; i += 128) {
-                        const int v = __ldg(bt + i);
-                        bad |= (v < 0 || v >= a.num_pages);
-                    }
-                }
-                bad = named_bar_or<1, 128>(bad);
-                fence_proxy_async_smem();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&misc.q_full);
+                const int32_t* bt = a.block_table + (size_t)n * a.max_pages;
 #pragma unroll
                 for (int b = 0; b < NB; ++b)
 #pragma unroll
@@ -555,6 +731,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                 for (int j = tb; j < te && !dead; ++j) {
                     const int valid = min(kT, L - j * kT);
                     const bool masked = row >= valid;
+                    const int page = masked ? 0 : __ldg(bt + (j * kT + row) / P);
                     float r[kHP];  // this token's RoPE score per head, shared by the tile's branches
 #pragma unroll 1
                     for (int st = 0; st < C::NSTEP; ++st) {
@@ -636,7 +813,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                             if (j > tb) {
                                 // O holds earlier tiles of this range: rescale it once the
                                 // previous output MMA has finished
-                                const bool ok2 = mbar_wait(&misc.o_done, (gs - 1) & 1);
+                                const bool ok2 = mbar_wait(&misc.p_empty[(gs - 1) & 1], ((gs - 1) >> 1) & 1);
                                 if (named_bar_or<1, 128>(!ok2)) {
                                     dead = true;
                                     break;
@@ -709,6 +886,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                         }
                         ++gs;
                     }
+                    bad |= page < 0 || page >= a.num_pages;
                     ++tcnt;
                 }
                 if (dead) break;
@@ -732,7 +910,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                         if ((lane & 1) == 0) misc.red_sum[quad][lane >> 1] = f[0];
                     }
                 }
-                named_bar_sync<1, 128>();
+                bad = named_bar_or<1, 128>(bad);  // also publishes red_sum
                 int first_cta, last_cta;
                 seq_owners(cum, tiles, chunk, &first_cta, &last_cta);
                 const bool single = first_cta == last_cta;
@@ -745,11 +923,9 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                     if (!single && i < H)
                         a.lse_part[(slot * NB + b) * H + i] = bad ? bad_split_marker() : misc.m_run[stid] + __log2f(lt);
                 }
-                // the range's own barrier: two output MMAs may be in flight, so
-                // o_done's parity cannot tell them apart (the barrier below also
-                // publishes inv_l)
+                // the range's last output MMA (the barrier below also publishes inv_l)
                 {
-                    const bool ok = mbar_wait(&misc.seg_done, sc & 1);
+                    const bool ok = mbar_wait(&misc.p_empty[(gs - 1) & 1], ((gs - 1) >> 1) & 1);
                     if (named_bar_or<1, 128>(!ok)) {
                         dead = true;
                         break;
@@ -791,12 +967,28 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
                 if (bad && stid == 0) record_error(a.err, MLRA_ERR_DEVICE_BAD_INDEX);
                 tc_fence_before();
                 named_bar_sync<1, 128>();  // inv_l and red_sum are reused by the next range
+                if (stid == 0) {
+                    // a split's partials are complete: counted for the merge when
+                    // this CTA's work ends (only its first and last ranges can be
+                    // splits, and their merges wait for the kernel's end anyway)
+                    if (!single) {
+                        if (pend_a < 0) pend_a = n; else pend_b = n;
+                    }
+                    misc.last_seg[0] = n;
+                    misc.last_seg[1] = cum;
+                    misc.last_seg[2] = tiles;
+                }
                 ++sc;
                 finish_segment(n, cum, tiles);
             }
             if (dead && stid == 0) {
                 record_error(a.err, MLRA_ERR_DEVICE_TIMEOUT);
                 *abort_flag = 1;
+            }
+            if (!dead && stid == 0 && pend_a >= 0) {
+                __threadfence();
+                red_add_release_gpu(a.seq_cnt + pend_a, 1);
+                if (pend_b >= 0) red_add_release_gpu(a.seq_cnt + pend_b, 1);
             }
         }
     }
@@ -805,6 +997,11 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const DecodeArgs a) {
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+    if (*abort_flag) return;
+    // the ring's shared memory is free from here on: the merge stages its
+    // weights there
+    merge_tail<NB, DC>(a, misc.last_seg[0], misc.last_seg[1], misc.last_seg[2], chunk,
+                       reinterpret_cast<float*>(sm + C::OFF_PAIR), &misc.merge_flag, &misc.merge_bar);
 }
 
 // ------------------------------------------------------------------ host side
@@ -833,6 +1030,19 @@ bool encode_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool encode_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+               uint32_t box_inner, uint32_t box_mid, CUtensorMapSwizzle swizzle) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[3] = {inner, mid, outer};
+    const cuuint64_t strides[2] = {inner * 2, inner * mid * 2};
+    const cuuint32_t box[3] = {box_inner, box_mid, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int NB, int DC, int DR>
 cudaError_t launch_cfg(const DecodeArgs& a, cudaStream_t stream) {
     using C = Cfg<NB, DC, DR>;
@@ -841,13 +1051,33 @@ cudaError_t launch_cfg(const DecodeArgs& a, cudaStream_t stream) {
     const uint32_t box_rows = (uint32_t)a.page_size;
     if (!encode_2d(&maps.lat, a.latent, (uint64_t)C::W, rows, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_2d(&maps.rope, a.rope, (uint64_t)DR, rows, DR, box_rows,
+                   DR == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !encode_3d(&maps.q, a.q_lat, (uint64_t)C::W, (uint64_t)a.heads, (uint64_t)a.batch, 64, kHP,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_3d(&maps.qr, a.q_rope, (uint64_t)DR, (uint64_t)a.heads, (uint64_t)a.batch, DR, kHP,
                    DR == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
     auto kernel = decode_tc_kernel<NB, DC, DR>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kernel<<<a.num_ctas, kThreads, C::SMEM_BYTES, stream>>>(maps, a);
-    return cudaGetLastError();
+    // the merge stages in the ring: the weights of all S <= grid splits of a
+    // sequence and S row slices of at most R / (S - 1) + 1 rows of 64 bytes
+    if ((size_t)a.num_ctas * NB * kHP * sizeof(float) + (2 * (size_t)C::W + a.num_ctas) * kHP * sizeof(float) >
+        (size_t)C::NSTAGE * C::PAIR_BYTES)
+        return cudaErrorInvalidConfiguration;
+    // Cooperative: every CTA is resident at once, so the merge's wait for the
+    // other splits of a sequence always ends.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.num_ctas);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, maps, a);
 }
 
 }  // namespace

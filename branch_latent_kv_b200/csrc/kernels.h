@@ -18,8 +18,9 @@ struct DecodeArgs {
     const int32_t* seqlens;       // [N]
     __nv_bfloat16* out;           // [N, H, B, d_c]
     float* lse_part;              // [slots, B, H]        log2 domain
-    float* o_part;                // [slots, B, H, d_c]
+    float* o_part;                // [slots, B, d_c, HP]   HP = partial_heads(H)
     int* err;                     // device error word
+    int* seq_cnt;                 // [N] split counters of the in-kernel merge (zero between calls)
     int batch, heads, branches, d_c, d_r, page_size, max_pages, num_pages;
     int num_ctas;                 // grid of the split kernel (partial slots = num_ctas + batch)
     float scale_log2;             // scale * log2(e)

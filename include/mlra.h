@@ -78,9 +78,13 @@ typedef struct {
  * `num_ctas` CTAs; num_ctas <= 0 means "the current device's SM count"
  * (the grid mlra_decode launches).  Pure host computation (the SM count query
  * is the only CUDA call).  Returns 0 if dims are invalid.
- * The workspace holds the split-KV partial outputs (fp32), their
- * log-sum-exps and the device error word.  Zero it once before first use
- * (the error word must start at 0); mlra_decode never needs it re-zeroed.
+ * The workspace holds the device error word, a split counter per sequence
+ * (a fixed 256 KB region, so a workspace can serve calls with different
+ * dims), the split-KV partial outputs (fp32) and their log-sum-exps.
+ * Zero it once before first use (the error word and the counters must start
+ * at 0).  Every call that ends without MLRA_ERR_DEVICE_TIMEOUT leaves the
+ * counters at 0 again, so it never needs re-zeroing; after a timeout, zero it
+ * before the next call.
  */
 MLRA_API size_t mlra_decode_workspace_bytes(const mlra_dims* dims, int32_t num_ctas);
 
@@ -108,12 +112,14 @@ MLRA_API size_t mlra_decode_workspace_bytes(const mlra_dims* dims, int32_t num_c
  *   workspace    device buffer of >= mlra_decode_workspace_bytes(dims, 0)
  *                bytes, zeroed before its first use; one call at a time
  *
- * Runs on the tensor cores (tcgen05, operands staged by TMA).  Supported
+ * Runs on the tensor cores (tcgen05, operands staged by TMA) as one
+ * cooperative kernel (one CTA per SM, all resident; the CTAs that share a
+ * sequence merge their partials at the end).  Supported
  * shapes: heads <= 16; (branches, d_c) in {(2,64), (4,64), (1,128), (2,128),
  * (4,128), (1,256), (2,256), (1,512)}; d_r in {32, 64}; page_size in
  * {16, 32, 64, 128}.  Other shapes return MLRA_ERR_UNSUPPORTED
  * (mlra_decode_simt covers more).
- * Returns MLRA_OK once the kernels are enqueued.
+ * Returns MLRA_OK once the kernel is enqueued.
  */
 MLRA_API mlra_status mlra_decode(const mlra_dims* dims, const void* q_lat, const void* q_rope,
                         const void* latent_cache, const void* rope_cache,
@@ -155,8 +161,9 @@ MLRA_API mlra_status mlra_decode_simt(const mlra_dims* dims, const void* q_lat, 
  * It allocates and frees nothing.  All calls on a device share the array:
  * calls that may overlap on the GPU race and corrupt each other's results,
  * so order them on one stream.  The array keeps the last call's contents;
- * the only part that must start at zero (the error word) starts zeroed and
- * is cleared again at the end of every call.  The first call on each device
+ * the parts that must start at zero (the error word and the split counters)
+ * start zeroed; the error word is cleared again at the end of every call and
+ * the counters return to zero unless the call reports a device timeout.  The first call on each device
  * looks up the array's address with that device current; make it before any
  * stream capture starts.
  */

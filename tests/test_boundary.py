@@ -52,7 +52,8 @@ def test_workspace_bytes_layout():
 
     def a256(x):
         return (x + 255) // 256 * 256
-    lse_off = 256                           # after the error word
+    cnt_off = 256                           # after the error word: split counters
+    lse_off = a256(cnt_off + 4 * 65536)     # sized for the largest batch
     o_off = a256(lse_off + 4 * slots * 4 * 16)
     assert n == a256(o_off + 4 * slots * 4 * 128 * 16)  # partial rows padded to 16 heads
     assert b.library().mlra_decode_workspace_bytes(ctypes.byref(_dims(batch=0)), 148) == 0

@@ -158,6 +158,28 @@ def test_repeat_calls_are_deterministic():
         assert torch.equal(_run(x), a)
 
 
+def _split_counters(ws, dims):
+    """The per-sequence split counters: int32 from byte 256 of the workspace
+    (after the error word), one per sequence."""
+    return ws[256:256 + 4 * dims.batch].view(torch.int32)
+
+
+@pytest.mark.parametrize("seqlens", [[131072], [9000, 1, 300, 130000, 128, 129], [64] * 300])
+def test_split_merge_leaves_counters_at_zero(oracle_lib, seqlens):
+    w = WORKLOADS["decode_2p9b"].with_(batch=len(seqlens), seqlen=None)
+    x = make_inputs(w, seed=7, seqlens=torch.tensor(seqlens, dtype=torch.int32),
+                    max_pages_per_seq=max(seqlens) // w.page_size + 1).to("cuda")
+    dims = b.decode_dims(x.q_lat, x.q_rope, x.latent_cache, x.block_table)
+    ws = torch.zeros(b.mlra_decode_workspace_bytes(dims), dtype=torch.uint8, device="cuda")
+    first = _run(x, workspace=ws).clone()
+    assert (_split_counters(ws, dims) == 0).all()
+    assert torch.equal(_run(x, workspace=ws), first)
+    assert b.mlra_read_device_error(ws) == b.MLRA_OK
+    ids = sorted({0, len(seqlens) - 1, len(seqlens) // 2})
+    ref, _ = _oracle(oracle_lib, x, seq_ids=ids)
+    _assert_close(first, ref, seq_ids=ids, what=f"merge {seqlens[:4]}")
+
+
 def test_invalid_sequences_are_zeroed_and_reported(oracle_lib):
     w = WORKLOADS["decode_2p9b"].with_(batch=4, seqlen=None)
     seqlens = torch.tensor([500, 700, 900, 300], dtype=torch.int32)
