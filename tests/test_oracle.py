@@ -188,6 +188,25 @@ def test_lse_is_logsumexp_of_scores(oracle_lib):
             assert lse[0, h, b] == pytest.approx(logsumexp(s), rel=1e-13)
 
 
+def test_two_way_split_merged_by_logsumexp_equals_the_whole(oracle_lib):
+    """Attention over tokens [0, L) equals the log-sum-exp weighted merge of
+    the attentions over [0, L1) and [L1, L) (the split-KV identity)."""
+    rng = np.random.default_rng(13)
+    B, d_c, d_r, P, L, L1 = 2, 8, 4, 4, 23, 10
+    lat, rope = _logical(rng, [L], B, d_c, d_r)
+    lat3 = [lat[0], lat[0][:L1], lat[0][L1:]]
+    rope3 = [rope[0], rope[0][:L1], rope[0][L1:]]
+    q_lat, q_rope = _queries(rng, 1, 3, B, d_c, d_r, gain=8.0)
+    q_lat3, q_rope3 = np.repeat(q_lat, 3, axis=0), np.repeat(q_rope, 3, axis=0)
+    pool, rpool, table, seqlens = paged_from_logical(lat3, rope3, P, rng)
+    out, lse, status = oracle_lib.decode(q_lat3, q_rope3, pool, rpool, table, seqlens, 0.7, 0.5)
+    assert status == 0
+    w1, w2 = np.exp(lse[1] - lse[0]), np.exp(lse[2] - lse[0])
+    merged = w1[..., None] * out[1] + w2[..., None] * out[2]
+    np.testing.assert_allclose(merged, out[0], rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(np.logaddexp(lse[1], lse[2]), lse[0], rtol=1e-13)
+
+
 def test_up_proj_is_the_concatenated_gemm(oracle_lib):
     """sum over branches of per-branch products == one GEMM over K = B*d_c."""
     rng = np.random.default_rng(10)
