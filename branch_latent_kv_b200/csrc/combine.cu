@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(DecodeArgs a) {
     // all S x H log-sum-exps in one round of independent loads
     for (int e = tid; e < S * HP; e += kThreads) {
         const int s = e / HP, h = e % HP;
-        w_s[e] = h < H ? __ldg(a.lse_part + ((size_t)(c0 + s + n) * B + b) * H + h) : -INFINITY;
+        w_s[e] = h < H ? __ldg(a.lse_part + ((size_t)(c0 + s + n) * B + b) * partial_heads(H) + h) : -INFINITY;
     }
     __syncthreads();
     // weights per head: 2^(lse - max) * out_scale / sum (one warp per head)

@@ -21,7 +21,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 // ---------------------------------------------------------------------------
 // Workspace layout (byte offsets, each region 256-byte aligned):
 //   [0, 256)        int32 error word (first device-side error code, else 0)
-//   lse partials    fp32 [slots][branches][heads]      (log2 domain)
+//   lse partials    fp32 [slots][branches][HP]         (log2 domain; HP = 16,
+//                   or the head count when above 16: 64-byte rows)
 //   o partials      fp32 [slots][branches][d_c][16]    (normalised per split;
 //                   heads innermost, padded to 16: one 64-byte row per column)
 // slots = num_ctas + batch: the partial of CTA c for sequence n lives in slot
@@ -47,8 +48,8 @@ __host__ __device__ inline WorkspaceLayout workspace_layout(int batch, int heads
     // that reuse the workspace find them where they left them (at zero)
     w.cnt_off = 256;
     w.lse_off = align256(w.cnt_off + sizeof(int) * (size_t)(kMaxBatch + 1));
-    w.o_off = align256(w.lse_off + sizeof(float) * (size_t)w.slots * branches * heads);
     const size_t hp = heads <= 16 ? 16 : (size_t)heads;  // heads padded to 16 (more for the CUDA-core kernel)
+    w.o_off = align256(w.lse_off + sizeof(float) * (size_t)w.slots * branches * hp);
     w.total = align256(w.o_off + sizeof(float) * (size_t)w.slots * branches * d_c * hp);
     return w;
 }

@@ -201,7 +201,7 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
             }
             for (int hb = tid; hb < HB; hb += kThreads) {
                 const int h = hb / B, b = hb % B;
-                a.lse_part[(slot * B + b) * H + h] =
+                a.lse_part[(slot * B + b) * partial_heads(H) + h] =
                     bad ? bad_split_marker() : m_s[hb] + log2f(l_s[hb]);
             }
         }

@@ -78,32 +78,39 @@ struct Cfg {
     static constexpr int P_BRANCH_BYTES = kT * kHP * 2;     // 4 KB
     static constexpr int P_BYTES = SBR * P_BRANCH_BYTES;   // one P slot (a step)
     static constexpr int MISC_BYTES = 4096;
-    static constexpr int QSET_BYTES = Q_BYTES + QR_SPAN;  // one sequence's queries (two slots)
-    static constexpr int FIXED = ROPE_BYTES + 2 * QSET_BYTES + 2 * P_BYTES + MISC_BYTES;
+    static constexpr int QSET_BYTES = Q_BYTES + QR_SPAN;  // one sequence's queries
+    // Pipeline depths: NSP steps may be between their score MMA and their
+    // output MMA at once (S slots in TMEM, P slots in shared memory); NROPE
+    // RoPE tiles are in flight, so the producer never waits for a tile's RoPE
+    // score before it loads the next tile; one query set (a sequence change
+    // waits for the previous range's score MMAs, rare: at most two per CTA).
+    static constexpr int NSP = 3;
+    static constexpr int NROPE = 2;
+    static constexpr int FIXED = NROPE * ROPE_BYTES + QSET_BYTES + NSP * P_BYTES + MISC_BYTES;
     static constexpr int NSTAGE_FIT = (kSmemLimit - 1024 - FIXED) / PAIR_BYTES;
     static constexpr int NSTAGE = NSTAGE_FIT > 8 ? 8 : NSTAGE_FIT;
     // shared-memory offsets from a 1024-byte aligned base
     static constexpr int OFF_PAIR = 0;
-    static constexpr int OFF_ROPE = OFF_PAIR + NSTAGE * PAIR_BYTES;
-    static constexpr int OFF_Q = OFF_ROPE + ROPE_BYTES;  // one RoPE tile: its only reader runs at step 0
-    static constexpr int OFF_QR = OFF_Q + Q_BYTES;       // slot s at + s * QSET_BYTES
-    static constexpr int OFF_P = OFF_Q + 2 * QSET_BYTES;
-    static constexpr int OFF_MISC = OFF_P + 2 * P_BYTES;
+    static constexpr int OFF_ROPE = OFF_PAIR + NSTAGE * PAIR_BYTES;  // RoPE slot r at + r * ROPE_BYTES
+    static constexpr int OFF_Q = OFF_ROPE + NROPE * ROPE_BYTES;
+    static constexpr int OFF_QR = OFF_Q + Q_BYTES;
+    static constexpr int OFF_P = OFF_Q + QSET_BYTES;                  // P slot k at + k * P_BYTES
+    static constexpr int OFF_MISC = OFF_P + NSP * P_BYTES;
     static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
     // TMEM columns: O blocks first, then two S slots, then two slots of the
     // RoPE score shared by all branches of a tile
     static constexpr int O_BLOCKS = NPAIR * BPP;
     static constexpr int S_COL0 = O_BLOCKS * kHP;
     static constexpr int S_SLOT_COLS = SBR * kHP;
-    static constexpr int R_COL0 = S_COL0 + 2 * S_SLOT_COLS;
+    static constexpr int R_COL0 = S_COL0 + NSP * S_SLOT_COLS;
     static constexpr int TMEM_COLS = R_COL0 + 2 * kHP <= 128 ? 128 : 256;
     static_assert(NB % SBR == 0 && (SBR * DC) % 128 == 0, "branches must fill whole steps and pairs");
     static_assert(NSTEP * PPS == NPAIR, "step / pair bookkeeping");
     static_assert(NSTAGE >= PPS, "a step's pairs must fit the stage ring");
     static_assert(R_COL0 + 2 * kHP <= TMEM_COLS, "TMEM budget");
     static_assert(SMEM_BYTES <= kSmemLimit, "shared-memory budget");
-    static_assert(OFF_QR + QSET_BYTES + QR_BYTES <= OFF_P && OFF_Q + Q_BYTES <= OFF_QR &&
-                  OFF_P + 2 * P_BYTES <= OFF_MISC && QSET_BYTES % 1024 == 0,
+    static_assert(OFF_QR + QR_BYTES <= OFF_P && OFF_Q + Q_BYTES <= OFF_QR &&
+                  OFF_P + NSP * P_BYTES <= OFF_MISC && QSET_BYTES % 1024 == 0 && ROPE_BYTES % 1024 == 0,
                   "shared-memory regions must not overlap");
     static_assert(DR == 32 || DR == 64, "RoPE width");
 };
@@ -113,20 +120,19 @@ template <int NSTAGE>
 struct Misc {
     uint64_t pair_full[NSTAGE];
     uint64_t pair_empty[NSTAGE];
-    uint64_t rope_full[2];
-    uint64_t rope_empty[2];
-    uint64_t s_full[2];   // step g in slot g & 1: its scores are in TMEM
-    uint64_t p_full[2];   // its probabilities are in shared memory
-    uint64_t p_empty[2];  // its output MMA finished (S and P slots free, O up to date)
-    uint64_t q_full[2];   // sequence range r in slot r & 1: its queries are in shared memory
-    uint64_t q_empty[2];  // its score MMAs finished
+    uint64_t rope_full[2];  // tile t in RoPE slot t & 1: its RoPE keys are in shared memory
+    uint64_t rope_empty[2];  // its RoPE score MMA finished
+    uint64_t s_full[3];   // step g in slot g % NSP: its scores are in TMEM
+    uint64_t p_full[3];   // its probabilities are in shared memory
+    uint64_t p_empty[3];  // its output MMA finished (S and P slots free, O up to date)
+    uint64_t q_full;      // sequence range r (phase r & 1): its queries are in shared memory
+    uint64_t q_empty;     // its score MMAs finished
     uint64_t drain[2];
     uint32_t tmem_base;
     int abort_flag;
     int plan[4];
     int last_seg[3];  // this CTA's last sequence range: sequence, cost start, tiles (-1: none)
-    int merge_flag;   // merge: bit 0 a split met a bad page, bit 1 the wait expired
-    uint64_t merge_bar;  // merge: the bulk copies of the partial slices
+    int merge_flag;   // merge: bit 0 a split met a bad page, bit 1 a wait expired
     float red_max[4][2 * kHP];
     float red_sum[4][4 * kHP];
     alignas(16) float m_run[8 * kHP];  // running max per (branch, head), base-2 logits; read as float4
@@ -247,14 +253,17 @@ __device__ __forceinline__ void finish_segment(int& n, int& cum, int tiles) {
 // (branch, latent column) rows, i = c - c0, G the group size:
 //   o = out_scale * sum_s w_s o_s / sum_s w_s,  w_s = 2^(lse_s - max_s lse_s)
 // per (branch, head) -- the log-sum-exp merge of independent softmax
-// partitions.  The last of the S + G counts returns seq_cnt[n] to zero.
+// partitions.  Every split's log-sum-exp row and its slice of partial rows
+// are fetched together (one round of L2 loads).  The last of the S + G
+// counts returns seq_cnt[n] to zero.
 template <int NB, int DC>
 __device__ __forceinline__ void merge_tail(const DecodeArgs& a, int n, int cum, int tiles, int chunk,
-                                        float* w_s, int* flag, uint64_t* bar) {
-    constexpr int HB = NB * kHP;  // (branch, head) weights per split
+                                           float* w_s, float* red, int* flag) {
+    constexpr int HB = NB * kHP;  // (branch, head) columns of a split's log-sum-exp row
     constexpr int R = NB * DC;    // (branch, latent column) rows
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     const int H = a.heads;
+    static_assert(kThreads >= HB && kThreads / HB * HB <= 4 * 64, "merge reduction scratch");
 
     // invalid lengths: zeros and an error code, sequence m by CTA m mod grid
     const int next_len = (n >= 0 && n + 1 < a.batch) ? __ldg(a.seqlens + n + 1) : 0;
@@ -280,9 +289,8 @@ __device__ __forceinline__ void merge_tail(const DecodeArgs& a, int n, int cum, 
     }
     const int G = c1_member ? S : S - 1;
     const int gi = blockIdx.x - c0;  // 0 <= gi < G: n is this CTA's last sequence
-    // this CTA's rows; a work item is (row, head quad), quads fastest so that
-    // each split's loads are contiguous 16-byte units
     const int r0 = (int)((long long)gi * R / G), r1 = (int)((long long)(gi + 1) * R / G);
+    const int rows = r1 - r0;
     // wait until every split of n has counted its partials
     if (tid == 0) {
         const uint64_t t0 = globaltimer_ns();
@@ -298,72 +306,83 @@ __device__ __forceinline__ void merge_tail(const DecodeArgs& a, int n, int cum, 
     __syncthreads();
     if (*flag & 2) return;
 
-    // this CTA's row slice of every split's partial -> shared memory by bulk
-    // copies (rows are contiguous within a slot), in flight while the weights
-    // are formed
-    const int rows = r1 - r0;
-    float* part_s = w_s + S * HB;  // [S][rows][16 heads]
-    if (warp == 0 && rows > 0) {
-        const uint32_t slice = (uint32_t)rows * kHP * 4;
-        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)S * slice);
-        __syncwarp();
-        for (int sp = lane; sp < S; sp += 32)
-            bulk_load(part_s + (size_t)sp * rows * kHP,
-                      a.o_part + ((size_t)(c0 + n + sp) * R + r0) * kHP, slice, bar);
-    }
-    // log-sum-exps -> shared memory, eight independent loads per thread at a time
-    const float* lse = a.lse_part;
-    for (int e0 = tid; e0 < S * HB; e0 += 8 * kThreads) {
-        float v[8];
+    // shared memory: w_s [S][HB] log-sum-exps (then weights), part_s
+    // [S][rows][16 heads] partial rows; slot of split s = c0 + s + n.  Every
+    // thread copies 16-byte units with L2 loads, sixteen in flight at a time
+    // (many small rows: plain loads keep far more requests in flight than
+    // one bulk copy per row would).
+    float* part_s = w_s + S * HB;
+    {
+        constexpr int LQ = HB / 4;               // 16-byte units per log-sum-exp row
+        const int lse_units = S * LQ;
+        const int row_units = rows * (kHP / 4);  // 16-byte units of one split's slice
+        const int total = lse_units + S * row_units;
+        for (int e0 = tid; e0 < total; e0 += 16 * kThreads) {
+            float4 v[16];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int e = e0 + j * kThreads, sp = e / HB, bh = e % HB, b = bh / kHP, h = bh % kHP;
-            v[j] = (e < S * HB && h < H) ? __ldcg(lse + ((size_t)(c0 + sp + n) * NB + b) * H + h) : 0.f;
+            for (int j = 0; j < 16; ++j) {
+                const int e = e0 + j * kThreads;
+                if (e < lse_units) {
+                    v[j] = __ldcg(reinterpret_cast<const float4*>(a.lse_part + (size_t)(c0 + n + e / LQ) * HB) + e % LQ);
+                } else if (e < total) {
+                    const int u = e - lse_units, sp = u / row_units, r = u % row_units;
+                    v[j] = __ldcg(reinterpret_cast<const float4*>(a.o_part + ((size_t)(c0 + n + sp) * R + r0) * kHP) + r);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int e = e0 + j * kThreads;
+                if (e < total) reinterpret_cast<float4*>(w_s)[e] = v[j];  // part_s follows w_s contiguously
+            }
         }
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            if (e0 + j * kThreads < S * HB) w_s[e0 + j * kThreads] = v[j];
     }
     __syncthreads();
-    // weights out_scale * 2^(lse - max) / sum per (branch, head): eight lanes
-    // per (branch, head), the splits strided over them
+    // weights out_scale * 2^(lse - max) / sum per (branch, head) column: TPC
+    // threads per column, each over every TPC-th split (consecutive threads
+    // take consecutive columns: conflict-free), partial maxima and sums
+    // combined through red[TPC][HB]
     {
-        const int sub = lane & 7;
-        for (int bh = warp * 4 + (lane >> 3); bh < HB; bh += (kThreads / 32) * 4) {
-            float mx = -INFINITY;
-            bool bad = false;
-            for (int sp = sub; sp < S; sp += 8) {
-                const float l = w_s[sp * HB + bh];
+        constexpr int TPC = kThreads / HB;
+        const int col = tid % HB, grp = tid / HB;
+        const bool act = grp < TPC;
+        float mx = -INFINITY;
+        bool bad = false;
+        if (act)
+            for (int sp = grp; sp < S; sp += TPC) {
+                const float l = w_s[sp * HB + col];
                 if (l == bad_split_marker()) bad = true; else mx = fmaxf(mx, l);
             }
-#pragma unroll
-            for (int o = 4; o > 0; o >>= 1) {
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                bad |= __shfl_xor_sync(0xffffffffu, (int)bad, o) != 0;
+        if (act) red[grp * HB + col] = bad ? bad_split_marker() : mx;
+        __syncthreads();
+        float M = -INFINITY;
+        bool bad_col = false;
+        if (act)
+            for (int g = 0; g < TPC; ++g) {
+                const float v = red[g * HB + col];
+                if (v == bad_split_marker()) bad_col = true; else M = fmaxf(M, v);
             }
-            float sum = 0.f;
-            for (int sp = sub; sp < S; sp += 8) {
-                const float w = bad ? 0.f : exp2f(w_s[sp * HB + bh] - mx);
-                w_s[sp * HB + bh] = w;
+        __syncthreads();
+        float sum = 0.f;
+        if (act) {
+            for (int sp = grp; sp < S; sp += TPC) {
+                const float w = bad_col ? 0.f : fast_exp2(w_s[sp * HB + col] - M);
+                w_s[sp * HB + col] = w;
                 sum += w;
             }
-#pragma unroll
-            for (int o = 4; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-            if (bad) {
-                if (sub == 0 && bh % kHP < H) atomicOr(flag, 1);
-            } else {
-                const float norm = a.out_scale / sum;
-                for (int sp = sub; sp < S; sp += 8) w_s[sp * HB + bh] *= norm;
-            }
+            red[grp * HB + col] = sum;
+        }
+        __syncthreads();
+        if (act) {
+            float total = 0.f;
+            for (int g = 0; g < TPC; ++g) total += red[g * HB + col];
+            const float norm = bad_col ? 0.f : a.out_scale / total;
+            for (int sp = grp; sp < S; sp += TPC) w_s[sp * HB + col] *= norm;
+            if (bad_col && grp == 0 && col % kHP < H) atomicOr(flag, 1);
         }
     }
     __syncthreads();
     const bool bad = *flag & 1;
     if (bad && tid == 0) record_error(a.err, MLRA_ERR_DEVICE_BAD_INDEX);
-    if (rows > 0 && !mbar_wait(bar, 0, 200000000ull)) {
-        if (tid == 0) record_error(a.err, MLRA_ERR_DEVICE_TIMEOUT);
-        return;
-    }
 
     // items (row, head quad), quads fastest: conflict-free 16-byte reads
     for (int e = tid; e < rows * 4; e += kThreads) {
@@ -398,6 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ DecodeArgs a) {
     using C = Cfg<NB, DC, DR>;
     using M = Misc<C::NSTAGE>;
+    static_assert(C::NSP <= 3 && C::NROPE == 2, "barrier arrays of Misc");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     M& misc = *reinterpret_cast<M*>(sm + C::OFF_MISC);
@@ -412,16 +432,15 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
         for (int i = 0; i < 2; ++i) {
             mbar_init(&misc.rope_full[i], 1);
             mbar_init(&misc.rope_empty[i], 1);
+            mbar_init(&misc.drain[i], 1);
+        }
+        for (int i = 0; i < C::NSP; ++i) {
             mbar_init(&misc.s_full[i], 1);
             mbar_init(&misc.p_full[i], 4);
             mbar_init(&misc.p_empty[i], 1);
-            mbar_init(&misc.drain[i], 1);
         }
-        mbar_init(&misc.q_full[0], 1);
-        mbar_init(&misc.q_full[1], 1);
-        mbar_init(&misc.q_empty[0], 1);
-        mbar_init(&misc.q_empty[1], 1);
-        mbar_init(&misc.merge_bar, 1);
+        mbar_init(&misc.q_full, 1);
+        mbar_init(&misc.q_empty, 1);
         misc.abort_flag = 0;
         misc.last_seg[0] = -1;
         misc.merge_flag = 0;
@@ -465,13 +484,13 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
             uint32_t pc = 0, tc = 0, sc = 0;
             bool ok = true;
             while (ok && next_segment(a, n, cum, A0, A1, L, tiles, tb, te, next_len)) {
-                // the sequence's queries into slot sc & 1, once the range two
-                // before has finished its score MMAs
+                // the sequence's queries, once the previous range has finished
+                // its score MMAs
                 if (lane == 0) {
-                    if (sc >= 2) ok = mbar_wait(&misc.q_empty[sc & 1], ((sc >> 1) - 1) & 1);
+                    if (sc >= 1) ok = mbar_wait(&misc.q_empty, (sc - 1) & 1);
                     if (ok) {
-                        uint64_t* qb = &misc.q_full[sc & 1];
-                        uint8_t* qd = sm + C::OFF_Q + (sc & 1) * C::QSET_BYTES;
+                        uint64_t* qb = &misc.q_full;
+                        uint8_t* qd = sm + C::OFF_Q;
                         mbar_arrive_expect_tx(qb, C::Q_BYTES + C::QR_BYTES);
                         for (int c = 0; c < C::NCHUNK; ++c)
                             tma_load_3d(qd + c * C::Q_CHUNK_BYTES, &maps.q, c * 64, 0, n, qb);
@@ -494,17 +513,18 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                         const int v = idx < a.max_pages ? __ldg(bt + idx) : 0;
                         win_val = (v >= 0 && v < a.num_pages) ? v : 0;  // bad entries are reported by the softmax warps
                     }
+                    const int rs = tc & 1;  // RoPE slot of this tile
                     if (lane == 0) {
-                        ok = mbar_wait(&misc.rope_empty[0], (tc & 1) ^ 1);
-                        if (ok) mbar_arrive_expect_tx(&misc.rope_full[0], npages * P * C::ROPE_ROW);
+                        if (tc >= 2) ok = mbar_wait(&misc.rope_empty[rs], ((tc >> 1) - 1) & 1);
+                        if (ok) mbar_arrive_expect_tx(&misc.rope_full[rs], npages * P * C::ROPE_ROW);
                     }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
                     for (int q = 0; q < npages; ++q) {
                         const int page = __shfl_sync(0xffffffffu, win_val, page0 + q - win_base);
                         if (lane == 0)
-                            tma_load_2d(sm + C::OFF_ROPE + q * P * C::ROPE_ROW, &maps.rope, 0, page * P,
-                                        &misc.rope_full[0]);
+                            tma_load_2d(sm + C::OFF_ROPE + rs * C::ROPE_BYTES + q * P * C::ROPE_ROW, &maps.rope,
+                                        0, page * P, &misc.rope_full[rs]);
                     }
                     ++tc;
                     for (int sp = 0; sp < C::NSTEP * C::PPS && ok; ++sp) {
@@ -544,11 +564,11 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                     const uint32_t k = pc - 1 - i;
                     mbar_wait(&misc.pair_full[k % C::NSTAGE], (k / C::NSTAGE) & 1, 200000000ull);
                 }
-                if (tc > 0) mbar_wait(&misc.rope_full[0], (tc - 1) & 1, 200000000ull);
-                for (uint32_t i = 0; i < 2u && i < sc; ++i) {
-                    const uint32_t k = sc - 1 - i;
-                    mbar_wait(&misc.q_full[k & 1], (k >> 1) & 1, 200000000ull);
+                for (uint32_t i = 0; i < 2u && i < tc; ++i) {
+                    const uint32_t k = tc - 1 - i;
+                    mbar_wait(&misc.rope_full[k & 1], (k >> 1) & 1, 200000000ull);
                 }
+                if (sc > 0) mbar_wait(&misc.q_full, (sc - 1) & 1, 200000000ull);
             }
         } else if (warp == 1) {
             // ------------------------------------------------------------ score MMA issuer
@@ -568,11 +588,10 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
             uint32_t stage = 0, phase = 0;  // ring position of the next pair to consume
             bool ok = true;
             while (ok && next_segment(a, n, cum, A0, A1, L, tiles, tb, te, next_len)) {
-                ok = mbar_wait_warp(&misc.q_full[sc & 1], (sc >> 1) & 1);
+                ok = mbar_wait_warp(&misc.q_full, sc & 1);
                 tc_fence_after();
-                const uint32_t qoff = ((sc & 1) * C::QSET_BYTES) >> 4;  // descriptor offset of the slot
                 for (int j = tb; j < te && ok; ++j) {
-                    ok = mbar_wait_warp(&misc.rope_full[0], tc & 1);
+                    ok = mbar_wait_warp(&misc.rope_full[tc & 1], (tc >> 1) & 1);
 #pragma unroll 1
                     for (int st = 0; st < C::NSTEP && ok; ++st) {
                         const uint32_t stage0 = stage;
@@ -585,21 +604,24 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                         }
                         // the S slot (and the P slot the softmax fills next) of
                         // this step is free once the output MMA of step gs-2 is done
-                        if (ok && gs >= 2) ok = mbar_wait_warp(&misc.p_empty[gs & 1], ((gs >> 1) - 1) & 1);
+                        const uint32_t slot = gs % C::NSP;
+                        if (ok && gs >= (uint32_t)C::NSP)
+                            ok = mbar_wait_warp(&misc.p_empty[slot], ((gs / C::NSP) - 1) & 1);
                         if (!ok) break;
                         tc_fence_after();
                         if (st == 0) {
                             // RoPE score of the tile, shared by every branch
                             const uint32_t dRt = tmem + C::R_COL0 + (tc & 1) * kHP;
+                            const uint64_t dRs = dR + (((tc & 1) * C::ROPE_BYTES) >> 4);
 #pragma unroll
                             for (int kk = 0; kk < DR / 16; ++kk)
-                                if (elect_one()) mma_bf16(dRt, dR + kk * 2, dQR + qoff + kk * 2, IDESC_S, kk ? 1u : 0u);
-                            if (elect_one()) mma_commit(&misc.rope_empty[0]);
+                                if (elect_one()) mma_bf16(dRt, dRs + kk * 2, dQR + kk * 2, IDESC_S, kk ? 1u : 0u);
+                            if (elect_one()) mma_commit(&misc.rope_empty[tc & 1]);
                             __syncwarp();
                         }
-                        const uint32_t dS = tmem + C::S_COL0 + (gs & 1) * C::S_SLOT_COLS;
+                        const uint32_t dS = tmem + C::S_COL0 + slot * C::S_SLOT_COLS;
                         // this step's branches start at chunk st*SBR*(DC/64) of the token row
-                        const uint64_t dQs = dQ + qoff + ((st * C::SBR * (DC / 64) * C::Q_CHUNK_BYTES) >> 4);
+                        const uint64_t dQs = dQ + ((st * C::SBR * (DC / 64) * C::Q_CHUNK_BYTES) >> 4);
 #pragma unroll
                         for (int g = 0; g < C::SBR; ++g) {
 #pragma unroll
@@ -617,7 +639,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                                         mma_bf16(dS + g * kHP, a0 + kk * 2, q0 + kk * 2, IDESC_S, (c | kk) ? 1u : 0u);
                             }
                         }
-                        if (elect_one()) mma_commit(&misc.s_full[gs & 1]);
+                        if (elect_one()) mma_commit(&misc.s_full[slot]);
                         __syncwarp();
                         ++gs;
                     }
@@ -625,7 +647,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                     if (__shfl_sync(0xffffffffu, *abort_flag, 0)) ok = false;
                 }
                 // the queries' slot is free once this range's score MMAs finish
-                if (ok && elect_one()) mma_commit(&misc.q_empty[sc & 1]);
+                if (ok && elect_one()) mma_commit(&misc.q_empty);
                 __syncwarp();
                 ++sc;
                 finish_segment(n, cum, tiles);
@@ -654,10 +676,11 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                 for (int j = tb; j < te && ok; ++j) {
 #pragma unroll 1
                     for (int st = 0; st < C::NSTEP; ++st) {
-                        ok = mbar_wait_warp(&misc.p_full[gs & 1], (gs >> 1) & 1);
+                        const uint32_t slot = gs % C::NSP;
+                        ok = mbar_wait_warp(&misc.p_full[slot], (gs / C::NSP) & 1);
                         if (!ok) break;
                         tc_fence_after();
-                        const uint64_t b0 = dP + ((gs & 1) * C::P_BYTES >> 4);
+                        const uint64_t b0 = dP + ((slot * C::P_BYTES) >> 4);
 #pragma unroll
                         for (int p = 0; p < C::PPS; ++p) {
                             uint32_t sp = stage + p;
@@ -682,7 +705,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                             if (sp >= (uint32_t)C::NSTAGE) sp -= C::NSTAGE;
                             if (elect_one()) mma_commit(&misc.pair_empty[sp]);
                         }
-                        if (elect_one()) mma_commit(&misc.p_empty[gs & 1]);
+                        if (elect_one()) mma_commit(&misc.p_empty[slot]);
                         __syncwarp();
                         stage += C::PPS;
                         if (stage >= (uint32_t)C::NSTAGE) stage -= C::NSTAGE;
@@ -735,13 +758,14 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                     float r[kHP];  // this token's RoPE score per head, shared by the tile's branches
 #pragma unroll 1
                     for (int st = 0; st < C::NSTEP; ++st) {
-                        const bool ok = mbar_wait(&misc.s_full[gs & 1], (gs >> 1) & 1);
+                        const uint32_t slot = gs % C::NSP;
+                        const bool ok = mbar_wait(&misc.s_full[slot], (gs / C::NSP) & 1);
                         tc_fence_after();
                         float x[C::SBR][kHP];
                         if (st == 0) tmem_ld16(tmem + lane_off + C::R_COL0 + (tcnt & 1) * kHP, r);
 #pragma unroll
                         for (int g = 0; g < C::SBR; ++g)
-                            tmem_ld16(tmem + lane_off + C::S_COL0 + (gs & 1) * C::S_SLOT_COLS + g * kHP, x[g]);
+                            tmem_ld16(tmem + lane_off + C::S_COL0 + slot * C::S_SLOT_COLS + g * kHP, x[g]);
                         tmem_wait_ld();
 #pragma unroll
                         for (int g = 0; g < C::SBR; ++g)
@@ -813,7 +837,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                             if (j > tb) {
                                 // O holds earlier tiles of this range: rescale it once the
                                 // previous output MMA has finished
-                                const bool ok2 = mbar_wait(&misc.p_empty[(gs - 1) & 1], ((gs - 1) >> 1) & 1);
+                                const bool ok2 = mbar_wait(&misc.p_empty[(gs - 1) % C::NSP], ((gs - 1) / C::NSP) & 1);
                                 if (named_bar_or<1, 128>(!ok2)) {
                                     dead = true;
                                     break;
@@ -836,7 +860,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                             }
                         }
                         // probabilities -> bf16 P (MN-major, 8x8 core matrices)
-                        uint8_t* p_slot = sm + C::OFF_P + (gs & 1) * C::P_BYTES;
+                        uint8_t* p_slot = sm + C::OFF_P + slot * C::P_BYTES;
 #pragma unroll
                         for (int g = 0; g < C::SBR; ++g) {
                             uint32_t packed[kHP / 2];
@@ -870,7 +894,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                         fence_proxy_async_smem();
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&misc.p_full[gs & 1]);
+                        if (lane == 0) mbar_arrive(&misc.p_full[slot]);
                         // rotate the denominator rows: the next step's branches first
 #pragma unroll
                         for (int r = 0; r < C::SBR; ++r) {
@@ -920,12 +944,12 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                                      misc.red_sum[3][stid];
                     misc.inv_l[stid] = 1.0f / lt;
                     const int b = stid / kHP, i = stid % kHP;
-                    if (!single && i < H)
-                        a.lse_part[(slot * NB + b) * H + i] = bad ? bad_split_marker() : misc.m_run[stid] + __log2f(lt);
+                    if (!single)  // all 16 columns (padded heads too): the merge reads whole rows
+                        a.lse_part[(slot * NB + b) * kHP + i] = bad ? bad_split_marker() : misc.m_run[stid] + __log2f(lt);
                 }
                 // the range's last output MMA (the barrier below also publishes inv_l)
                 {
-                    const bool ok = mbar_wait(&misc.p_empty[(gs - 1) & 1], ((gs - 1) >> 1) & 1);
+                    const bool ok = mbar_wait(&misc.p_empty[(gs - 1) % C::NSP], ((gs - 1) / C::NSP) & 1);
                     if (named_bar_or<1, 128>(!ok)) {
                         dead = true;
                         break;
@@ -1001,7 +1025,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
     // the ring's shared memory is free from here on: the merge stages its
     // weights there
     merge_tail<NB, DC>(a, misc.last_seg[0], misc.last_seg[1], misc.last_seg[2], chunk,
-                       reinterpret_cast<float*>(sm + C::OFF_PAIR), &misc.merge_flag, &misc.merge_bar);
+                       reinterpret_cast<float*>(sm + C::OFF_PAIR), &misc.red_sum[0][0], &misc.merge_flag);
 }
 
 // ------------------------------------------------------------------ host side
