@@ -72,15 +72,20 @@ __device__ __forceinline__ void record_error(int* err, int code) {
 // enters a new sequence.  Sequence n occupies the cost interval
 // [cum_n, cum_n + cost_n), cost_n = kTileCost * tiles_n + kSeqCost, and its
 // tile t starts at cum_n + kTileCost * t.  With
-//   chunk = max(ceil(total_cost / num_ctas), kTileCost)
-// CTA c owns the tiles whose start lies in [c * chunk, (c + 1) * chunk).
+//   chunk = kTileCost * max(ceil(total_cost / (num_ctas * kTileCost)), 1)
+// CTA c owns the tiles whose start lies in [c * chunk, (c + 1) * chunk): a
+// whole number of tiles per window, so no CTA holds more than
+// ceil(total_cost / (num_ctas * kTileCost)) tiles (the slowest CTA bounds the
+// kernel).  kSeqCost is half a tile: a range that crosses into another
+// sequence reloads queries and pays a second epilogue, which the other CTAs'
+// pipelines absorb but its own does not entirely.
 // Ranges are contiguous in the tile list, and because chunk >= kTileCost
 // every CTA between the first and the last owner of a sequence owns at least
 // one of its tiles.  Every kernel recomputes this from seqlens with the warp
 // routines below (no plan buffer).
 // ---------------------------------------------------------------------------
 constexpr int kTileCost = 8;
-constexpr int kSeqCost = 8;
+constexpr int kSeqCost = 4;
 
 __device__ __forceinline__ bool seqlen_valid(int L, int page_size, int max_pages) {
     return L >= 1 && (long long)L <= (long long)max_pages * page_size;
@@ -96,8 +101,9 @@ __device__ __forceinline__ int seq_cost(int L, int page_size, int max_pages) {
 }
 
 __host__ __device__ __forceinline__ int plan_chunk(int total_cost, int num_ctas) {
-    const int c = (total_cost + num_ctas - 1) / num_ctas;
-    return c > kTileCost ? c : kTileCost;
+    const long long per = ((long long)total_cost + (long long)num_ctas * kTileCost - 1) /
+                          ((long long)num_ctas * kTileCost);
+    return kTileCost * (per > 1 ? (int)per : 1);
 }
 
 // First tile of a sequence (cost start cum, `tiles` tiles) that starts at or

@@ -6,14 +6,15 @@ L_n < 1 or L_n > max_pages_per_seq * page_size.  Each tile costs TILE_COST
 units and each valid sequence SEQ_COST more, placed after its last tile, so a
 CTA whose range enters a new sequence is given less token work.  Tile t of
 sequence n starts at cum_n + TILE_COST * t; with
-chunk = max(ceil(total / num_ctas), TILE_COST), CTA c owns the tiles that
-start in [c * chunk, (c + 1) * chunk).
+chunk = TILE_COST * max(ceil(total / (num_ctas * TILE_COST)), 1) (a whole
+number of tiles), CTA c owns the tiles that start in
+[c * chunk, (c + 1) * chunk).
 """
 from __future__ import annotations
 
 TILE = 128
 TILE_COST = 8
-SEQ_COST = 8
+SEQ_COST = 4
 
 
 def seq_tiles(L, page_size, max_pages):
@@ -26,7 +27,7 @@ def owners(seqlens, page_size, max_pages, num_ctas):
     """Owner CTA of every tile, as a list of (sequence, tile, cta)."""
     tiles = [seq_tiles(int(L), page_size, max_pages) for L in seqlens]
     total = sum(TILE_COST * t + SEQ_COST for t in tiles if t)
-    chunk = max(-(-total // num_ctas), TILE_COST)
+    chunk = TILE_COST * max(-(-total // (num_ctas * TILE_COST)), 1)
     out, cum = [], 0
     for n, t in enumerate(tiles):
         if not t:

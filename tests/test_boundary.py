@@ -134,14 +134,17 @@ def test_plan_model_covers_every_tile_once(seqlens, ctas):
             assert (g0, g1, n0, n1) == (0, 0, -1, -1)
     assert covered == list(range(total))
     # a CTA's tiles plus the per-sequence charge of each sequence it enters
-    # fit within one chunk of cost, up to one tile and one sequence charge
+    # fit within one chunk of cost, up to one sequence charge; the chunk is a
+    # whole number of tiles, so no CTA holds more than chunk / TILE_COST tiles
     total_cost = sum(plan_model.TILE_COST * t + plan_model.SEQ_COST for t in tiles if t)
-    chunk = max(-(-total_cost // ctas), plan_model.TILE_COST)
+    per = max(-(-total_cost // (ctas * plan_model.TILE_COST)), 1)
+    chunk = plan_model.TILE_COST * per
     for c in range(ctas):
         g0, g1, n0, n1 = flat[4 * c:4 * c + 4]
         if g0 < g1:
             cost = plan_model.TILE_COST * (g1 - g0) + plan_model.SEQ_COST * (n1 - n0)
-            assert cost <= chunk + plan_model.TILE_COST + plan_model.SEQ_COST
+            assert cost <= chunk + plan_model.SEQ_COST
+            assert g1 - g0 <= per
     for n, t in enumerate(tiles):
         splits, first = flat[4 * ctas + 2 * n:4 * ctas + 2 * n + 2]
         if t == 0:
@@ -152,14 +155,10 @@ def test_plan_model_covers_every_tile_once(seqlens, ctas):
             assert owners == list(range(first, first + splits))
 
 
-def test_plan_model_gives_sequence_crossing_ctas_fewer_tiles():
-    # 16 sequences of 64 tiles over 148 CTAs: a CTA whose range enters a
-    # second sequence pays that sequence's charge in tiles
+def test_plan_model_bounds_the_slowest_cta():
+    # 16 sequences of 64 tiles over 148 CTAs: 1024 tiles need 7 per CTA at
+    # least, and no CTA gets more, whether or not its range crosses into a
+    # second sequence
     flat = plan_model.plan([8192] * 16, 64, 128, 148)
-    one, two = [], []
-    for c in range(148):
-        g0, g1, n0, n1 = flat[4 * c:4 * c + 4]
-        if g0 < g1:
-            (two if n1 > n0 else one).append(g1 - g0)
-    assert two and max(two) < max(one)
-    assert sum(one) + sum(two) == 16 * 64
+    counts = [flat[4 * c + 1] - flat[4 * c] for c in range(148)]
+    assert max(counts) == 7 and sum(counts) == 16 * 64
