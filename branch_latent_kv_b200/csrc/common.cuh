@@ -21,6 +21,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 // ---------------------------------------------------------------------------
 // Workspace layout (byte offsets, each region 256-byte aligned):
 //   [0, 256)        int32 error word (first device-side error code, else 0)
+//   split counters  int32 [kMaxBatch + 1]              (fixed place)
 //   lse partials    fp32 [slots][branches][HP]         (log2 domain; HP = 16,
 //                   or the head count when above 16: 64-byte rows)
 //   o partials      fp32 [slots][branches][d_c][16]    (normalised per split;

@@ -82,10 +82,16 @@ struct Cfg {
     // Pipeline depths: NSP steps may be between their score MMA and their
     // output MMA at once (S slots in TMEM, P slots in shared memory); NROPE
     // RoPE tiles are in flight, so the producer never waits for a tile's RoPE
-    // score before it loads the next tile; one query set (a sequence change
-    // waits for the previous range's score MMAs, rare: at most two per CTA).
+    // score before it loads the next tile (more slots when a tile is only one
+    // or two pairs of latents, so that the RoPE ring is not the shorter one);
+    // one query set (a sequence change waits for the previous range's score
+    // MMAs, rare: at most two per CTA).  The RoPE score of tile t lives in
+    // TMEM slot t % NRS: the score MMA of a tile's first step waits for the
+    // output MMA NSP steps back, so the softmax has read every RoPE score
+    // more than ceil(NSP / NSTEP) tiles back.
     static constexpr int NSP = 3;
-    static constexpr int NROPE = 2;
+    static constexpr int NROPE = NPAIR == 1 ? 4 : NPAIR == 2 ? 3 : 2;
+    static constexpr int NRS = (NSP + NSTEP - 1) / NSTEP > 2 ? (NSP + NSTEP - 1) / NSTEP : 2;
     static constexpr int FIXED = NROPE * ROPE_BYTES + QSET_BYTES + NSP * P_BYTES + MISC_BYTES;
     static constexpr int NSTAGE_FIT = (kSmemLimit - 1024 - FIXED) / PAIR_BYTES;
     static constexpr int NSTAGE = NSTAGE_FIT > 8 ? 8 : NSTAGE_FIT;
@@ -103,11 +109,11 @@ struct Cfg {
     static constexpr int S_COL0 = O_BLOCKS * kHP;
     static constexpr int S_SLOT_COLS = SBR * kHP;
     static constexpr int R_COL0 = S_COL0 + NSP * S_SLOT_COLS;
-    static constexpr int TMEM_COLS = R_COL0 + 2 * kHP <= 128 ? 128 : 256;
+    static constexpr int TMEM_COLS = R_COL0 + NRS * kHP <= 128 ? 128 : 256;
     static_assert(NB % SBR == 0 && (SBR * DC) % 128 == 0, "branches must fill whole steps and pairs");
     static_assert(NSTEP * PPS == NPAIR, "step / pair bookkeeping");
     static_assert(NSTAGE >= PPS, "a step's pairs must fit the stage ring");
-    static_assert(R_COL0 + 2 * kHP <= TMEM_COLS, "TMEM budget");
+    static_assert(R_COL0 + NRS * kHP <= TMEM_COLS, "TMEM budget");
     static_assert(SMEM_BYTES <= kSmemLimit, "shared-memory budget");
     static_assert(OFF_QR + QR_BYTES <= OFF_P && OFF_Q + Q_BYTES <= OFF_QR &&
                   OFF_P + NSP * P_BYTES <= OFF_MISC && QSET_BYTES % 1024 == 0 && ROPE_BYTES % 1024 == 0,
@@ -120,8 +126,8 @@ template <int NSTAGE>
 struct Misc {
     uint64_t pair_full[NSTAGE];
     uint64_t pair_empty[NSTAGE];
-    uint64_t rope_full[2];  // tile t in RoPE slot t & 1: its RoPE keys are in shared memory
-    uint64_t rope_empty[2];  // its RoPE score MMA finished
+    uint64_t rope_full[4];  // tile t in RoPE slot t % NROPE: its RoPE keys are in shared memory
+    uint64_t rope_empty[4];  // its RoPE score MMA finished
     uint64_t s_full[3];   // step g in slot g % NSP: its scores are in TMEM
     uint64_t p_full[3];   // its probabilities are in shared memory
     uint64_t p_empty[3];  // its output MMA finished (S and P slots free, O up to date)
@@ -207,6 +213,10 @@ __device__ __forceinline__ void warp_sum_scatter(float (&v)[N], int lane) {
         }
     }
 }
+
+struct bool4_t {
+    bool x, y, z, w;
+};
 
 template <int DR>
 __device__ __forceinline__ uint64_t rope_desc(uint32_t addr) {
@@ -417,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ DecodeArgs a) {
     using C = Cfg<NB, DC, DR>;
     using M = Misc<C::NSTAGE>;
-    static_assert(C::NSP <= 3 && C::NROPE == 2, "barrier arrays of Misc");
+    static_assert(C::NSP <= 3 && C::NROPE <= 4, "barrier arrays of Misc");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     M& misc = *reinterpret_cast<M*>(sm + C::OFF_MISC);
@@ -429,11 +439,12 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
             mbar_init(&misc.pair_full[i], 1);
             mbar_init(&misc.pair_empty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < C::NROPE; ++i) {
             mbar_init(&misc.rope_full[i], 1);
             mbar_init(&misc.rope_empty[i], 1);
-            mbar_init(&misc.drain[i], 1);
         }
+        mbar_init(&misc.drain[0], 1);
+        mbar_init(&misc.drain[1], 1);
         for (int i = 0; i < C::NSP; ++i) {
             mbar_init(&misc.s_full[i], 1);
             mbar_init(&misc.p_full[i], 4);
@@ -513,9 +524,9 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                         const int v = idx < a.max_pages ? __ldg(bt + idx) : 0;
                         win_val = (v >= 0 && v < a.num_pages) ? v : 0;  // bad entries are reported by the softmax warps
                     }
-                    const int rs = tc & 1;  // RoPE slot of this tile
+                    const int rs = tc % C::NROPE;  // RoPE slot of this tile
                     if (lane == 0) {
-                        if (tc >= 2) ok = mbar_wait(&misc.rope_empty[rs], ((tc >> 1) - 1) & 1);
+                        if (tc >= (uint32_t)C::NROPE) ok = mbar_wait(&misc.rope_empty[rs], ((tc / C::NROPE) - 1) & 1);
                         if (ok) mbar_arrive_expect_tx(&misc.rope_full[rs], npages * P * C::ROPE_ROW);
                     }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -564,9 +575,9 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                     const uint32_t k = pc - 1 - i;
                     mbar_wait(&misc.pair_full[k % C::NSTAGE], (k / C::NSTAGE) & 1, 200000000ull);
                 }
-                for (uint32_t i = 0; i < 2u && i < tc; ++i) {
+                for (uint32_t i = 0; i < (uint32_t)C::NROPE && i < tc; ++i) {
                     const uint32_t k = tc - 1 - i;
-                    mbar_wait(&misc.rope_full[k & 1], (k >> 1) & 1, 200000000ull);
+                    mbar_wait(&misc.rope_full[k % C::NROPE], (k / C::NROPE) & 1, 200000000ull);
                 }
                 if (sc > 0) mbar_wait(&misc.q_full, (sc - 1) & 1, 200000000ull);
             }
@@ -591,19 +602,14 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                 ok = mbar_wait_warp(&misc.q_full, sc & 1);
                 tc_fence_after();
                 for (int j = tb; j < te && ok; ++j) {
-                    ok = mbar_wait_warp(&misc.rope_full[tc & 1], (tc >> 1) & 1);
+                    const uint32_t rs = tc % C::NROPE;
+                    ok = mbar_wait_warp(&misc.rope_full[rs], (tc / C::NROPE) & 1);
 #pragma unroll 1
                     for (int st = 0; st < C::NSTEP && ok; ++st) {
-                        const uint32_t stage0 = stage;
-                        for (int p = 0; p < C::PPS && ok; ++p) {
-                            ok = mbar_wait_warp(&misc.pair_full[stage], phase);
-                            if (++stage == (uint32_t)C::NSTAGE) {
-                                stage = 0;
-                                phase ^= 1;
-                            }
-                        }
-                        // the S slot (and the P slot the softmax fills next) of
-                        // this step is free once the output MMA of step gs-2 is done
+                        // the step's first pair, then its S slot (and the P slot the
+                        // softmax fills next): free once the output MMA NSP steps
+                        // back is done
+                        ok = mbar_wait_warp(&misc.pair_full[stage], phase);
                         const uint32_t slot = gs % C::NSP;
                         if (ok && gs >= (uint32_t)C::NSP)
                             ok = mbar_wait_warp(&misc.p_empty[slot], ((gs / C::NSP) - 1) & 1);
@@ -611,34 +617,43 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                         tc_fence_after();
                         if (st == 0) {
                             // RoPE score of the tile, shared by every branch
-                            const uint32_t dRt = tmem + C::R_COL0 + (tc & 1) * kHP;
-                            const uint64_t dRs = dR + (((tc & 1) * C::ROPE_BYTES) >> 4);
+                            const uint32_t dRt = tmem + C::R_COL0 + (tc % C::NRS) * kHP;
+                            const uint64_t dRs = dR + ((rs * C::ROPE_BYTES) >> 4);
 #pragma unroll
                             for (int kk = 0; kk < DR / 16; ++kk)
                                 if (elect_one()) mma_bf16(dRt, dRs + kk * 2, dQR + kk * 2, IDESC_S, kk ? 1u : 0u);
-                            if (elect_one()) mma_commit(&misc.rope_empty[tc & 1]);
+                            if (elect_one()) mma_commit(&misc.rope_empty[rs]);
                             __syncwarp();
                         }
                         const uint32_t dS = tmem + C::S_COL0 + slot * C::S_SLOT_COLS;
                         // this step's branches start at chunk st*SBR*(DC/64) of the token row
                         const uint64_t dQs = dQ + ((st * C::SBR * (DC / 64) * C::Q_CHUNK_BYTES) >> 4);
+                        // each pair's MMAs as soon as it lands: chunk lc = 2 pp + hf of
+                        // the step is column chunk c of branch g of the step
+#pragma unroll 1
+                        for (int pp = 0; pp < C::PPS && ok; ++pp) {
+                            if (pp > 0) {
+                                ok = mbar_wait_warp(&misc.pair_full[stage], phase);
+                                if (!ok) break;
+                                tc_fence_after();
+                            }
 #pragma unroll
-                        for (int g = 0; g < C::SBR; ++g) {
-#pragma unroll
-                            for (int c = 0; c < DC / 64; ++c) {
-                                // chunk (g*(DC/64) + c) of this step: pair pp, half hf
-                                const int lc = g * (DC / 64) + c;
-                                const int pp = lc / 2, hf = lc % 2;
-                                uint32_t sp = stage0 + pp;
-                                if (sp >= (uint32_t)C::NSTAGE) sp -= C::NSTAGE;
-                                const uint64_t a0 = dA_s + ((sp * C::PAIR_BYTES + hf * C::CHUNK_BYTES) >> 4);
+                            for (int hf = 0; hf < 2; ++hf) {
+                                const int lc = 2 * pp + hf;
+                                const int g = lc / (DC / 64), c = lc % (DC / 64);
+                                const uint64_t a0 = dA_s + ((stage * C::PAIR_BYTES + hf * C::CHUNK_BYTES) >> 4);
                                 const uint64_t q0 = dQs + ((lc * C::Q_CHUNK_BYTES) >> 4);
 #pragma unroll
                                 for (int kk = 0; kk < 4; ++kk)
                                     if (elect_one())
                                         mma_bf16(dS + g * kHP, a0 + kk * 2, q0 + kk * 2, IDESC_S, (c | kk) ? 1u : 0u);
                             }
+                            if (++stage == (uint32_t)C::NSTAGE) {
+                                stage = 0;
+                                phase ^= 1;
+                            }
                         }
+                        if (!ok) break;
                         if (elect_one()) mma_commit(&misc.s_full[slot]);
                         __syncwarp();
                         ++gs;
@@ -698,11 +713,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                                         mma_bf16(d, a0 + (kt * 2048 >> 4), b0 + ((gl * C::P_BRANCH_BYTES + kt * 256) >> 4),
                                                  IDESC_PV, (j == tb && kt == 0) ? 0u : 1u);
                             }
-                        }
-#pragma unroll
-                        for (int p = 0; p < C::PPS; ++p) {
-                            uint32_t sp = stage + p;
-                            if (sp >= (uint32_t)C::NSTAGE) sp -= C::NSTAGE;
+                            // the pair's stage is free once its MMAs (and all before) finish
                             if (elect_one()) mma_commit(&misc.pair_empty[sp]);
                         }
                         if (elect_one()) mma_commit(&misc.p_empty[slot]);
@@ -762,7 +773,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                         const bool ok = mbar_wait(&misc.s_full[slot], (gs / C::NSP) & 1);
                         tc_fence_after();
                         float x[C::SBR][kHP];
-                        if (st == 0) tmem_ld16(tmem + lane_off + C::R_COL0 + (tcnt & 1) * kHP, r);
+                        if (st == 0) tmem_ld16(tmem + lane_off + C::R_COL0 + (tcnt % C::NRS) * kHP, r);
 #pragma unroll
                         for (int g = 0; g < C::SBR; ++g)
                             tmem_ld16(tmem + lane_off + C::S_COL0 + slot * C::S_SLOT_COLS + g * kHP, x[g]);
@@ -994,7 +1005,8 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                 if (stid == 0) {
                     // a split's partials are complete: counted for the merge when
                     // this CTA's work ends (only its first and last ranges can be
-                    // splits, and their merges wait for the kernel's end anyway)
+                    // splits, and their merges wait for the kernel's end anyway;
+                    // a fence here would stall the pipeline)
                     if (!single) {
                         if (pend_a < 0) pend_a = n; else pend_b = n;
                     }
@@ -1084,11 +1096,13 @@ cudaError_t launch_cfg(const DecodeArgs& a, cudaStream_t stream) {
     auto kernel = decode_tc_kernel<NB, DC, DR>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    // the merge stages in the ring: the weights of all S <= grid splits of a
-    // sequence and S row slices of at most R / (S - 1) + 1 rows of 64 bytes
-    if ((size_t)a.num_ctas * NB * kHP * sizeof(float) + (2 * (size_t)C::W + a.num_ctas) * kHP * sizeof(float) >
-        (size_t)C::NSTAGE * C::PAIR_BYTES)
-        return cudaErrorInvalidConfiguration;
+    // the merge stages in the ring: for all S <= grid splits of a sequence the
+    // log-sum-exp rows (S NB 16 floats), S row slices of at most
+    // R / (S - 1) + 1 rows of 16 floats (at most 2 R + S rows in all), the
+    // column partials (2 kThreads floats at most) and factors (NB 16 floats)
+    const size_t merge_bytes = sizeof(float) * ((size_t)a.num_ctas * NB * kHP + (2 * (size_t)C::W + a.num_ctas) * kHP +
+                                                2 * (size_t)kThreads + NB * kHP);
+    if (merge_bytes > (size_t)C::NSTAGE * C::PAIR_BYTES) return cudaErrorInvalidConfiguration;
     // Cooperative: every CTA is resident at once, so the merge's wait for the
     // other splits of a sequence always ends.
     cudaLaunchConfig_t cfg = {};
