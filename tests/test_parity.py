@@ -13,7 +13,7 @@ import pytest
 import torch
 
 from branch_latent_kv_b200 import binding as b
-from branch_latent_kv_b200.inputs import WORKLOADS, make_inputs
+from branch_latent_kv_b200.inputs import Workload, WORKLOADS, make_inputs
 from tests import plan_model
 
 pytestmark = pytest.mark.gpu
@@ -85,6 +85,30 @@ def test_small_cases_match_oracle(oracle_lib, name, peaked, impl):
     assert status == 0
     assert torch.isfinite(out.float()).all()
     _assert_close(out, ref, what=f"{name} peaked={peaked} {impl}")
+
+
+SHAPES = [(2, 64), (4, 64), (1, 128), (2, 128), (4, 128), (1, 256), (2, 256), (1, 512)]
+
+
+@pytest.mark.parametrize("branches,d_c", SHAPES)
+@pytest.mark.parametrize("d_r", [32, 64])
+@pytest.mark.parametrize("page_size", [16, 64, 128])
+def test_every_supported_shape_matches_oracle(oracle_lib, branches, d_c, d_r, page_size):
+    """Every (branches, d_c) the tensor-core kernel implements, both RoPE
+    widths and three page sizes (the kernel's ring depths and slot counts
+    differ per shape): short ragged sequences across several tiles, splits
+    and a partial last page, 12 heads (padding to the MMA's 16), scores
+    peaked enough to take the lazy-rescale path."""
+    w = Workload("shape", batch=5, heads=12, branches=branches, d_c=d_c, d_r=d_r,
+                 page_size=page_size, page_order="permuted")
+    seqlens = torch.tensor([1000, 1, 640, 129, 2047], dtype=torch.int32)
+    x = make_inputs(w, seed=11, q_gain=_score_gain(w, 4.0), slack_pages=3, nan_fill_unused=True,
+                    seqlens=seqlens).to("cuda")
+    out = _run(x)
+    ref, status = _oracle(oracle_lib, x)
+    assert status == 0
+    assert torch.isfinite(out.float()).all()
+    _assert_close(out, ref, what=f"B={branches} d_c={d_c} d_r={d_r} P={page_size}")
 
 
 @pytest.mark.parametrize("impl", sorted(IMPLS))
