@@ -12,9 +12,10 @@ L2 cannot serve the cache: each step reads the next of k copies of the
 pools, k * KV bytes >= 4x the L2 size.
 roofline: the decode kernel alone, CUDA events around each of K decode-only
 graph replays (same rotation), algorithmic KV bytes / mean duration.
-e2e: the same metric through the public Python API with the step's inputs
-(queries, block table, seqlens) copied from pinned host memory and the result
-y copied back, inside the timed region, one host synchronisation per step.
+e2e: the same metric through the public Python API (DecodeStep: one graph
+launch per step) with the step's inputs (queries, block table, seqlens)
+copied from pinned host memory and the result y copied back, inside the
+timed region, one host synchronisation per step.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
        [--impl ours|reference]
@@ -42,6 +43,7 @@ sys.path.insert(0, ROOT)
 
 from branch_latent_kv_b200 import binding as b  # noqa: E402
 from branch_latent_kv_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+from branch_latent_kv_b200.step import DecodeStep  # noqa: E402
 
 METRIC = "MLRA decode-attention KV GB/s and tokens/s at 1 B200; % of HBM roofline"
 FALLBACK_HBM_GBS = 6650.0
@@ -357,26 +359,23 @@ def main():
     elapsed_ms, decode_ms = max_over_ranks([elapsed_ms, decode_ms], pg, dev)
     del step_graphs, decode_graphs
 
-    # end to end through the public API, host buffers
-    h_q_lat = x.q_lat.cpu().pin_memory()
-    h_q_rope = x.q_rope.cpu().pin_memory()
-    h_bt = x.block_table.cpu().pin_memory()
-    h_sl = x.seqlens.cpu().pin_memory()
+    # end to end through the public API, host buffers: a DecodeStep per KV
+    # copy (the same bound device inputs), each step one graph launch that
+    # copies the inputs from pinned host memory, runs both kernels and copies
+    # y back; the host waits for every step
+    h_in = {"q_lat": x.q_lat.cpu().pin_memory(), "q_rope": x.q_rope.cpu().pin_memory(),
+            "block_table": x.block_table.cpu().pin_memory(), "seqlens": x.seqlens.cpu().pin_memory()}
     h_y = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-    d_q_lat, d_q_rope = torch.empty_like(x.q_lat), torch.empty_like(x.q_rope)
-    d_bt, d_sl = torch.empty_like(x.block_table), torch.empty_like(x.seqlens)
-    h2d = sum(t.numel() * t.element_size() for t in (h_q_lat, h_q_rope, h_bt, h_sl))
-    d2h = h_y.numel() * h_y.element_size()
+    d_in = {k: torch.empty_like(v, device=dev) for k, v in h_in.items()}
+    for k in d_in:
+        d_in[k].copy_(h_in[k])
+    steps_e2e = [DecodeStep(d_in["q_lat"], d_in["q_rope"], lat[c], rope[c], d_in["block_table"],
+                            d_in["seqlens"], x.scale, x.out_scale, w_uv=x.w_uv, host_inputs=h_in,
+                            host_output=h_y) for c in range(copies)]
+    h2d, d2h = steps_e2e[0].h2d_bytes(), steps_e2e[0].d2h_bytes()
 
     def e2e_step(i):
-        d_q_lat.copy_(h_q_lat, non_blocking=True)
-        d_q_rope.copy_(h_q_rope, non_blocking=True)
-        d_bt.copy_(h_bt, non_blocking=True)
-        d_sl.copy_(h_sl, non_blocking=True)
-        b.mlra_decode(d_q_lat, d_q_rope, lat[i % copies], rope[i % copies], d_bt, d_sl, x.scale,
-                      x.out_scale, out=out, workspace=ws)
-        b.mlra_up_proj(out, x.w_uv, y=y)
-        h_y.copy_(y, non_blocking=True)
+        steps_e2e[i % copies]()
         stream.synchronize()
 
     for k in range(args.warmup):
