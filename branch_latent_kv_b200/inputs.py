@@ -53,7 +53,7 @@ class Workload:
         return replace(self, **kw)
 
 
-# The five decode workloads (the fifth has three shapes).
+# The five decode workloads (the fifth has three shapes) and the variant sweep.
 WORKLOADS = {
     "tiny": Workload("tiny", batch=1, heads=8, branches=4, d_c=64, d_r=32, page_size=64,
                      seqlen=256, d_h=64),
@@ -71,6 +71,13 @@ WORKLOADS = {
     # replicated RoPE key; the calibration factor of the 4-branch model stays.
     "tp_shard": Workload("tp_shard", batch=32, heads=16, branches=1, d_c=128, d_r=64,
                          page_size=64, seqlen=16384, out_scale=0.5),
+    # Variant sweep: the two-branch model at the same cache bytes per token
+    # (2 x 256 + 64), and one sequence at the longest context the pages
+    # measure (2M tokens, 2.4 GB of cache).
+    "mlra2_equal_bytes": Workload("mlra2_equal_bytes", batch=32, heads=16, branches=2, d_c=256,
+                                  d_r=64, page_size=64, seqlen=16384),
+    "context_2m": Workload("context_2m", batch=1, heads=16, branches=4, d_c=128, d_r=64,
+                           page_size=64, seqlen=2097152, page_order="permuted"),
 }
 
 

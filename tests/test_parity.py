@@ -122,6 +122,7 @@ def test_tiny_workload_exact_recipe(oracle_lib, impl):
 
 @pytest.mark.parametrize("name,samples", [
     ("decode_2p9b", [0, 15]), ("long_context", [2]), ("ragged", [0, 17, 63]),
+    ("mlra2_equal_bytes", [0, 31]), ("context_2m", [0]),
     ("mla_equal_bytes", [5]), ("mlra4_equal_bytes", [31]), ("tp_shard", [0, 9]),
 ])
 def test_full_size_sampled_sequences(oracle_lib, name, samples):
