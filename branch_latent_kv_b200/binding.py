@@ -67,6 +67,8 @@ def library() -> ctypes.CDLL:
             lib.mlra_decode_simt.restype = ctypes.c_int
             lib.mlra_up_proj.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp]
             lib.mlra_up_proj.restype = ctypes.c_int
+            lib.mlra_up_proj_gated.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp]
+            lib.mlra_up_proj_gated.restype = ctypes.c_int
             lib.mlra_read_device_error.argtypes = [vp, vp]
             lib.mlra_read_device_error.restype = ctypes.c_int
             lib.mlra_status_string.argtypes = [ctypes.c_int]
@@ -191,6 +193,18 @@ def mlra_decode_simt(q_lat, q_rope, latent_cache, rope_cache, block_table, seqle
 
 def mlra_up_proj(out_lat, w_uv, d_h: Optional[int] = None, y=None, stream=None) -> torch.Tensor:
     """y bf16 [N, H*d_h] = per-branch W_UV up-projection summed over branches."""
+    return _up_proj(out_lat, w_uv, None, d_h, y, stream)
+
+
+def mlra_up_proj_gated(out_lat, w_uv, gate, d_h: Optional[int] = None, y=None,
+                       stream=None) -> torch.Tensor:
+    """mlra_up_proj times sigmoid(gate) elementwise; gate bf16 [N, H*d_h]."""
+    if gate is None:
+        raise ValueError("mlra_up_proj_gated needs a gate tensor")
+    return _up_proj(out_lat, w_uv, gate, d_h, y, stream)
+
+
+def _up_proj(out_lat, w_uv, gate, d_h, y, stream) -> torch.Tensor:
     dev = out_lat.device
     if dev.type != "cuda":
         raise ValueError("mlra_up_proj runs on CUDA tensors only")
@@ -207,9 +221,19 @@ def mlra_up_proj(out_lat, w_uv, d_h: Optional[int] = None, y=None, stream=None) 
         y = torch.empty((N, H * d_h), dtype=torch.bfloat16, device=dev)
     else:
         _require(y, "y", torch.bfloat16, 2, dev)
-    st = library().mlra_up_proj(N, H, B, d_c, d_h, _ptr(out_lat), _ptr(w_uv), _ptr(y),
-                                _stream_ptr(stream, dev))
-    _check(st, "mlra_up_proj")
+        if tuple(y.shape) != (N, H * d_h):
+            raise ValueError("y must be [N, heads*d_h]")
+    if gate is None:
+        st = library().mlra_up_proj(N, H, B, d_c, d_h, _ptr(out_lat), _ptr(w_uv), _ptr(y),
+                                    _stream_ptr(stream, dev))
+        _check(st, "mlra_up_proj")
+    else:
+        _require(gate, "gate", torch.bfloat16, 2, dev)
+        if tuple(gate.shape) != (N, H * d_h):
+            raise ValueError("gate must be [N, heads*d_h]")
+        st = library().mlra_up_proj_gated(N, H, B, d_c, d_h, _ptr(out_lat), _ptr(w_uv), _ptr(gate),
+                                          _ptr(y), _stream_ptr(stream, dev))
+        _check(st, "mlra_up_proj_gated")
     return y
 
 

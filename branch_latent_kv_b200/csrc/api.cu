@@ -146,18 +146,34 @@ mlra_status mlra_decode_simt(const mlra_dims* dims, const void* q_lat, const voi
                        seqlens, scale, out_scale, out, workspace, workspace_bytes, stream);
 }
 
-mlra_status mlra_up_proj(int32_t batch, int32_t heads, int32_t branches, int32_t d_c, int32_t d_h,
-                         const void* out_lat, const void* w_uv, void* y, void* stream) {
+namespace {
+mlra_status up_proj_impl(int32_t batch, int32_t heads, int32_t branches, int32_t d_c, int32_t d_h,
+                         const void* out_lat, const void* w_uv, const void* gate, void* y, void* stream) {
     if (batch < 1 || heads < 1 || branches < 1 || d_c < 1 || d_h < 1) return MLRA_ERR_INVALID_ARG;
     if (!aligned16(out_lat) || !aligned16(w_uv) || !aligned16(y)) return MLRA_ERR_INVALID_ARG;
+    if (gate != nullptr && (reinterpret_cast<uintptr_t>(gate) & 1u) != 0) return MLRA_ERR_INVALID_ARG;
     if ((int64_t)batch * heads * d_h > INT32_MAX) return MLRA_ERR_INVALID_ARG;
     const int K = branches * d_c;
     if (K % 64 != 0 || K > 512 || (d_h != 64 && d_h != 128)) return MLRA_ERR_UNSUPPORTED;
     return cuda_status(launch_up_proj(batch, heads, branches, d_c, d_h,
                                       static_cast<const __nv_bfloat16*>(out_lat),
                                       static_cast<const __nv_bfloat16*>(w_uv),
+                                      static_cast<const __nv_bfloat16*>(gate),
                                       static_cast<__nv_bfloat16*>(y),
                                       static_cast<cudaStream_t>(stream)));
+}
+}  // namespace
+
+mlra_status mlra_up_proj(int32_t batch, int32_t heads, int32_t branches, int32_t d_c, int32_t d_h,
+                         const void* out_lat, const void* w_uv, void* y, void* stream) {
+    return up_proj_impl(batch, heads, branches, d_c, d_h, out_lat, w_uv, nullptr, y, stream);
+}
+
+mlra_status mlra_up_proj_gated(int32_t batch, int32_t heads, int32_t branches, int32_t d_c,
+                               int32_t d_h, const void* out_lat, const void* w_uv, const void* gate,
+                               void* y, void* stream) {
+    if (gate == nullptr) return MLRA_ERR_INVALID_ARG;
+    return up_proj_impl(batch, heads, branches, d_c, d_h, out_lat, w_uv, gate, y, stream);
 }
 
 mlra_status mlra_read_device_error(void* workspace, void* stream) {

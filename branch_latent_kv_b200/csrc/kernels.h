@@ -40,10 +40,11 @@ size_t decode_simt_smem_bytes(int heads, int branches, int d_c, int d_r);
 // code for invalid sequences.
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t stream);
 
-// y = per-branch W_UV up-projection summed over branches.
+// y = per-branch W_UV up-projection summed over branches, times
+// sigmoid(gate) elementwise when gate is not null.
 cudaError_t launch_up_proj(int batch, int heads, int branches, int d_c, int d_h,
                            const __nv_bfloat16* out_lat, const __nv_bfloat16* w_uv,
-                           __nv_bfloat16* y, cudaStream_t stream);
+                           const __nv_bfloat16* gate, __nv_bfloat16* y, cudaStream_t stream);
 
 // Writes the work partition (see mlra_decode_plan in mlra.h).
 cudaError_t launch_plan_dump(int batch, int page_size, int max_pages, const int32_t* seqlens,

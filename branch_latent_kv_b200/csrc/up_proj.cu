@@ -21,6 +21,12 @@
 // [r*nt/KS, (r+1)*nt/KS) from all KS CTAs and writes them as bf16.
 // Rows j >= d_h (d_h = 64) are computed from neighbouring columns or TMA
 // zero fill and discarded.
+//
+// Optional output gate ("Critical Insight: The Value of 'Gating'" on the same
+// page: a gate on the attention output adds a non-linearity; its formula is
+// lost in the page text, read here as the usual elementwise sigmoid gate):
+//   y[n, c] *= 1 / (1 + exp(-gate[n, c]))   for every output element c,
+// applied to the fp32 sum before the bf16 rounding.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -50,7 +56,7 @@ struct UpSmem {
 
 __global__ void __launch_bounds__(kThreads, 1)
 up_proj_tc_kernel(const __grid_constant__ UpMaps maps, int batch, int heads, int K, int d_h, int nt, int ks,
-                  __nv_bfloat16* __restrict__ y) {
+                  const __nv_bfloat16* __restrict__ gate, __nv_bfloat16* __restrict__ y) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int cpc = K / 64 / ks;                 // K chunks of this CTA
@@ -152,7 +158,11 @@ up_proj_tc_kernel(const __grid_constant__ UpMaps maps, int batch, int heads, int
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int n = n0 + nn + i;
-                if (n < batch) y[(size_t)n * heads * d_h + (size_t)h * d_h + j] = to_bf16(vals[i]);
+                if (n >= batch) continue;
+                const size_t o = (size_t)n * heads * d_h + (size_t)h * d_h + j;
+                float v = vals[i];
+                if (gate != nullptr) v *= 1.f / (1.f + expf(-__bfloat162float(gate[o])));
+                y[o] = to_bf16(v);
             }
         }
     }
@@ -189,7 +199,7 @@ bool encode(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, u
 
 cudaError_t launch_up_proj(int batch, int heads, int branches, int d_c, int d_h,
                            const __nv_bfloat16* out_lat, const __nv_bfloat16* w_uv,
-                           __nv_bfloat16* y, cudaStream_t stream) {
+                           const __nv_bfloat16* gate, __nv_bfloat16* y, cudaStream_t stream) {
     const int K = branches * d_c;
     if (K % 64 != 0 || K / 64 > kMaxChunks) return cudaErrorInvalidValue;
     const int nchunk = K / 64;
@@ -221,7 +231,7 @@ cudaError_t launch_up_proj(int batch, int heads, int branches, int d_c, int d_h,
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, up_proj_tc_kernel, maps, batch, heads, K, d_h, nt, ks, y);
+    return cudaLaunchKernelEx(&cfg, up_proj_tc_kernel, maps, batch, heads, K, d_h, nt, ks, gate, y);
 }
 
 }  // namespace mlra

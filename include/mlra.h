@@ -189,6 +189,20 @@ MLRA_API mlra_status mlra_up_proj(int32_t batch, int32_t heads, int32_t branches
                          const void* out_lat, const void* w_uv, void* y, void* stream);
 
 /*
+ * mlra_up_proj followed by an elementwise output gate ("Critical Insight:
+ * The Value of 'Gating'" section of the blog page: a gate on the attention
+ * output; its formula is lost in the page text and is read here as the
+ * usual sigmoid gate on each output element):
+ *   y[n, c] = sigmoid(gate[n, c]) * sum_b sum_k out_lat[n,h,b,k] * w_uv[b][k][c]
+ * with c = h*d_h + j, applied to the fp32 sum before the bf16 rounding.
+ *   gate  bf16 [batch, heads * d_h]  gate logits (device memory, not null)
+ * Other arguments, shapes and errors as mlra_up_proj.
+ */
+MLRA_API mlra_status mlra_up_proj_gated(int32_t batch, int32_t heads, int32_t branches, int32_t d_c,
+                                        int32_t d_h, const void* out_lat, const void* w_uv,
+                                        const void* gate, void* y, void* stream);
+
+/*
  * Synchronises `stream`, returns the first device-side error code recorded
  * in `workspace` since the last read (MLRA_OK if none) and resets it to 0.
  * Returns MLRA_ERR_CUDA if the synchronisation or copy fails.

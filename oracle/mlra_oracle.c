@@ -212,6 +212,23 @@ int oracle_mlra_up_proj(int32_t batch, int32_t heads, int32_t branches, int32_t 
     return ORACLE_OK;
 }
 
+/*
+ * Output gate ("Critical Insight: The Value of 'Gating'" section of the blog
+ * page above: a gate on the attention output adds a non-linearity; its
+ * formula is lost in the page text, read as the usual elementwise sigmoid
+ * gate):
+ *   y[i] = y[i] / (1 + exp(-gate[i]))     for i < count
+ *   gate  bf16 bits or double (input_kind), y double (in place)
+ */
+int oracle_mlra_gate(int64_t count, int input_kind, const void* gate, double* y)
+{
+    if (count < 0) return ORACLE_ERR_ARG;
+    if (input_kind != ORACLE_BF16 && input_kind != ORACLE_F64) return ORACLE_ERR_ARG;
+    for (int64_t i = 0; i < count; ++i)
+        y[i] = y[i] / (1.0 + exp(-load(gate, i, input_kind)));
+    return ORACLE_OK;
+}
+
 /* Threads OpenMP will use (1 when built without OpenMP). */
 #ifdef _OPENMP
 #include <omp.h>

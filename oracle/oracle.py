@@ -5,9 +5,9 @@ CPU-baseline leg may call this module; the product path (the CUDA library and
 its Python binding) never does.  It shares no code with the CUDA path.
 
 ``build()`` compiles the C file with gcc and OpenMP into ``liboracle.so`` next
-to it.  ``decode`` and ``up_proj`` accept torch CPU tensors (bf16, passed as
-their bit patterns, or float64) or numpy float64 arrays and return float64
-numpy arrays.
+to it.  ``decode``, ``up_proj`` and ``gate`` accept torch CPU tensors (bf16,
+passed as their bit patterns, or float64) or numpy float64 arrays and return
+float64 numpy arrays.
 """
 from __future__ import annotations
 
@@ -46,6 +46,8 @@ def open_library(path: str):
     lib.oracle_mlra_decode.argtypes = [i32] * 8 + [ctypes.c_int] + [vp] * 6 + [dbl, dbl, vp, i32, vp, vp]
     lib.oracle_mlra_up_proj.restype = ctypes.c_int
     lib.oracle_mlra_up_proj.argtypes = [i32] * 5 + [ctypes.c_int, vp, vp, vp]
+    lib.oracle_mlra_gate.restype = ctypes.c_int
+    lib.oracle_mlra_gate.argtypes = [ctypes.c_int64, ctypes.c_int, vp, vp]
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
     return lib
@@ -143,3 +145,16 @@ def up_proj(out_lat, w_uv, d_h, lib=None):
     if status != 0:
         raise ValueError(f"oracle up_proj rejected its arguments (status {status})")
     return y
+
+
+def gate(y, gate_logits, lib=None):
+    """fp64 elementwise sigmoid output gate: y / (1 + exp(-gate)), same shape
+    as y (the gated up-projection; see oracle_mlra_gate)."""
+    yy = np.array(y, dtype=np.float64, copy=True, order="C")
+    g, kind = _as_input(gate_logits, None)
+    if g.shape != yy.shape:
+        raise ValueError("gate must have the shape of y")
+    status = (lib or _load()).oracle_mlra_gate(yy.size, kind, g.ctypes.data, yy.ctypes.data)
+    if status != 0:
+        raise ValueError(f"oracle gate rejected its arguments (status {status})")
+    return yy

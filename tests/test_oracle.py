@@ -318,3 +318,64 @@ def test_up_proj_bf16_and_float64_inputs_agree(oracle_lib):
     out_lat = torch.from_numpy(bf16_exact((3, 2, 4, 8), rng)).to(torch.bfloat16)
     w_uv = torch.from_numpy(bf16_exact((4, 8, 2 * 5), rng)).to(torch.bfloat16)
     assert np.array_equal(oracle_lib.up_proj(out_lat, w_uv, 5), oracle_lib.up_proj(out_lat.double(), w_uv, 5))
+
+
+# ---------------------------------------------------------------- output gate
+def test_gate_special_values(oracle_lib):
+    """The sigmoid gate: a zero logit halves the output exactly, a large
+    positive logit passes it, a large negative one closes it (the page reads
+    the gate as a non-linearity on the attention output)."""
+    y = np.array([[1.5, -2.0, 0.25, 3.0]])
+    half = oracle_lib.gate(y, torch.zeros(1, 4, dtype=torch.bfloat16))
+    assert np.array_equal(half, y / 2)
+    open_ = oracle_lib.gate(y, torch.full((1, 4), 80.0, dtype=torch.bfloat16))
+    assert np.allclose(open_, y, rtol=1e-15, atol=0)
+    shut = oracle_lib.gate(y, torch.full((1, 4), -80.0, dtype=torch.bfloat16))
+    assert np.all(np.abs(shut) <= np.abs(y) * 1e-34)
+
+
+def test_gate_is_a_logistic_split(oracle_lib):
+    """sigmoid(g) + sigmoid(-g) = 1: the gated outputs under g and -g add up
+    to the ungated output, and each lies between 0 and the output."""
+    rng = np.random.default_rng(21)
+    y = rng.normal(size=(6, 40))
+    g = torch.from_numpy(bf16_exact((6, 40), rng) * 4).to(torch.bfloat16)
+    a, b_ = oracle_lib.gate(y, g), oracle_lib.gate(y, -g)
+    assert np.allclose(a + b_, y, rtol=1e-14, atol=1e-15)
+    assert np.all(np.abs(a) <= np.abs(y)) and np.all(a * y >= 0)
+    assert np.array_equal(oracle_lib.gate(y, g), oracle_lib.gate(y, g.double()))
+
+
+GATE_MUTANTS = {
+    "gate_sign": ("y[i] = y[i] / (1.0 + exp(-load(gate, i, input_kind)));",
+                  "y[i] = y[i] / (1.0 + exp(load(gate, i, input_kind)));"),
+    "gate_no_one": ("y[i] = y[i] / (1.0 + exp(-load(gate, i, input_kind)));",
+                    "y[i] = y[i] / exp(-load(gate, i, input_kind));"),
+    "gate_multiplies": ("y[i] = y[i] / (1.0 + exp(-load(gate, i, input_kind)));",
+                        "y[i] = y[i] * (1.0 + exp(-load(gate, i, input_kind)));"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(GATE_MUTANTS))
+def test_planted_gate_mistakes_are_caught(tmp_path, name):
+    from oracle import oracle as orc
+    src = open(orc._SRC).read()
+    old, new = GATE_MUTANTS[name]
+    assert src.count(old) == 1, name
+    mut_src = tmp_path / "mut.c"
+    mut_src.write_text(src.replace(old, new))
+    so = tmp_path / "libmut.so"
+    subprocess.run(["gcc", "-O1", "-fopenmp", "-fPIC", "-shared", str(mut_src), "-o", str(so), "-lm"],
+                   check=True)
+    lib = orc.open_library(str(so))
+
+    class mut:
+        gate = staticmethod(lambda *a, **k: orc.gate(*a, lib=lib, **k))
+
+    caught = 0
+    for pin in (test_gate_special_values, test_gate_is_a_logistic_split):
+        try:
+            pin(mut)
+        except AssertionError:
+            caught += 1
+    assert caught >= 1, f"mutant {name} passed every pin"

@@ -263,6 +263,27 @@ def test_up_proj_matches_oracle(oracle_lib):
     assert np.linalg.norm(g - y_ref2) / np.linalg.norm(y_ref2) <= REL_L2
 
 
+@pytest.mark.parametrize("name", ["decode_2p9b", "mlra2_equal_bytes", "tiny"])
+def test_gated_up_proj_matches_oracle(oracle_lib, name):
+    """The fused output gate: y = sigmoid(gate) * up-projection, against the
+    oracle's up-projection followed by its gate."""
+    w = WORKLOADS[name]
+    x = make_inputs(w.with_(batch=min(w.batch, 16), seqlen=300, seqlen_range=None), seed=8).to("cuda")
+    out_lat = _run(x)
+    gen = torch.Generator(device="cpu").manual_seed(9)
+    gate = (torch.randn((x.q_lat.shape[0], x.q_lat.shape[1] * w.d_h), generator=gen) * 3).to(torch.bfloat16)
+    y = b.mlra_up_proj_gated(out_lat, x.w_uv, gate.to("cuda"))
+    ref = oracle_lib.gate(oracle_lib.up_proj(out_lat.cpu(), x.w_uv.cpu(), w.d_h), gate)
+    g = y.float().cpu().double().numpy()
+    assert np.abs(g - ref).max() <= MAX_ABS
+    assert np.linalg.norm(g - ref) / np.linalg.norm(ref) <= REL_L2
+    # gate logits of zero halve the ungated result exactly
+    y0 = b.mlra_up_proj_gated(out_lat, x.w_uv, torch.zeros_like(gate, device="cuda"))
+    y1 = b.mlra_up_proj(out_lat, x.w_uv)
+    assert torch.equal(y0.float(), (y1.float() / 2).to(torch.bfloat16).float()) or \
+        (y0.float() - y1.float() / 2).abs().max() <= 2 ** -8 * y1.float().abs().max()
+
+
 @pytest.mark.parametrize("batch", [1, 5, 16, 33, 300])
 def test_up_proj_batches(oracle_lib, batch):
     torch.manual_seed(batch)
