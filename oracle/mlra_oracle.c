@@ -229,6 +229,88 @@ int oracle_mlra_gate(int64_t count, int input_kind, const void* gate, double* y)
     return ORACLE_OK;
 }
 
+/*
+ * Decode pre-step: the work between the layer's projections and the decode
+ * attention for one new token per sequence.
+ *
+ *  1. Query absorption (the key up-projection folded into the query; the
+ *     "TransMLA" Hacker News thread quotes that only latents are cached and
+ *     attention runs against them after absorption; "The Core Insight" of the
+ *     blog page: each branch b has its own up-projection per head h):
+ *        q_lat[n,h,b,k] = sum_j w_uk[b,h,j,k] * q_c[n,h,j]
+ *  2. Rotary position embedding of the RoPE query and of the new token's
+ *     shared RoPE key at the new token's position p = seqlens[n] - 1, as
+ *     RoFormer defines it (pairs of adjacent dimensions rotated):
+ *        theta_i = base^(-2 i / d_r),  a = p * theta_i,  i < d_r / 2
+ *        x'[2i]   = x[2i] cos a - x[2i+1] sin a
+ *        x'[2i+1] = x[2i] sin a + x[2i+1] cos a
+ *  3. Append: the new token's latents c_new[n] and rotated key go to
+ *     page = block_table[n][p / P], slot = p mod P.
+ *
+ *   q_c     [batch, heads, d_h]            w_uk [branches, heads, d_h, d_c]
+ *   q_r     [batch, heads, d_r] (unrotated) kr_new [batch, d_r] (unrotated)
+ *   inputs as bf16 bits or doubles (input_kind)
+ *   q_lat   [batch, heads, branches, d_c] double (written)
+ *   q_rope  [batch, heads, d_r]           double (written, rotated)
+ *   kr_rot  [batch, d_r]                  double (written, rotated)
+ *   dest    [batch, 2] int32: (page, slot) the new token goes to, or (-1, -1)
+ *           when seqlens[n] < 1, p >= max_pages_per_seq * P or the page is
+ *           outside [0, num_pages) (the first such problem is returned:
+ *           6 = bad length, 5 = bad page)
+ */
+int oracle_mlra_prepare(int32_t batch, int32_t heads, int32_t branches, int32_t d_c, int32_t d_h,
+                        int32_t d_r, int32_t page_size, int32_t max_pages_per_seq,
+                        int32_t num_pages, int input_kind, const void* q_c, const void* q_r,
+                        const void* w_uk, const void* kr_new, const int32_t* seqlens,
+                        const int32_t* block_table, double rope_base, double* q_lat,
+                        double* q_rope, double* kr_rot, int32_t* dest)
+{
+    if (batch < 1 || heads < 1 || branches < 1 || d_c < 1 || d_h < 1 || d_r < 2 || d_r % 2 ||
+        page_size < 1 || max_pages_per_seq < 1 || num_pages < 1 || !(rope_base > 1.0))
+        return ORACLE_ERR_ARG;
+    if (input_kind != ORACLE_BF16 && input_kind != ORACLE_F64) return ORACLE_ERR_ARG;
+    int status = ORACLE_OK;
+    for (int64_t n = 0; n < batch; ++n) {
+        for (int64_t h = 0; h < heads; ++h)
+            for (int64_t b = 0; b < branches; ++b)
+                for (int64_t k = 0; k < d_c; ++k) {
+                    double sum = 0.0;
+                    for (int64_t j = 0; j < d_h; ++j)
+                        sum += load(w_uk, ((b * heads + h) * d_h + j) * d_c + k, input_kind) *
+                               load(q_c, (n * heads + h) * d_h + j, input_kind);
+                    q_lat[((n * heads + h) * branches + b) * d_c + k] = sum;
+                }
+        const int64_t p = (int64_t)seqlens[n] - 1;
+        for (int64_t i = 0; i < d_r / 2; ++i) {
+            const double a = (double)(p < 0 ? 0 : p) * pow(rope_base, -2.0 * (double)i / (double)d_r);
+            const double c = cos(a), sn = sin(a);
+            for (int64_t h = 0; h < heads; ++h) {
+                const int64_t o = (n * heads + h) * d_r + 2 * i;
+                const double x0 = load(q_r, o, input_kind), x1 = load(q_r, o + 1, input_kind);
+                q_rope[o] = x0 * c - x1 * sn;
+                q_rope[o + 1] = x0 * sn + x1 * c;
+            }
+            const double k0 = load(kr_new, n * d_r + 2 * i, input_kind);
+            const double k1 = load(kr_new, n * d_r + 2 * i + 1, input_kind);
+            kr_rot[n * d_r + 2 * i] = k0 * c - k1 * sn;
+            kr_rot[n * d_r + 2 * i + 1] = k0 * sn + k1 * c;
+        }
+        dest[2 * n] = dest[2 * n + 1] = -1;
+        if (p < 0 || p >= (int64_t)max_pages_per_seq * page_size) {
+            if (status == ORACLE_OK) status = ORACLE_ERR_BAD_SEQLEN;
+            continue;
+        }
+        const int32_t page = block_table[n * (int64_t)max_pages_per_seq + p / page_size];
+        if (page < 0 || page >= num_pages) {
+            if (status == ORACLE_OK) status = ORACLE_ERR_BAD_INDEX;
+            continue;
+        }
+        dest[2 * n] = page;
+        dest[2 * n + 1] = (int32_t)(p % page_size);
+    }
+    return status;
+}
+
 /* Threads OpenMP will use (1 when built without OpenMP). */
 #ifdef _OPENMP
 #include <omp.h>

@@ -46,6 +46,8 @@ def open_library(path: str):
     lib.oracle_mlra_decode.argtypes = [i32] * 8 + [ctypes.c_int] + [vp] * 6 + [dbl, dbl, vp, i32, vp, vp]
     lib.oracle_mlra_up_proj.restype = ctypes.c_int
     lib.oracle_mlra_up_proj.argtypes = [i32] * 5 + [ctypes.c_int, vp, vp, vp]
+    lib.oracle_mlra_prepare.restype = ctypes.c_int
+    lib.oracle_mlra_prepare.argtypes = [i32] * 9 + [ctypes.c_int] + [vp] * 6 + [dbl] + [vp] * 4
     lib.oracle_mlra_gate.restype = ctypes.c_int
     lib.oracle_mlra_gate.argtypes = [ctypes.c_int64, ctypes.c_int, vp, vp]
     lib.oracle_num_threads.restype = ctypes.c_int
@@ -158,3 +160,32 @@ def gate(y, gate_logits, lib=None):
     if status != 0:
         raise ValueError(f"oracle gate rejected its arguments (status {status})")
     return yy
+
+
+def prepare(q_c, q_r, w_uk, kr_new, seqlens, block_table, num_pages, page_size, rope_base=10000.0,
+            lib=None):
+    """fp64 decode pre-step (see oracle_mlra_prepare).  Returns
+    (q_lat [N,H,B,d_c], q_rope [N,H,d_r], kr_rot [N,d_r], dest [N,2] int32, status).
+    The new token's latents are copied, not computed, so they are not returned."""
+    arrs = [_as_input(a, None) for a in (q_c, q_r, w_uk, kr_new)]
+    kinds = {k for _, k in arrs}
+    if len(kinds) != 1:
+        raise TypeError("oracle inputs must share one float type (all bf16 or all float64)")
+    kind = kinds.pop()
+    (qc, _), (qr, _), (wk, _), (kr, _) = arrs
+    bt = np.ascontiguousarray(_as_input(block_table, None)[0], dtype=np.int32)
+    sl = np.ascontiguousarray(_as_input(seqlens, None)[0], dtype=np.int32)
+    N, H, d_h = qc.shape
+    B, _, _, d_c = wk.shape
+    d_r = qr.shape[2]
+    if wk.shape != (B, H, d_h, d_c) or qr.shape[:2] != (N, H) or kr.shape != (N, d_r):
+        raise ValueError("inconsistent oracle prepare shapes")
+    q_lat = np.empty((N, H, B, d_c), dtype=np.float64)
+    q_rope = np.empty((N, H, d_r), dtype=np.float64)
+    kr_rot = np.empty((N, d_r), dtype=np.float64)
+    dest = np.empty((N, 2), dtype=np.int32)
+    status = (lib or _load()).oracle_mlra_prepare(
+        N, H, B, d_c, d_h, d_r, page_size, bt.shape[1], num_pages, kind,
+        qc.ctypes.data, qr.ctypes.data, wk.ctypes.data, kr.ctypes.data, sl.ctypes.data, bt.ctypes.data,
+        float(rope_base), q_lat.ctypes.data, q_rope.ctypes.data, kr_rot.ctypes.data, dest.ctypes.data)
+    return q_lat, q_rope, kr_rot, dest, int(status)

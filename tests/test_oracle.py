@@ -379,3 +379,142 @@ def test_planted_gate_mistakes_are_caught(tmp_path, name):
         except AssertionError:
             caught += 1
     assert caught >= 1, f"mutant {name} passed every pin"
+
+
+# ---------------------------------------------------------------- decode pre-step
+def _prepare_inputs(rng, N=3, H=2, B=2, d_c=8, d_h=6, d_r=4):
+    q_c = bf16_exact((N, H, d_h), rng)
+    q_r = bf16_exact((N, H, d_r), rng)
+    w_uk = bf16_exact((B, H, d_h, d_c), rng)
+    kr = bf16_exact((N, d_r), rng)
+    return q_c, q_r, w_uk, kr
+
+
+def test_prepare_absorbed_scores_equal_explicit_keys(oracle_lib):
+    """q_lat . c equals q_c . (W_UK c) for any latent c: the absorbed query
+    scores a latent exactly as the explicit key would."""
+    rng = np.random.default_rng(31)
+    q_c, q_r, w_uk, kr = _prepare_inputs(rng)
+    N, H, d_h = q_c.shape
+    B, d_c = w_uk.shape[0], w_uk.shape[3]
+    table = np.arange(N * 2, dtype=np.int32).reshape(N, 2)
+    q_lat, _, _, _, st = oracle_lib.prepare(q_c, q_r, w_uk, kr, np.array([5, 1, 8], np.int32), table,
+                                            N * 2, 4)
+    assert st == 0
+    c = rng.standard_normal((B, d_c))
+    for n in range(N):
+        for h in range(H):
+            for b in range(B):
+                key = w_uk[b, h] @ c[b]  # [d_h]
+                assert abs(q_lat[n, h, b] @ c[b] - q_c[n, h] @ key) <= 1e-12 * (1 + abs(q_c[n, h] @ key))
+
+
+def test_prepare_feeds_decode_like_explicit_attention(oracle_lib):
+    """prepare -> decode -> up-projection equals explicit attention with
+    materialised keys (W_UK c) and values (W_UV c), the query's RoPE part
+    rotated at the new token's position."""
+    rng = np.random.default_rng(32)
+    N, H, B, d_c, d_r, d_h, P = 2, 3, 2, 8, 4, 6, 4
+    lengths = [7, 13]
+    lat, rope = _logical(rng, lengths, B, d_c, d_r)
+    q_c, q_r, w_uk, kr = _prepare_inputs(rng, N, H, B, d_c, d_h, d_r)
+    w_uv = rng.standard_normal((B, d_c, H * d_h)) / math.sqrt(B * d_c)
+    pool, rpool, table, seqlens = paged_from_logical(lat, rope, P, rng, slack_pages=2)
+    q_lat, q_rope, _, _, st = oracle_lib.prepare(q_c, q_r, w_uk, kr, seqlens, table, pool.shape[0], P)
+    assert st == 0
+    out_lat, _, st = oracle_lib.decode(q_lat, q_rope, pool, rpool, table, seqlens, 0.3, 0.7)
+    assert st == 0
+    y = oracle_lib.up_proj(out_lat, w_uv, d_h)
+    y_exp = explicit.explicit_decode(q_c, q_rope, np.asarray(w_uk), w_uv, lat, rope, 0.3, 0.7)
+    np.testing.assert_allclose(y, y_exp, rtol=1e-10, atol=1e-13)
+
+
+def test_prepare_rope_closed_forms(oracle_lib):
+    """RoFormer's rotation: position 0 is the identity; with d_r = 4 and base
+    10000, pair 0 turns by p radians and pair 1 by p / 100."""
+    e = np.zeros((1, 1, 4))
+    e[0, 0] = [1.0, 0.0, 0.0, 1.0]
+    k = np.array([[0.0, 1.0, 1.0, 0.0]])
+    w = np.zeros((1, 1, 1, 2))
+    q_c = np.zeros((1, 1, 1))
+    table = np.zeros((1, 4), np.int32)
+    for p in (0, 1, 100):
+        _, q_rope, kr_rot, dest, st = oracle_lib.prepare(q_c, e, w, k, np.array([p + 1], np.int32),
+                                                         table, 1, 64)
+        assert st == 0 and tuple(dest[0]) == (0, p % 64)
+        a0, a1 = float(p), p / 100.0
+        np.testing.assert_allclose(q_rope[0, 0], [math.cos(a0), math.sin(a0), -math.sin(a1), math.cos(a1)],
+                                   rtol=0, atol=1e-15)
+        np.testing.assert_allclose(kr_rot[0], [-math.sin(a0), math.cos(a0), math.cos(a1), math.sin(a1)],
+                                   rtol=0, atol=1e-15)
+
+
+def test_prepare_rotation_keeps_dot_products_and_norms(oracle_lib):
+    """Query and key rotated at the same position keep their dot product
+    (RoPE scores depend only on the relative position) and each pair keeps
+    its length."""
+    rng = np.random.default_rng(33)
+    q_c, q_r, w_uk, kr = _prepare_inputs(rng, N=3, H=2, d_r=8)
+    table = np.arange(3 * 300, dtype=np.int32).reshape(3, 300)
+    seqlens = np.array([1, 77, 19000], np.int32)
+    _, q_rope, kr_rot, _, st = oracle_lib.prepare(q_c, q_r, w_uk, kr, seqlens, table, 900, 64)
+    assert st == 0
+    for n in range(3):
+        for h in range(2):
+            assert abs(q_rope[n, h] @ kr_rot[n] - q_r[n, h] @ kr[n]) <= 1e-12
+            np.testing.assert_allclose(np.hypot(q_rope[n, h, 0::2], q_rope[n, h, 1::2]),
+                                       np.hypot(q_r[n, h, 0::2], q_r[n, h, 1::2]), rtol=1e-13)
+    np.testing.assert_array_equal(q_rope[0], q_r[0])  # position 0
+
+
+def test_prepare_append_target_and_errors(oracle_lib):
+    rng = np.random.default_rng(34)
+    q_c, q_r, w_uk, kr = _prepare_inputs(rng, N=4)
+    table = np.array([[7, 2, -1], [4, 9, 3], [0, -1, -1], [5, 6, 8]], np.int32)
+    seqlens = np.array([20, 33, 0, 100], np.int32)  # P = 16: slots 3 and 0 of pages 2, 3; bad; too long
+    _, _, _, dest, st = oracle_lib.prepare(q_c, q_r, w_uk, kr, seqlens, table, 10, 16)
+    assert tuple(dest[0]) == (2, 3) and tuple(dest[1]) == (3, 0)
+    assert tuple(dest[2]) == (-1, -1) and tuple(dest[3]) == (-1, -1)
+    assert st == 6  # the first problem: a bad length
+    seqlens = np.array([20, 33, 5, 10], np.int32)
+    table[3, 0] = 10  # outside the pool
+    _, _, _, dest, st = oracle_lib.prepare(q_c, q_r, w_uk, kr, seqlens, table, 10, 16)
+    assert st == 5 and tuple(dest[3]) == (-1, -1) and tuple(dest[2]) == (0, 4)
+
+
+PREPARE_MUTANTS = {
+    "rope_sin_sign": ("q_rope[o + 1] = x0 * sn + x1 * c;", "q_rope[o + 1] = -x0 * sn + x1 * c;"),
+    "rope_theta": ("pow(rope_base, -2.0 * (double)i / (double)d_r)", "pow(rope_base, -1.0 * (double)i / (double)d_r)"),
+    "rope_position": ("const int64_t p = (int64_t)seqlens[n] - 1;", "const int64_t p = (int64_t)seqlens[n];"),
+    "absorb_transposed": ("sum += load(w_uk, ((b * heads + h) * d_h + j) * d_c + k, input_kind) *",
+                          "sum += load(w_uk, ((b * heads + h) * d_c + k) * d_h + j, input_kind) *"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PREPARE_MUTANTS))
+def test_planted_prepare_mistakes_are_caught(tmp_path, name):
+    from oracle import oracle as orc
+    src = open(orc._SRC).read()
+    old, new = PREPARE_MUTANTS[name]
+    assert src.count(old) == 1, name
+    mut_src = tmp_path / "mut.c"
+    mut_src.write_text(src.replace(old, new))
+    so = tmp_path / "libmut.so"
+    subprocess.run(["gcc", "-O1", "-fopenmp", "-fPIC", "-shared", str(mut_src), "-o", str(so), "-lm"],
+                   check=True)
+    lib = orc.open_library(str(so))
+
+    class mut:
+        prepare = staticmethod(lambda *a, **k: orc.prepare(*a, lib=lib, **k))
+        decode = staticmethod(lambda *a, **k: orc.decode(*a, lib=lib, **k))
+        up_proj = staticmethod(lambda *a, **k: orc.up_proj(*a, lib=lib, **k))
+
+    caught = 0
+    for pin in (test_prepare_absorbed_scores_equal_explicit_keys, test_prepare_feeds_decode_like_explicit_attention,
+                test_prepare_rope_closed_forms, test_prepare_rotation_keeps_dot_products_and_norms,
+                test_prepare_append_target_and_errors):
+        try:
+            pin(mut)
+        except AssertionError:
+            caught += 1
+    assert caught >= 1, f"mutant {name} passed every pin"
