@@ -200,6 +200,48 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def prestep_time_us(x, w, dev, stream, steps):
+    """Mean duration of mlra_prepare on the workload's batch: CUDA events
+    around replays of a graph of 20 back-to-back launches, after warm-up."""
+    g = torch.Generator(device="cpu").manual_seed(w.seed + 1)
+    N, H, B, d_c = x.q_lat.shape
+    d_r, d_h = x.q_rope.shape[2], w.d_h
+
+    def draw(shape, fan):
+        return (torch.randn(shape, generator=g) / math.sqrt(fan)).to(torch.bfloat16).to(dev)
+    q_c, q_r, w_uk = draw((N, H, d_h), d_h), draw((N, H, d_r), d_r), draw((B, H, d_h, d_c), d_h)
+    c_new, kr_new = draw((N, B, d_c), d_c), draw((N, d_r), d_r)
+    q_lat, q_rope = torch.empty_like(x.q_lat), torch.empty_like(x.q_rope)
+    lat, rope = x.latent_cache.clone(), x.rope_cache.clone()  # the pre-step writes one row per sequence
+
+    def call(st):
+        b.mlra_prepare(q_c, q_r, w_uk, c_new, kr_new, x.seqlens, x.block_table, lat, rope,
+                       q_lat=q_lat, q_rope=q_rope, stream=st)
+    for _ in range(3):
+        call(stream)
+    # a few microseconds of kernel: 20 launches per graph replay so that the
+    # host's replay path does not starve the GPU between launches
+    per_graph = 20
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=cap):
+        for _ in range(per_graph):
+            call(cap)
+    torch.cuda.synchronize(dev)
+    for _ in range(3):
+        graph.replay()
+    reps = max(1, steps // per_graph)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    del lat, rope
+    return e0.elapsed_time(e1) / (reps * per_graph) * 1e3
+
+
 def workload_config(w, copies):
     cfg = {"workload": w.name, "batch": w.batch, "heads": w.heads, "branches": w.branches,
            "d_c": w.d_c, "d_r": w.d_r, "page_size": w.page_size, "d_h": w.d_h,
@@ -392,6 +434,10 @@ def main():
     e2e_ms, = max_over_ranks([e_start.elapsed_time(e_end)], pg, dev)
     sampler.stop()
 
+    # the decode pre-step (query absorption, rotary embedding, append) on the
+    # same batch, its own timed loop: events around each launch
+    pre_us = prestep_time_us(x, w, dev, stream, args.steps)
+
     err = b.mlra_read_device_error(ws)
     if err != 0:
         raise RuntimeError(f"device error during the benchmark: {b.mlra_status_string(err)}")
@@ -421,6 +467,10 @@ def main():
         "e2e": {"value": kv * world * args.steps / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * args.steps,  # per step: the decode kernel and the up-projection
+        "prestep": {"kernel": "prepare_kernel (mlra_prepare: query absorption, rotary embedding, "
+                              "append of the new token)", "us_per_launch": pre_us,
+                    "note": "not part of the step above; timed in its own loop on the same batch "
+                            "(back-to-back launches in a graph)"},
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -69,6 +69,9 @@ def library() -> ctypes.CDLL:
             lib.mlra_up_proj.restype = ctypes.c_int
             lib.mlra_up_proj_gated.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp]
             lib.mlra_up_proj_gated.restype = ctypes.c_int
+            lib.mlra_prepare.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, vp,
+                                         vp, vp]
+            lib.mlra_prepare.restype = ctypes.c_int
             lib.mlra_read_device_error.argtypes = [vp, vp]
             lib.mlra_read_device_error.restype = ctypes.c_int
             lib.mlra_status_string.argtypes = [ctypes.c_int]
@@ -253,3 +256,57 @@ def mlra_decode_plan(seqlens: torch.Tensor, page_size: int, max_pages_per_seq: i
                                     num_ctas, _ptr(out), _stream_ptr(stream, dev))
     _check(st, "mlra_decode_plan")
     return out
+
+
+def mlra_prepare(q_c, q_r, w_uk, c_new, kr_new, seqlens, block_table, latent_cache, rope_cache,
+                 rope_base: float = 10000.0, q_lat=None, q_rope=None, device_status=None,
+                 stream=None):
+    """The decode pre-step (see mlra_prepare in mlra.h): absorbed queries
+    q_lat bf16 [N,H,B,d_c], rotated RoPE queries q_rope bf16 [N,H,d_r], and the
+    new token's latents and rotated RoPE key written into the caches in place.
+
+    q_c bf16 [N,H,d_h], q_r bf16 [N,H,d_r], w_uk bf16 [B,H,d_h,d_c], c_new bf16
+    [N,B,d_c], kr_new bf16 [N,d_r], seqlens int32 [N] (including the new
+    token), block_table int32 [N,max_pages]; device_status: optional int32 [1]
+    device tensor receiving the first device-detected error code.
+    Returns (q_lat, q_rope).
+    """
+    dev = q_c.device
+    if dev.type != "cuda":
+        raise ValueError("mlra_prepare runs on CUDA tensors only")
+    _require(q_c, "q_c", torch.bfloat16, 3, dev)
+    _require(q_r, "q_r", torch.bfloat16, 3, dev)
+    _require(w_uk, "w_uk", torch.bfloat16, 4, dev)
+    _require(c_new, "c_new", torch.bfloat16, 3, dev)
+    _require(kr_new, "kr_new", torch.bfloat16, 2, dev)
+    _require(seqlens, "seqlens", torch.int32, 1, dev)
+    _require(block_table, "block_table", torch.int32, 2, dev)
+    _require(latent_cache, "latent_cache", torch.bfloat16, 4, dev)
+    _require(rope_cache, "rope_cache", torch.bfloat16, 3, dev)
+    N, H, d_h = q_c.shape
+    B, _, _, d_c = w_uk.shape
+    d_r = q_r.shape[2]
+    num_pages, P = latent_cache.shape[:2]
+    if (tuple(w_uk.shape) != (B, H, d_h, d_c) or tuple(q_r.shape[:2]) != (N, H)
+            or tuple(c_new.shape) != (N, B, d_c) or tuple(kr_new.shape) != (N, d_r)
+            or tuple(latent_cache.shape[2:]) != (B, d_c) or tuple(rope_cache.shape) != (num_pages, P, d_r)
+            or seqlens.shape[0] != N or block_table.shape[0] != N):
+        raise ValueError("inconsistent mlra_prepare shapes")
+    if q_lat is None:
+        q_lat = torch.empty((N, H, B, d_c), dtype=torch.bfloat16, device=dev)
+    else:
+        _require(q_lat, "q_lat", torch.bfloat16, 4, dev)
+    if q_rope is None:
+        q_rope = torch.empty((N, H, d_r), dtype=torch.bfloat16, device=dev)
+    else:
+        _require(q_rope, "q_rope", torch.bfloat16, 3, dev)
+    if device_status is not None:
+        _require(device_status, "device_status", torch.int32, 1, dev)
+    dims = mlra_dims(N, H, B, d_c, d_r, P, block_table.shape[1], num_pages)
+    st = library().mlra_prepare(ctypes.byref(dims), d_h, _ptr(q_c), _ptr(q_r), _ptr(w_uk), _ptr(c_new),
+                                _ptr(kr_new), _ptr(seqlens), _ptr(block_table), float(rope_base),
+                                _ptr(q_lat), _ptr(q_rope), _ptr(latent_cache), _ptr(rope_cache),
+                                _ptr(device_status) if device_status is not None else None,
+                                _stream_ptr(stream, dev))
+    _check(st, "mlra_prepare")
+    return q_lat, q_rope

@@ -176,6 +176,49 @@ mlra_status mlra_up_proj_gated(int32_t batch, int32_t heads, int32_t branches, i
     return up_proj_impl(batch, heads, branches, d_c, d_h, out_lat, w_uv, gate, y, stream);
 }
 
+mlra_status mlra_prepare(const mlra_dims* dims, int32_t d_h, const void* q_c, const void* q_r,
+                         const void* w_uk, const void* c_new, const void* kr_new,
+                         const int32_t* seqlens, const int32_t* block_table, float rope_base,
+                         void* q_lat, void* q_rope, void* latent_cache, void* rope_cache,
+                         int32_t* device_status, void* stream) {
+    mlra_status s = check_dims(dims);
+    if (s != MLRA_OK) return s;
+    if (d_h < 8 || d_h > 256 || d_h % 8 != 0 || dims->d_c % 8 != 0 || dims->d_r % 2 != 0 ||
+        dims->d_r > 64)
+        return MLRA_ERR_UNSUPPORTED;
+    if (!aligned16(q_c) || !aligned16(w_uk) || !aligned16(c_new) || !aligned16(q_lat) ||
+        !aligned16(latent_cache) || !aligned16(q_r) || !aligned16(kr_new) || !aligned16(q_rope) ||
+        !aligned16(rope_cache) || !aligned16(seqlens) || !aligned16(block_table))
+        return MLRA_ERR_INVALID_ARG;
+    if (device_status != nullptr && (reinterpret_cast<uintptr_t>(device_status) & 3u) != 0)
+        return MLRA_ERR_INVALID_ARG;
+    if (!(rope_base > 1.f) || !(rope_base < 3.0e38f)) return MLRA_ERR_INVALID_ARG;
+    PrepareArgs a;
+    a.q_c = static_cast<const __nv_bfloat16*>(q_c);
+    a.q_r = static_cast<const __nv_bfloat16*>(q_r);
+    a.w_uk = static_cast<const __nv_bfloat16*>(w_uk);
+    a.c_new = static_cast<const __nv_bfloat16*>(c_new);
+    a.kr_new = static_cast<const __nv_bfloat16*>(kr_new);
+    a.seqlens = seqlens;
+    a.block_table = block_table;
+    a.q_lat = static_cast<__nv_bfloat16*>(q_lat);
+    a.q_rope = static_cast<__nv_bfloat16*>(q_rope);
+    a.latent_cache = static_cast<__nv_bfloat16*>(latent_cache);
+    a.rope_cache = static_cast<__nv_bfloat16*>(rope_cache);
+    a.status = device_status;
+    a.batch = dims->batch;
+    a.heads = dims->heads;
+    a.branches = dims->branches;
+    a.d_c = dims->d_c;
+    a.d_r = dims->d_r;
+    a.d_h = d_h;
+    a.page_size = dims->page_size;
+    a.max_pages = dims->max_pages_per_seq;
+    a.num_pages = dims->num_pages;
+    a.rope_base = rope_base;
+    return cuda_status(launch_prepare(a, static_cast<cudaStream_t>(stream)));
+}
+
 mlra_status mlra_read_device_error(void* workspace, void* stream) {
     if (workspace == nullptr) return MLRA_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

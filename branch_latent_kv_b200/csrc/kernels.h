@@ -46,6 +46,28 @@ cudaError_t launch_up_proj(int batch, int heads, int branches, int d_c, int d_h,
                            const __nv_bfloat16* out_lat, const __nv_bfloat16* w_uv,
                            const __nv_bfloat16* gate, __nv_bfloat16* y, cudaStream_t stream);
 
+// Arguments of the decode pre-step (validated on the host).
+struct PrepareArgs {
+    const __nv_bfloat16* q_c;     // [N, H, d_h]
+    const __nv_bfloat16* q_r;     // [N, H, d_r] unrotated
+    const __nv_bfloat16* w_uk;    // [B, H, d_h, d_c]
+    const __nv_bfloat16* c_new;   // [N, B, d_c]
+    const __nv_bfloat16* kr_new;  // [N, d_r] unrotated
+    const int32_t* seqlens;       // [N] lengths including the new token
+    const int32_t* block_table;   // [N, max_pages]
+    __nv_bfloat16* q_lat;         // [N, H, B, d_c] written
+    __nv_bfloat16* q_rope;        // [N, H, d_r] written (rotated)
+    __nv_bfloat16* latent_cache;  // [pages, P, B, d_c] one row per sequence written
+    __nv_bfloat16* rope_cache;    // [pages, P, d_r] one row per sequence written
+    int* status;                  // optional device error word
+    int batch, heads, branches, d_c, d_r, d_h, page_size, max_pages, num_pages;
+    float rope_base;
+};
+
+// Query absorption, rotary embedding and the new token's append.
+cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t stream);
+size_t prepare_smem_bytes(int d_h);
+
 // Writes the work partition (see mlra_decode_plan in mlra.h).
 cudaError_t launch_plan_dump(int batch, int page_size, int max_pages, const int32_t* seqlens,
                              int num_ctas, int32_t* plan_out, cudaStream_t stream);

@@ -203,6 +203,47 @@ MLRA_API mlra_status mlra_up_proj_gated(int32_t batch, int32_t heads, int32_t br
                                         const void* gate, void* y, void* stream);
 
 /*
+ * The decode pre-step for one new token per sequence: the work between the
+ * layer's projections and mlra_decode.
+ *  1. Query absorption: q_lat[n,h,b,k] = sum_j w_uk[b,h,j,k] * q_c[n,h,j]
+ *     (each branch's key up-projection folded into the query, so that
+ *     attention runs against the cached latents; "The Core Insight" section
+ *     of the blog page: every branch has its own up-projection per head).
+ *  2. Rotary embedding (RoFormer's definition; the pages do not specify one)
+ *     of the RoPE query and the new token's RoPE key at its position
+ *     p = seqlens[n] - 1: pair i = (x[2i], x[2i+1]) turns by the angle
+ *     p * rope_base^(-2i/d_r) (angles formed in fp64).
+ *  3. Append: latent_cache[page][slot] = c_new[n], rope_cache[page][slot] =
+ *     the rotated key, page = block_table[n][p / P], slot = p mod P.
+ *   dims         as mlra_decode's (batch, heads, branches, d_c, d_r,
+ *                page_size, max_pages_per_seq, num_pages)
+ *   d_h          head dimension of q_c (a multiple of 8, at most 256)
+ *   q_c          bf16 [batch, heads, d_h]             no-RoPE query per head
+ *   q_r          bf16 [batch, heads, d_r]             RoPE query, unrotated
+ *   w_uk         bf16 [branches, heads, d_h, d_c]     key up-projections
+ *   c_new        bf16 [batch, branches, d_c]          the new token's latents
+ *   kr_new       bf16 [batch, d_r]                    its RoPE key, unrotated
+ *   seqlens      int32 [batch]  lengths including the new token
+ *   block_table  int32 [batch, max_pages_per_seq]
+ *   rope_base    e.g. 10000
+ *   q_lat        bf16 [batch, heads, branches, d_c]   written (mlra_decode's q_lat)
+ *   q_rope       bf16 [batch, heads, d_r]             written (mlra_decode's q_rope)
+ *   latent_cache, rope_cache  one row per valid sequence written in place
+ *   device_status  optional int32 (device, may be NULL): zeroed, then the
+ *                first device-detected problem (MLRA_ERR_DEVICE_BAD_SEQLEN for
+ *                seqlens[n] < 1 or beyond the block table,
+ *                MLRA_ERR_DEVICE_BAD_INDEX for a page outside the pool); such
+ *                a sequence's row is not written (its queries still are)
+ * Requires d_c a multiple of 8, d_r even and at most 64, 16-byte aligned
+ * arrays.  Allocates nothing; fp32 arithmetic, bf16 results.
+ */
+MLRA_API mlra_status mlra_prepare(const mlra_dims* dims, int32_t d_h, const void* q_c, const void* q_r,
+                                  const void* w_uk, const void* c_new, const void* kr_new,
+                                  const int32_t* seqlens, const int32_t* block_table, float rope_base,
+                                  void* q_lat, void* q_rope, void* latent_cache, void* rope_cache,
+                                  int32_t* device_status, void* stream);
+
+/*
  * Synchronises `stream`, returns the first device-side error code recorded
  * in `workspace` since the last read (MLRA_OK if none) and resets it to 0.
  * Returns MLRA_ERR_CUDA if the synchronisation or copy fails.
