@@ -111,6 +111,22 @@ def test_every_supported_shape_matches_oracle(oracle_lib, branches, d_c, d_r, pa
     _assert_close(out, ref, what=f"B={branches} d_c={d_c} d_r={d_r} P={page_size}")
 
 
+@pytest.mark.parametrize("heads", [1, 5, 16])
+@pytest.mark.parametrize("page_size", [32, 128])
+def test_head_counts_and_page_sizes(oracle_lib, heads, page_size):
+    """Head counts below the MMA's 16 (queries padded by the TMA's zero
+    fill) and the page sizes the other tests leave out, on the 2.9B shape."""
+    w = Workload("heads", batch=3, heads=heads, branches=4, d_c=128, d_r=64, page_size=page_size,
+                 page_order="permuted")
+    seqlens = torch.tensor([513, 33, 4097], dtype=torch.int32)
+    x = make_inputs(w, seed=12, q_gain=_score_gain(w, 3.0), slack_pages=2, nan_fill_unused=True,
+                    seqlens=seqlens).to("cuda")
+    out = _run(x)
+    ref, status = _oracle(oracle_lib, x)
+    assert status == 0
+    _assert_close(out, ref, what=f"H={heads} P={page_size}")
+
+
 @pytest.mark.parametrize("impl", sorted(IMPLS))
 def test_tiny_workload_exact_recipe(oracle_lib, impl):
     x = make_inputs(WORKLOADS["tiny"]).to("cuda")
