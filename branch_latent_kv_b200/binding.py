@@ -72,6 +72,21 @@ def library() -> ctypes.CDLL:
             lib.mlra_prepare.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, vp,
                                          vp, vp]
             lib.mlra_prepare.restype = ctypes.c_int
+            lib.mlra_exchange_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
+            lib.mlra_exchange_bytes.restype = sz
+            lib.mlra_exchange_alloc.argtypes = [sz, ctypes.POINTER(vp), vp]
+            lib.mlra_exchange_alloc.restype = ctypes.c_int
+            lib.mlra_exchange_open.argtypes = [vp, ctypes.POINTER(vp)]
+            lib.mlra_exchange_open.restype = ctypes.c_int
+            lib.mlra_exchange_close.argtypes = [vp]
+            lib.mlra_exchange_close.restype = ctypes.c_int
+            lib.mlra_exchange_free.argtypes = [vp]
+            lib.mlra_exchange_free.restype = ctypes.c_int
+            lib.mlra_exchange_reset.argtypes = [vp, sz, vp]
+            lib.mlra_exchange_reset.restype = ctypes.c_int
+            lib.mlra_up_proj_allreduce.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, i32, i32, i32,
+                                                   vp, ctypes.c_uint64, vp]
+            lib.mlra_up_proj_allreduce.restype = ctypes.c_int
             lib.mlra_read_device_error.argtypes = [vp, vp]
             lib.mlra_read_device_error.restype = ctypes.c_int
             lib.mlra_status_string.argtypes = [ctypes.c_int]
@@ -310,3 +325,100 @@ def mlra_prepare(q_c, q_r, w_uk, c_new, kr_new, seqlens, block_table, latent_cac
                                 _stream_ptr(stream, dev))
     _check(st, "mlra_prepare")
     return q_lat, q_rope
+
+
+# ------------------------------------------------------------------ branch sharding
+MLRA_IPC_HANDLE_BYTES = 64
+
+
+def mlra_exchange_bytes(batch: int, heads: int, branches: int, d_c: int, d_h: int, world: int) -> int:
+    """Bytes of one rank's exchange region (branches = the rank's own count)."""
+    n = library().mlra_exchange_bytes(batch, heads, branches, d_c, d_h, world)
+    if n == 0:
+        raise MlraError(MLRA_ERR_INVALID_ARG, "mlra_exchange_bytes")
+    return int(n)
+
+
+def mlra_exchange_alloc(nbytes: int, with_handle: bool = True):
+    """A zeroed exchange region on the current device: (pointer, IPC handle
+    bytes or None).  Release it with mlra_exchange_free."""
+    p = ctypes.c_void_p()
+    h = ctypes.create_string_buffer(MLRA_IPC_HANDLE_BYTES) if with_handle else None
+    _check(library().mlra_exchange_alloc(int(nbytes), ctypes.byref(p), h), "mlra_exchange_alloc")
+    return int(p.value), (h.raw if h is not None else None)
+
+
+def mlra_exchange_open(handle: bytes) -> int:
+    """Map another process's exchange region from its handle."""
+    if len(handle) != MLRA_IPC_HANDLE_BYTES:
+        raise ValueError("an exchange handle has 64 bytes")
+    p = ctypes.c_void_p()
+    _check(library().mlra_exchange_open(ctypes.create_string_buffer(handle, MLRA_IPC_HANDLE_BYTES),
+                                        ctypes.byref(p)), "mlra_exchange_open")
+    return int(p.value)
+
+
+def mlra_exchange_close(ptr: int) -> None:
+    _check(library().mlra_exchange_close(ptr), "mlra_exchange_close")
+
+
+def mlra_exchange_free(ptr: int) -> None:
+    _check(library().mlra_exchange_free(ptr), "mlra_exchange_free")
+
+
+def mlra_exchange_reset(ptr: int, nbytes: int, device: Optional[torch.device] = None, stream=None) -> None:
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    _check(library().mlra_exchange_reset(ptr, int(nbytes), _stream_ptr(stream, dev)), "mlra_exchange_reset")
+
+
+def mlra_up_proj_allreduce(out_lat, w_uv, regions: torch.Tensor, rank: int, gate=None,
+                           d_h: Optional[int] = None, y=None, ranks_in_launch: int = 1,
+                           device_status=None, wait_limit_ns: int = 2_000_000_000,
+                           stream=None) -> torch.Tensor:
+    """Branch-sharded up-projection with the cross-rank branch sum (see
+    mlra_up_proj_allreduce in mlra.h).
+
+    out_lat bf16 [N,H,B_r,d_c] and w_uv bf16 [B_r,d_c,H*d_h] hold this rank's
+    B_r branches; regions is an int64 device tensor [world] of the ranks'
+    exchange-region pointers; returns the full y bf16 [N,H*d_h].  With
+    ranks_in_launch = k > 1 the operands carry a leading rank dimension
+    ([k,N,H,B_r,d_c], [k,B_r,d_c,H*d_h] -> y [k,N,H*d_h]) for ranks rank ..
+    rank+k-1, all computed in one launch on this device.
+    """
+    dev = out_lat.device
+    if dev.type != "cuda":
+        raise ValueError("mlra_up_proj_allreduce runs on CUDA tensors only")
+    k = int(ranks_in_launch)
+    lead = 1 if k > 1 else 0
+    _require(out_lat, "out_lat", torch.bfloat16, 4 + lead, dev)
+    _require(w_uv, "w_uv", torch.bfloat16, 3 + lead, dev)
+    _require(regions, "regions", torch.int64, 1, dev)
+    if lead and (out_lat.shape[0] != k or w_uv.shape[0] != k):
+        raise ValueError("stacked operands need a leading dimension of ranks_in_launch")
+    N, H, B, d_c = out_lat.shape[lead:]
+    if tuple(w_uv.shape[lead:lead + 2]) != (B, d_c) or w_uv.shape[-1] % H != 0:
+        raise ValueError("w_uv must be [branches, d_c, heads*d_h]")
+    if d_h is None:
+        d_h = w_uv.shape[-1] // H
+    if w_uv.shape[-1] != H * d_h:
+        raise ValueError("w_uv last dimension must be heads*d_h")
+    y_shape = ((k,) if lead else ()) + (N, H * d_h)
+    if y is None:
+        y = torch.empty(y_shape, dtype=torch.bfloat16, device=dev)
+    else:
+        _require(y, "y", torch.bfloat16, 2 + lead, dev)
+        if tuple(y.shape) != y_shape:
+            raise ValueError(f"y must be {list(y_shape)}")
+    if gate is not None:
+        _require(gate, "gate", torch.bfloat16, 2, dev)
+        if tuple(gate.shape) != (N, H * d_h):
+            raise ValueError("gate must be [N, heads*d_h]")
+    if device_status is not None:
+        _require(device_status, "device_status", torch.int32, 1, dev)
+    st = library().mlra_up_proj_allreduce(N, H, B, d_c, d_h, _ptr(out_lat), _ptr(w_uv),
+                                          _ptr(gate) if gate is not None else None, _ptr(y), _ptr(regions),
+                                          regions.numel(), int(rank), k,
+                                          _ptr(device_status) if device_status is not None else None,
+                                          int(wait_limit_ns), _stream_ptr(stream, dev))
+    _check(st, "mlra_up_proj_allreduce")
+    return y

@@ -176,6 +176,95 @@ mlra_status mlra_up_proj_gated(int32_t batch, int32_t heads, int32_t branches, i
     return up_proj_impl(batch, heads, branches, d_c, d_h, out_lat, w_uv, gate, y, stream);
 }
 
+size_t mlra_exchange_bytes(int32_t batch, int32_t heads, int32_t branches, int32_t d_c, int32_t d_h,
+                           int32_t world) {
+    if (batch < 1 || heads < 1 || branches < 1 || d_c < 1 || d_h < 1 || world < 1 || world > kMaxWorld) return 0;
+    if ((branches * d_c) % 64 != 0 || branches * d_c > 512) return 0;
+    if ((int64_t)batch * heads * d_h > INT32_MAX) return 0;
+    return exchange_layout(batch, heads, d_h, world, up_proj_tiles(batch, heads, branches, d_c)).total;
+}
+
+mlra_status mlra_exchange_alloc(size_t bytes, void** region, void* ipc_handle) {
+    if (region == nullptr || bytes == 0) return MLRA_ERR_INVALID_ARG;
+    *region = nullptr;
+    void* p = nullptr;
+    if (cudaMalloc(&p, bytes) != cudaSuccess) return MLRA_ERR_CUDA;
+    if (cudaMemset(p, 0, bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+        cudaFree(p);
+        return MLRA_ERR_CUDA;
+    }
+    if (ipc_handle != nullptr) {
+        static_assert(sizeof(cudaIpcMemHandle_t) == MLRA_IPC_HANDLE_BYTES, "IPC handle size");
+        cudaIpcMemHandle_t h;
+        if (cudaIpcGetMemHandle(&h, p) != cudaSuccess) {
+            cudaFree(p);
+            return MLRA_ERR_CUDA;
+        }
+        std::memcpy(ipc_handle, &h, sizeof(h));
+    }
+    *region = p;
+    return MLRA_OK;
+}
+
+mlra_status mlra_exchange_open(const void* ipc_handle, void** region) {
+    if (ipc_handle == nullptr || region == nullptr) return MLRA_ERR_INVALID_ARG;
+    *region = nullptr;
+    cudaIpcMemHandle_t h;
+    std::memcpy(&h, ipc_handle, sizeof(h));
+    void* p = nullptr;
+    if (cudaIpcOpenMemHandle(&p, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) return MLRA_ERR_CUDA;
+    *region = p;
+    return MLRA_OK;
+}
+
+mlra_status mlra_exchange_close(void* region) {
+    if (region == nullptr) return MLRA_ERR_INVALID_ARG;
+    return cuda_status(cudaIpcCloseMemHandle(region));
+}
+
+mlra_status mlra_exchange_free(void* region) {
+    if (region == nullptr) return MLRA_ERR_INVALID_ARG;
+    return cuda_status(cudaFree(region));
+}
+
+mlra_status mlra_exchange_reset(void* region, size_t bytes, void* stream) {
+    if (region == nullptr || bytes == 0) return MLRA_ERR_INVALID_ARG;
+    return cuda_status(cudaMemsetAsync(region, 0, bytes, static_cast<cudaStream_t>(stream)));
+}
+
+mlra_status mlra_up_proj_allreduce(int32_t batch, int32_t heads, int32_t branches, int32_t d_c, int32_t d_h,
+                                   const void* out_lat, const void* w_uv, const void* gate, void* y,
+                                   void* const* regions, int32_t world, int32_t rank, int32_t ranks_in_launch,
+                                   int32_t* device_status, uint64_t wait_limit_ns, void* stream) {
+    if (batch < 1 || heads < 1 || branches < 1 || d_c < 1 || d_h < 1) return MLRA_ERR_INVALID_ARG;
+    if (world < 1 || world > kMaxWorld || rank < 0 || ranks_in_launch < 1 || rank + ranks_in_launch > world)
+        return MLRA_ERR_INVALID_ARG;
+    if (!aligned16(out_lat) || !aligned16(w_uv) || !aligned16(y) || !aligned16(regions))
+        return MLRA_ERR_INVALID_ARG;
+    if (gate != nullptr && (reinterpret_cast<uintptr_t>(gate) & 1u) != 0) return MLRA_ERR_INVALID_ARG;
+    if (device_status != nullptr && (reinterpret_cast<uintptr_t>(device_status) & 3u) != 0)
+        return MLRA_ERR_INVALID_ARG;
+    if (wait_limit_ns == 0) return MLRA_ERR_INVALID_ARG;
+    if ((int64_t)batch * ranks_in_launch * heads * d_h > INT32_MAX) return MLRA_ERR_INVALID_ARG;
+    const int K = branches * d_c;
+    if (K % 64 != 0 || K > 512 || (d_h != 64 && d_h != 128)) return MLRA_ERR_UNSUPPORTED;
+    XRankArgs xr;
+    xr.regions = regions;
+    xr.world = world;
+    xr.rank_base = rank;
+    xr.tiles = up_proj_tiles(batch, heads, branches, d_c);
+    xr.status = device_status;
+    xr.limit_ns = wait_limit_ns;
+    const cudaError_t e = launch_up_proj_xrank(batch, heads, branches, d_c, d_h,
+                                               static_cast<const __nv_bfloat16*>(out_lat),
+                                               static_cast<const __nv_bfloat16*>(w_uv),
+                                               static_cast<const __nv_bfloat16*>(gate),
+                                               static_cast<__nv_bfloat16*>(y), xr, ranks_in_launch,
+                                               static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorCooperativeLaunchTooLarge) return MLRA_ERR_UNSUPPORTED;
+    return cuda_status(e);
+}
+
 mlra_status mlra_prepare(const mlra_dims* dims, int32_t d_h, const void* q_c, const void* q_r,
                          const void* w_uk, const void* c_new, const void* kr_new,
                          const int32_t* seqlens, const int32_t* block_table, float rope_base,

@@ -46,6 +46,51 @@ cudaError_t launch_up_proj(int batch, int heads, int branches, int d_c, int d_h,
                            const __nv_bfloat16* out_lat, const __nv_bfloat16* w_uv,
                            const __nv_bfloat16* gate, __nv_bfloat16* y, cudaStream_t stream);
 
+// ---------------------------------------------------------------------------
+// Cross-rank branch sum of the branch-sharded up-projection.  Every rank owns
+// one exchange region (device memory that every other rank can address):
+//   epoch [tiles]                u32  calls completed, per output tile
+//   flag  [2][world][tiles]      u32  flag[par][src][t] = call + 1 once rank
+//                                     src's tile t of that call has landed
+//   data  [2][world][batch][heads*d_h]  fp32 partial sums pushed by each rank
+// par = call & 1 double-buffers flags and data, so no flag is ever reset.
+constexpr int kMaxWorld = 8;
+
+struct ExchangeLayout {
+    size_t epoch_off, flag_off, data_off, total;
+};
+
+__host__ __device__ inline ExchangeLayout exchange_layout(int batch, int heads, int d_h, int world, int tiles) {
+    ExchangeLayout L;
+    L.epoch_off = 0;
+    L.flag_off = ((size_t)tiles * 4 + 255) & ~size_t(255);
+    L.data_off = L.flag_off + (((size_t)2 * world * tiles * 4 + 255) & ~size_t(255));
+    L.total = L.data_off + (((size_t)2 * world * batch * heads * d_h * 4 + 255) & ~size_t(255));
+    return L;
+}
+
+struct XRankArgs {
+    void* const* regions;  // device array [world]: every rank's exchange region
+    int world;             // ranks in the sum (0: no cross-rank sum)
+    int rank_base;         // rank computed by blockIdx.z == 0
+    int tiles;             // output tiles (CTAs) of one rank's grid
+    int* status;           // optional device error word
+    unsigned long long limit_ns;  // bound on the wait for the other ranks
+};
+
+// Output tiles (CTAs per rank) of the up-projection grid for these sizes.
+int up_proj_tiles(int batch, int heads, int branches, int d_c);
+
+// The branch-sharded up-projection: each rank multiplies its own branches,
+// then the ranks' fp32 partial sums are exchanged through the regions and
+// added in rank order.  ranks_in_launch > 1 runs ranks rank_base ..
+// rank_base + ranks_in_launch - 1 in one launch on one device, with their
+// out_lat, w_uv and y stacked along the leading dimension.
+cudaError_t launch_up_proj_xrank(int batch, int heads, int branches, int d_c, int d_h,
+                                 const __nv_bfloat16* out_lat, const __nv_bfloat16* w_uv,
+                                 const __nv_bfloat16* gate, __nv_bfloat16* y, const XRankArgs& xr,
+                                 int ranks_in_launch, cudaStream_t stream);
+
 // Arguments of the decode pre-step (validated on the host).
 struct PrepareArgs {
     const __nv_bfloat16* q_c;     // [N, H, d_h]

@@ -27,6 +27,20 @@
 // lost in the page text, read here as the usual elementwise sigmoid gate):
 //   y[n, c] *= 1 / (1 + exp(-gate[n, c]))   for every output element c,
 // applied to the fp32 sum before the bf16 rounding.
+//
+// Branch sharding ("The Core Insight" section of the same page: the branches
+// can live on different GPUs, so under 4-way tensor parallelism each GPU loads
+// only its own branch's latents plus the shared RoPE key, 1.5 d_h per token
+// against 4.5 d_h for MLA).  Rank r then holds out_lat and W_UV of its
+// branches only, and the branch sum crosses the ranks.  In that mode the cluster's column slice is
+// not written as y: each CTA stores its fp32 slice into slot r of every
+// rank's exchange region (plain stores, to peer memory over NVLink), then
+// raises its flag there (release at system scope).  Each rank waits, with a
+// bound, for the flags of all ranks on its own region, adds the slots in rank
+// order (the same order on every rank, so every rank's y is bit-identical)
+// and applies the gate.  The call number of each tile, kept per tile in the
+// region, selects one of two buffers, so a rank that runs ahead into the next
+// call never overwrites data that a slower rank is still adding up.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -52,21 +66,30 @@ struct UpSmem {
     uint64_t full[kMaxChunks];
     uint64_t mma_done;
     uint32_t tmem_base;
+    int xr_ok;  // cross-rank mode: every rank's slice arrived
 };
 
+// kXRank: the cross-rank branch sum (a separate instantiation, so that the
+// single-device kernel carries none of its code or registers)
+template <bool kXRank>
 __global__ void __launch_bounds__(kThreads, 1)
 up_proj_tc_kernel(const __grid_constant__ UpMaps maps, int batch, int heads, int K, int d_h, int nt, int ks,
-                  const __nv_bfloat16* __restrict__ gate, __nv_bfloat16* __restrict__ y) {
+                  const __nv_bfloat16* __restrict__ gate, __nv_bfloat16* __restrict__ y, const XRankArgs xr) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int cpc = K / 64 / ks;                 // K chunks of this CTA
     const int x_chunk_bytes = nt * 128;
     uint8_t* w_s = sm;                           // cpc x 16 KB
     uint8_t* x_s = sm + cpc * kWChunkBytes;      // cpc x nt*128 B
-    UpSmem& ms = *reinterpret_cast<UpSmem*>(x_s + cpc * x_chunk_bytes);
     float* part = reinterpret_cast<float*>(sm);  // [128][nt] fp32 partial, reuses the operand buffers
+    // barriers and flags past both the operands and the partial
+    UpSmem& ms = *reinterpret_cast<UpSmem*>(sm + max(cpc * (kWChunkBytes + x_chunk_bytes), 128 * nt * 4));
     const uint32_t rank = cluster_ctarank();
     const int h = blockIdx.x / ks, n0 = blockIdx.y * nt;
+    // blockIdx.z: which of the ranks stacked into this launch (0 otherwise);
+    // its operands start lr * K rows into w_uv and lr * batch rows into out_lat
+    const int lr = blockIdx.z;
+    y += (size_t)lr * batch * heads * d_h;
     const int c_first = (int)rank * cpc;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t tmem_cols = nt <= 32 ? 32 : 64;
@@ -94,12 +117,13 @@ up_proj_tc_kernel(const __grid_constant__ UpMaps maps, int batch, int heads, int
         for (int c = 0; c < cpc; ++c) {
             const int kc = c_first + c;
             mbar_arrive_expect_tx(&ms.full[c], kWChunkBytes + x_chunk_bytes);
-            tma_load_2d(w_s + c * kWChunkBytes, &maps.w, h * d_h, kc * 64, &ms.full[c]);
-            tma_load_2d(w_s + c * kWChunkBytes + kWChunkBytes / 2, &maps.w, h * d_h + 64, kc * 64, &ms.full[c]);
+            tma_load_2d(w_s + c * kWChunkBytes, &maps.w, h * d_h, lr * K + kc * 64, &ms.full[c]);
+            tma_load_2d(w_s + c * kWChunkBytes + kWChunkBytes / 2, &maps.w, h * d_h + 64, lr * K + kc * 64,
+                        &ms.full[c]);
         }
         wait_prerequisite_grid();
         for (int c = 0; c < cpc; ++c)
-            tma_load_2d(x_s + c * x_chunk_bytes, &maps.x, h * K + (c_first + c) * 64, n0, &ms.full[c]);
+            tma_load_2d(x_s + c * x_chunk_bytes, &maps.x, h * K + (c_first + c) * 64, lr * batch + n0, &ms.full[c]);
     }
     if (warp == 1) {
         bool ok = true;
@@ -144,6 +168,21 @@ up_proj_tc_kernel(const __grid_constant__ UpMaps maps, int batch, int heads, int
     const int per = nt / ks;
     const int n_lo = (int)rank * per, n_hi = n_lo + per;
     const uint32_t part_addr = smem_u32(part);
+    const size_t HD = (size_t)heads * d_h;
+    // cross-rank mode: this rank, this tile's call number and buffer
+    int xrank = 0, tile = 0;
+    uint32_t call = 0, par = 0;
+    ExchangeLayout L{};
+    uint8_t* own = nullptr;
+    if constexpr (kXRank) {
+        wait_prerequisite_grid();  // the previous call's epoch and buffers are settled
+        xrank = xr.rank_base + lr;
+        tile = blockIdx.y * gridDim.x + blockIdx.x;
+        L = exchange_layout(batch, heads, d_h, xr.world, xr.tiles);
+        own = static_cast<uint8_t*>(xr.regions[xrank]);
+        call = __ldcg(reinterpret_cast<const unsigned int*>(own + L.epoch_off) + tile);
+        par = call & 1u;
+    }
     if (j < d_h) {
         for (int nn = n_lo; nn < n_hi; nn += 4) {
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -159,8 +198,57 @@ up_proj_tc_kernel(const __grid_constant__ UpMaps maps, int batch, int heads, int
             for (int i = 0; i < 4; ++i) {
                 const int n = n0 + nn + i;
                 if (n >= batch) continue;
-                const size_t o = (size_t)n * heads * d_h + (size_t)h * d_h + j;
-                float v = vals[i];
+                const size_t o = (size_t)n * HD + (size_t)h * d_h + j;
+                if constexpr (kXRank) {
+                    // slot `xrank` of every rank's buffer `par`
+                    const size_t slot = ((size_t)par * xr.world + xrank) * batch * HD + o;
+                    for (int p = 0; p < xr.world; ++p)
+                        reinterpret_cast<float*>(static_cast<uint8_t*>(xr.regions[p]) + L.data_off)[slot] = vals[i];
+                } else {
+                    float v = vals[i];
+                    if (gate != nullptr) v *= 1.f / (1.f + expf(-__bfloat162float(gate[o])));
+                    y[o] = to_bf16(v);
+                }
+            }
+        }
+    }
+    if constexpr (kXRank) {
+        __syncthreads();  // every slice of this tile is stored
+        if (threadIdx.x == 0) {
+            __threadfence_system();
+            const size_t fi = ((size_t)par * xr.world + xrank) * xr.tiles + tile;
+            for (int p = 0; p < xr.world; ++p)
+                st_release_sys(reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(xr.regions[p]) + L.flag_off) + fi,
+                               call + 1);
+            // wait for every rank's slice of this tile in the own region
+            const uint32_t* own_flags = reinterpret_cast<const uint32_t*>(own + L.flag_off);
+            bool ok = true;
+            const uint64_t t0 = globaltimer_ns();
+            for (int src = 0; src < xr.world && ok; ++src) {
+                const uint32_t* f = own_flags + ((size_t)par * xr.world + src) * xr.tiles + tile;
+                while (ld_acquire_sys(f) != call + 1) {
+                    if (globaltimer_ns() - t0 > xr.limit_ns) {
+                        ok = false;
+                        break;
+                    }
+                    __nanosleep(100);
+                }
+            }
+            if (!ok && xr.status != nullptr) record_error(xr.status, MLRA_ERR_DEVICE_TIMEOUT);
+            reinterpret_cast<unsigned int*>(own + L.epoch_off)[tile] = call + 1;
+            ms.xr_ok = ok;
+        }
+        __syncthreads();
+        const bool ok = ms.xr_ok != 0;
+        if (j < d_h) {
+            const float* data = reinterpret_cast<const float*>(own + L.data_off);
+            for (int nn = n_lo; nn < n_hi; ++nn) {
+                const int n = n0 + nn;
+                if (n >= batch) break;
+                const size_t o = (size_t)n * HD + (size_t)h * d_h + j;
+                float v = 0.f;
+                if (ok)
+                    for (int src = 0; src < xr.world; ++src) v += __ldcg(data + ((size_t)par * xr.world + src) * batch * HD + o);
                 if (gate != nullptr) v *= 1.f / (1.f + expf(-__bfloat162float(gate[o])));
                 y[o] = to_bf16(v);
             }
@@ -197,41 +285,91 @@ bool encode(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, u
 
 }  // namespace
 
-cudaError_t launch_up_proj(int batch, int heads, int branches, int d_c, int d_h,
-                           const __nv_bfloat16* out_lat, const __nv_bfloat16* w_uv,
-                           const __nv_bfloat16* gate, __nv_bfloat16* y, cudaStream_t stream) {
-    const int K = branches * d_c;
-    if (K % 64 != 0 || K / 64 > kMaxChunks) return cudaErrorInvalidValue;
-    const int nchunk = K / 64;
-    const int ks = nchunk % 4 == 0 ? 4 : (nchunk % 2 == 0 ? 2 : 1);  // CTAs splitting K (cluster size)
+namespace {
+
+struct UpGrid {
+    int ks, nt, cpc;
+    size_t smem;
+};
+
+UpGrid up_grid(int batch, int branches, int d_c) {
+    UpGrid g;
+    const int nchunk = branches * d_c / 64;
+    g.ks = nchunk % 4 == 0 ? 4 : (nchunk % 2 == 0 ? 2 : 1);  // CTAs splitting K (cluster size)
     // sequences per CTA: a multiple of 16 (MMA N) and of 4 * ks, at most 64
-    const int nt = batch >= kMaxNT ? kMaxNT : ceil_div(batch, 16) * 16;
+    g.nt = batch >= kMaxNT ? kMaxNT : ceil_div(batch, 16) * 16;
+    g.cpc = nchunk / g.ks;
+    // operands (the fp32 partial reuses them), then the barriers; 1024 bytes
+    // of slack for aligning the base to the 128-byte swizzle atom
+    const size_t ops = (size_t)g.cpc * (kWChunkBytes + g.nt * 128), part_bytes = (size_t)128 * g.nt * 4;
+    g.smem = (ops > part_bytes ? ops : part_bytes) + sizeof(UpSmem) + 1024;
+    return g;
+}
+
+cudaError_t launch_impl(int batch, int heads, int branches, int d_c, int d_h, const __nv_bfloat16* out_lat,
+                        const __nv_bfloat16* w_uv, const __nv_bfloat16* gate, __nv_bfloat16* y,
+                        const XRankArgs& xr, int ranks_in_launch, cudaStream_t stream) {
+    const int K = branches * d_c;
+    if (K % 64 != 0 || K / 64 > kMaxChunks || ranks_in_launch < 1) return cudaErrorInvalidValue;
+    const UpGrid g = up_grid(batch, branches, d_c);
     UpMaps maps;
-    if (!encode(&maps.w, w_uv, (uint64_t)heads * d_h, (uint64_t)K, 64, 64) ||
-        !encode(&maps.x, out_lat, (uint64_t)heads * K, (uint64_t)batch, 64, (uint32_t)nt))
+    if (!encode(&maps.w, w_uv, (uint64_t)heads * d_h, (uint64_t)K * ranks_in_launch, 64, 64) ||
+        !encode(&maps.x, out_lat, (uint64_t)heads * K, (uint64_t)batch * ranks_in_launch, 64, (uint32_t)g.nt))
         return cudaErrorInvalidValue;
-    const int cpc = nchunk / ks;
-    size_t smem = (size_t)cpc * (kWChunkBytes + nt * 128) + sizeof(UpSmem) + 64;
-    const size_t part_bytes = (size_t)128 * nt * 4;
-    if (smem < part_bytes) smem = part_bytes + 64;  // the partial reuses the operand buffers
-    smem += 1024;
-    cudaError_t e = cudaFuncSetAttribute(up_proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const bool xrank = xr.world > 0;
+    auto kernel = xrank ? up_proj_tc_kernel<true> : up_proj_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(heads * ks, ceil_div(batch, nt));
+    cfg.gridDim = dim3(heads * g.ks, ceil_div(batch, g.nt), ranks_in_launch);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = g.smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = ks;
+    attr[0].val.clusterDim.x = g.ks;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, up_proj_tc_kernel, maps, batch, heads, K, d_h, nt, ks, gate, y);
+    if (xrank) {
+        // a tile waits for the same tile of every other rank: the whole grid
+        // must be resident at once, or a waiting CTA could hold the SM that a
+        // tile it waits for needs
+        int clusters = 0;
+        cfg.numAttrs = 1;
+        e = cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg);
+        cfg.numAttrs = 2;
+        if (e != cudaSuccess) return e;
+        const long long need = (long long)heads * ceil_div(batch, g.nt) * ranks_in_launch;
+        if (clusters < need) return cudaErrorCooperativeLaunchTooLarge;
+    }
+    return cudaLaunchKernelEx(&cfg, kernel, maps, batch, heads, K, d_h, g.nt, g.ks, gate, y, xr);
+}
+
+}  // namespace
+
+int up_proj_tiles(int batch, int heads, int branches, int d_c) {
+    const UpGrid g = up_grid(batch, branches, d_c);
+    return heads * g.ks * ceil_div(batch, g.nt);
+}
+
+cudaError_t launch_up_proj(int batch, int heads, int branches, int d_c, int d_h,
+                           const __nv_bfloat16* out_lat, const __nv_bfloat16* w_uv,
+                           const __nv_bfloat16* gate, __nv_bfloat16* y, cudaStream_t stream) {
+    XRankArgs none{};
+    return launch_impl(batch, heads, branches, d_c, d_h, out_lat, w_uv, gate, y, none, 1, stream);
+}
+
+cudaError_t launch_up_proj_xrank(int batch, int heads, int branches, int d_c, int d_h,
+                                 const __nv_bfloat16* out_lat, const __nv_bfloat16* w_uv,
+                                 const __nv_bfloat16* gate, __nv_bfloat16* y, const XRankArgs& xr,
+                                 int ranks_in_launch, cudaStream_t stream) {
+    if (xr.world < 1 || xr.world > kMaxWorld || xr.regions == nullptr) return cudaErrorInvalidValue;
+    if (xr.tiles != up_proj_tiles(batch, heads, branches, d_c)) return cudaErrorInvalidValue;
+    return launch_impl(batch, heads, branches, d_c, d_h, out_lat, w_uv, gate, y, xr, ranks_in_launch, stream);
 }
 
 }  // namespace mlra

@@ -26,7 +26,8 @@
  *    nearest even.
  *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *    stream).  Work is enqueued asynchronously; no entry point allocates,
- *    frees or synchronises, except mlra_read_device_error (documented below).
+ *    frees or synchronises, except mlra_read_device_error and the
+ *    exchange-region setup calls (mlra_exchange_*; documented below).
  *  - Arguments are validated on the host before anything is enqueued; a
  *    rejected call enqueues nothing.  No C++ exception crosses this ABI.
  *  - Problems that only the device can see (a bad block-table entry or
@@ -242,6 +243,84 @@ MLRA_API mlra_status mlra_prepare(const mlra_dims* dims, int32_t d_h, const void
                                   const int32_t* seqlens, const int32_t* block_table, float rope_base,
                                   void* q_lat, void* q_rope, void* latent_cache, void* rope_cache,
                                   int32_t* device_status, void* stream);
+
+/*
+ * Branch-sharded tensor parallelism ("The Core Insight" section of the blog
+ * page: the branches can be placed on different GPUs, so each GPU reads only
+ * its own branches' latents plus the shared RoPE key -- 1.5 d_h per token
+ * against MLA's 4.5 d_h under 4-way tensor parallelism).  Rank r of a group
+ * of `world` ranks holds branches [r*B/world, (r+1)*B/world): their slice of
+ * the latent cache, q_lat and W_UV, plus a full copy of the RoPE cache and
+ * q_rope.  Each rank runs mlra_decode on its branches (with the global
+ * out_scale), then mlra_up_proj_allreduce, which multiplies its branches and
+ * sums the ranks' products, so that every rank ends with the full y.
+ *
+ * The cross-rank sum runs inside the up-projection kernel over an exchange
+ * region per rank, device memory that every rank maps: each rank stores its
+ * fp32 partial products into every rank's region and raises a flag there;
+ * each rank waits (bounded) for all flags on its own region and adds the
+ * ranks' partials in rank order, so all ranks' y are bit-identical.
+ */
+
+/* Size in bytes of one rank's exchange region for these (per-rank) sizes;
+ * 0 if the sizes are invalid.  `branches` is the rank's branch count. */
+MLRA_API size_t mlra_exchange_bytes(int32_t batch, int32_t heads, int32_t branches, int32_t d_c,
+                                    int32_t d_h, int32_t world);
+
+#define MLRA_IPC_HANDLE_BYTES 64
+
+/*
+ * Allocates a zeroed exchange region of `bytes` on the current device
+ * (cudaMalloc; released with mlra_exchange_free) and, when `ipc_handle` is
+ * not NULL, writes the MLRA_IPC_HANDLE_BYTES-byte handle through which the
+ * other processes of the group map it.  Synchronises the device, so the
+ * zeroing is complete on return.  Every rank must hold its zeroed region
+ * before any rank makes its first mlra_up_proj_allreduce call (exchange the
+ * handles through a collective that all ranks enter after this returns).
+ */
+MLRA_API mlra_status mlra_exchange_alloc(size_t bytes, void** region, void* ipc_handle);
+
+/* Maps another process's region from its handle (peer access enabled
+ * lazily); unmap with mlra_exchange_close. */
+MLRA_API mlra_status mlra_exchange_open(const void* ipc_handle, void** region);
+MLRA_API mlra_status mlra_exchange_close(void* region);
+MLRA_API mlra_status mlra_exchange_free(void* region);
+
+/* Zeroes a region (asynchronously on `stream`).  After a timeout the ranks'
+ * call counters disagree: every rank zeroes its region, the group meets at a
+ * barrier, and the next call starts afresh. */
+MLRA_API mlra_status mlra_exchange_reset(void* region, size_t bytes, void* stream);
+
+/*
+ * Branch-sharded up-projection with the cross-rank branch sum:
+ *   y[n, c] = sigmoid(gate[n, c])? * sum_{ranks s} sum_{b in s} sum_k out_lat_s[n,h,b,k] * w_uv_s[b][k][c]
+ *   out_lat, w_uv   this rank's branches (`branches` of them), layouts as
+ *                   mlra_up_proj
+ *   gate            optional bf16 [batch, heads * d_h] (NULL: no gate); the
+ *                   same values on every rank
+ *   y               bf16 [batch, heads * d_h], the full sum, on every rank
+ *   regions         DEVICE array of `world` pointers: rank s's exchange region
+ *                   as this device addresses it (its own, or mapped with
+ *                   mlra_exchange_open); each of size
+ *                   mlra_exchange_bytes(batch, heads, branches, d_c, d_h, world)
+ *   rank            this rank (0 <= rank < world <= 8)
+ *   ranks_in_launch 1 normally.  k > 1 computes ranks rank .. rank + k - 1
+ *                   in one launch on this device, with their out_lat, w_uv
+ *                   and y stacked along the leading dimension ([k, ...]);
+ *                   for checking the exchange on one device
+ *   device_status   optional int32 (device, may be NULL): MLRA_ERR_DEVICE_TIMEOUT
+ *                   is recorded if another rank's partial does not arrive
+ *                   within wait_limit_ns (the tile's y is then written as zeros)
+ * Every rank must make the same sequence of calls with the same sizes.  The
+ * whole grid must fit on the device at once (a waiting tile must never hold
+ * the SM that another tile needs): MLRA_ERR_UNSUPPORTED otherwise.  Shape
+ * limits as mlra_up_proj.
+ */
+MLRA_API mlra_status mlra_up_proj_allreduce(int32_t batch, int32_t heads, int32_t branches, int32_t d_c,
+                                            int32_t d_h, const void* out_lat, const void* w_uv,
+                                            const void* gate, void* y, void* const* regions, int32_t world,
+                                            int32_t rank, int32_t ranks_in_launch, int32_t* device_status,
+                                            uint64_t wait_limit_ns, void* stream);
 
 /*
  * Synchronises `stream`, returns the first device-side error code recorded
