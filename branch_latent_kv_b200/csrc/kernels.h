@@ -49,23 +49,24 @@ cudaError_t launch_up_proj(int batch, int heads, int branches, int d_c, int d_h,
 // ---------------------------------------------------------------------------
 // Cross-rank branch sum of the branch-sharded up-projection.  Every rank owns
 // one exchange region (device memory that every other rank can address):
-//   epoch [tiles]                u32  calls completed, per output tile
-//   flag  [2][world][tiles]      u32  flag[par][src][t] = call + 1 once rank
-//                                     src's tile t of that call has landed
-//   data  [2][world][batch][heads*d_h]  fp32 partial sums pushed by each rank
-// par = call & 1 double-buffers flags and data, so no flag is ever reset.
+//   epoch [tiles]                        u32  calls completed, per output tile
+//   data  [2][world][batch][heads*d_h]   u64  rank src's fp32 partial in the
+//                                             low half, call + 1 in the high half
+// A partial and its call tag travel in one 64-bit store, so a reader that
+// sees the tag also sees the value: no flags and no fences.  par = call & 1
+// double-buffers the data, so a rank that runs ahead into the next call never
+// overwrites a value that a slower rank has not yet read.
 constexpr int kMaxWorld = 8;
 
 struct ExchangeLayout {
-    size_t epoch_off, flag_off, data_off, total;
+    size_t epoch_off, data_off, total;
 };
 
 __host__ __device__ inline ExchangeLayout exchange_layout(int batch, int heads, int d_h, int world, int tiles) {
     ExchangeLayout L;
     L.epoch_off = 0;
-    L.flag_off = ((size_t)tiles * 4 + 255) & ~size_t(255);
-    L.data_off = L.flag_off + (((size_t)2 * world * tiles * 4 + 255) & ~size_t(255));
-    L.total = L.data_off + (((size_t)2 * world * batch * heads * d_h * 4 + 255) & ~size_t(255));
+    L.data_off = ((size_t)tiles * 4 + 255) & ~size_t(255);
+    L.total = L.data_off + (((size_t)2 * world * batch * heads * d_h * 8 + 255) & ~size_t(255));
     return L;
 }
 

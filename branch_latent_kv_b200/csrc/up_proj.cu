@@ -66,8 +66,23 @@ struct UpSmem {
     uint64_t full[kMaxChunks];
     uint64_t mma_done;
     uint32_t tmem_base;
-    int xr_ok;  // cross-rank mode: every rank's slice arrived
+    uint32_t xr_call;                // cross-rank mode: this tile's call number
+    uint8_t* xr_region[kMaxWorld];   // and every rank's exchange region
 };
+
+// Row j, columns nn .. nn + 3 of the [128 x nt] fp32 partial, summed over the
+// ks CTAs of the cluster (distributed shared memory).
+__device__ __forceinline__ float4 cluster_column_sum(uint32_t part_addr, int j, int nt, int nn, int ks) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int r = 0; r < ks; ++r) {
+        const float4 v = ld_shared_cluster_f4(map_shared_rank(part_addr + (j * nt + nn) * 4, r));
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+    }
+    return acc;
+}
 
 // kXRank: the cross-rank branch sum (a separate instantiation, so that the
 // single-device kernel carries none of its code or registers)
@@ -124,6 +139,16 @@ up_proj_tc_kernel(const __grid_constant__ UpMaps maps, int batch, int heads, int
         wait_prerequisite_grid();
         for (int c = 0; c < cpc; ++c)
             tma_load_2d(x_s + c * x_chunk_bytes, &maps.x, h * K + (c_first + c) * 64, lr * batch + n0, &ms.full[c]);
+        if constexpr (kXRank) {
+            // under the GEMM: the regions and this tile's call number (written
+            // by the previous call, which the wait above has seen complete)
+            for (int p = 0; p < xr.world; ++p) ms.xr_region[p] = static_cast<uint8_t*>(xr.regions[p]);
+            const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+            uint32_t* epoch = reinterpret_cast<uint32_t*>(ms.xr_region[xr.rank_base + lr]) + tile;
+            const uint32_t call = __ldcg(epoch);
+            ms.xr_call = call;
+            *epoch = call + 1;  // read by the next call only
+        }
     }
     if (warp == 1) {
         bool ok = true;
@@ -169,89 +194,87 @@ up_proj_tc_kernel(const __grid_constant__ UpMaps maps, int batch, int heads, int
     const int n_lo = (int)rank * per, n_hi = n_lo + per;
     const uint32_t part_addr = smem_u32(part);
     const size_t HD = (size_t)heads * d_h;
-    // cross-rank mode: this rank, this tile's call number and buffer
-    int xrank = 0, tile = 0;
-    uint32_t call = 0, par = 0;
-    ExchangeLayout L{};
-    uint8_t* own = nullptr;
-    if constexpr (kXRank) {
-        wait_prerequisite_grid();  // the previous call's epoch and buffers are settled
-        xrank = xr.rank_base + lr;
-        tile = blockIdx.y * gridDim.x + blockIdx.x;
-        L = exchange_layout(batch, heads, d_h, xr.world, xr.tiles);
-        own = static_cast<uint8_t*>(xr.regions[xrank]);
-        call = __ldcg(reinterpret_cast<const unsigned int*>(own + L.epoch_off) + tile);
-        par = call & 1u;
-    }
-    if (j < d_h) {
-        for (int nn = n_lo; nn < n_hi; nn += 4) {
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int r = 0; r < ks; ++r) {
-                const float4 v = ld_shared_cluster_f4(map_shared_rank(part_addr + (j * nt + nn) * 4, r));
-                acc.x += v.x;
-                acc.y += v.y;
-                acc.z += v.z;
-                acc.w += v.w;
-            }
-            const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
+    if constexpr (!kXRank) {
+        if (j < d_h) {
+            for (int nn = n_lo; nn < n_hi; nn += 4) {
+                const float4 acc = cluster_column_sum(part_addr, j, nt, nn, ks);
+                const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int n = n0 + nn + i;
-                if (n >= batch) continue;
-                const size_t o = (size_t)n * HD + (size_t)h * d_h + j;
-                if constexpr (kXRank) {
-                    // slot `xrank` of every rank's buffer `par`
-                    const size_t slot = ((size_t)par * xr.world + xrank) * batch * HD + o;
-                    for (int p = 0; p < xr.world; ++p)
-                        reinterpret_cast<float*>(static_cast<uint8_t*>(xr.regions[p]) + L.data_off)[slot] = vals[i];
-                } else {
+                for (int i = 0; i < 4; ++i) {
+                    const int n = n0 + nn + i;
+                    if (n >= batch) continue;
+                    const size_t o = (size_t)n * HD + (size_t)h * d_h + j;
                     float v = vals[i];
                     if (gate != nullptr) v *= 1.f / (1.f + expf(-__bfloat162float(gate[o])));
                     y[o] = to_bf16(v);
                 }
             }
         }
-    }
-    if constexpr (kXRank) {
-        __syncthreads();  // every slice of this tile is stored
-        if (threadIdx.x == 0) {
-            __threadfence_system();
-            const size_t fi = ((size_t)par * xr.world + xrank) * xr.tiles + tile;
-            for (int p = 0; p < xr.world; ++p)
-                st_release_sys(reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(xr.regions[p]) + L.flag_off) + fi,
-                               call + 1);
-            // wait for every rank's slice of this tile in the own region
-            const uint32_t* own_flags = reinterpret_cast<const uint32_t*>(own + L.flag_off);
-            bool ok = true;
-            const uint64_t t0 = globaltimer_ns();
-            for (int src = 0; src < xr.world && ok; ++src) {
-                const uint32_t* f = own_flags + ((size_t)par * xr.world + src) * xr.tiles + tile;
-                while (ld_acquire_sys(f) != call + 1) {
-                    if (globaltimer_ns() - t0 > xr.limit_ns) {
-                        ok = false;
-                        break;
-                    }
-                    __nanosleep(100);
+    } else {
+        const int world = xr.world, xrank = xr.rank_base + lr;
+        const ExchangeLayout L = exchange_layout(batch, heads, d_h, world, xr.tiles);
+        const uint32_t call = ms.xr_call, tag = call + 1;
+        const size_t buf = (size_t)(call & 1u) * world;  // first slot of this call's buffer
+        if (j < d_h) {
+            // push: this rank's slice into slot xrank of every rank's buffer
+            for (int nn = n_lo; nn < n_hi; nn += 4) {
+                const float4 acc = cluster_column_sum(part_addr, j, nt, nn, ks);
+                const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int n = n0 + nn + i;
+                    if (n >= batch) continue;
+                    const size_t o = (size_t)n * HD + (size_t)h * d_h + j;
+                    const uint64_t word = (uint64_t)__float_as_uint(vals[i]) | ((uint64_t)tag << 32);
+                    for (int p = 0; p < world; ++p)
+                        st_relaxed_sys_u64(reinterpret_cast<uint64_t*>(ms.xr_region[p] + L.data_off) +
+                                               ((buf + xrank) * batch) * HD + o, word);
                 }
             }
-            if (!ok && xr.status != nullptr) record_error(xr.status, MLRA_ERR_DEVICE_TIMEOUT);
-            reinterpret_cast<unsigned int*>(own + L.epoch_off)[tile] = call + 1;
-            ms.xr_ok = ok;
-        }
-        __syncthreads();
-        const bool ok = ms.xr_ok != 0;
-        if (j < d_h) {
-            const float* data = reinterpret_cast<const float*>(own + L.data_off);
-            for (int nn = n_lo; nn < n_hi; ++nn) {
-                const int n = n0 + nn;
-                if (n >= batch) break;
-                const size_t o = (size_t)n * HD + (size_t)h * d_h + j;
-                float v = 0.f;
-                if (ok)
-                    for (int src = 0; src < xr.world; ++src) v += __ldcg(data + ((size_t)par * xr.world + src) * batch * HD + o);
-                if (gate != nullptr) v *= 1.f / (1.f + expf(-__bfloat162float(gate[o])));
-                y[o] = to_bf16(v);
+            // sum: every rank's slot in rank order, four columns' loads in
+            // flight at once; a slot whose tag is not this call's is polled
+            // (bounded), and a sum with a missing slot is written as zero
+            const uint64_t* data = reinterpret_cast<const uint64_t*>(ms.xr_region[xrank] + L.data_off);
+            bool alive = true;
+            uint64_t t0 = 0;
+            for (int nn = n_lo; nn < n_hi; nn += 4) {
+                uint64_t w[4][kMaxWorld];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int src = 0; src < kMaxWorld; ++src)
+                        if (src < world && n0 + nn + i < batch)
+                            w[i][src] = ld_relaxed_sys_u64(data + ((buf + src) * batch) * HD +
+                                                           (size_t)(n0 + nn + i) * HD + (size_t)h * d_h + j);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int n = n0 + nn + i;
+                    if (n >= batch) continue;
+                    const size_t o = (size_t)n * HD + (size_t)h * d_h + j;
+                    float v = 0.f;
+                    bool complete = true;
+#pragma unroll
+                    for (int src = 0; src < kMaxWorld; ++src) {
+                        if (src >= world) break;
+                        uint64_t x = w[i][src];
+                        while ((uint32_t)(x >> 32) != tag && alive) {
+                            const uint64_t now = globaltimer_ns();
+                            if (t0 == 0) t0 = now;
+                            if (now - t0 > xr.limit_ns) {
+                                alive = false;
+                                break;
+                            }
+                            x = ld_relaxed_sys_u64(data + ((buf + src) * batch) * HD + o);
+                        }
+                        if ((uint32_t)(x >> 32) == tag) v += __uint_as_float((uint32_t)x);
+                        else complete = false;
+                    }
+                    if (!complete) v = 0.f;
+                    if (gate != nullptr) v *= 1.f / (1.f + expf(-__bfloat162float(gate[o])));
+                    y[o] = to_bf16(v);
+                }
             }
+            if (!alive && xr.status != nullptr) record_error(xr.status, MLRA_ERR_DEVICE_TIMEOUT);
         }
     }
     cluster_sync();  // no CTA leaves while another still reads its shared memory
