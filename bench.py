@@ -14,8 +14,9 @@ roofline: the decode kernel alone, CUDA events around each of K decode-only
 graph replays (same rotation), algorithmic KV bytes / mean duration.
 e2e: the same metric through the public Python API (DecodeStep: one graph
 launch per step) with the step's inputs (queries, block table, seqlens)
-copied from pinned host memory and the result y copied back, inside the
-timed region, one host synchronisation per step.
+brought in from pinned host memory (one mlra_copy_ranges launch) and the
+result y written back into pinned host memory by the up-projection, inside
+the timed region, one host synchronisation per step.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
        [--impl ours|reference]
@@ -403,8 +404,9 @@ def main():
 
     # end to end through the public API, host buffers: a DecodeStep per KV
     # copy (the same bound device inputs), each step one graph launch that
-    # copies the inputs from pinned host memory, runs both kernels and copies
-    # y back; the host waits for every step
+    # reads the inputs from pinned host memory (one copy launch), runs both
+    # kernels and writes y into pinned host memory; the host waits for every
+    # step
     h_in = {"q_lat": x.q_lat.cpu().pin_memory(), "q_rope": x.q_rope.cpu().pin_memory(),
             "block_table": x.block_table.cpu().pin_memory(), "seqlens": x.seqlens.cpu().pin_memory()}
     h_y = torch.empty(y.shape, dtype=y.dtype).pin_memory()

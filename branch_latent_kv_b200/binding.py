@@ -87,6 +87,9 @@ def library() -> ctypes.CDLL:
             lib.mlra_up_proj_allreduce.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, i32, i32, i32,
                                                    vp, ctypes.c_uint64, vp]
             lib.mlra_up_proj_allreduce.restype = ctypes.c_int
+            lib.mlra_copy_ranges.argtypes = [i32, ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                             ctypes.POINTER(ctypes.c_uint64), vp]
+            lib.mlra_copy_ranges.restype = ctypes.c_int
             lib.mlra_read_device_error.argtypes = [vp, vp]
             lib.mlra_read_device_error.restype = ctypes.c_int
             lib.mlra_status_string.argtypes = [ctypes.c_int]
@@ -238,7 +241,10 @@ def _up_proj(out_lat, w_uv, gate, d_h, y, stream) -> torch.Tensor:
     if y is None:
         y = torch.empty((N, H * d_h), dtype=torch.bfloat16, device=dev)
     else:
-        _require(y, "y", torch.bfloat16, 2, dev)
+        # y may be pinned host memory: the kernel then writes it over PCIe
+        _require(y, "y", torch.bfloat16, 2, y.device if y.device.type == "cpu" else dev)
+        if y.device.type == "cpu" and not y.is_pinned():
+            raise ValueError("a host y must be pinned memory")
         if tuple(y.shape) != (N, H * d_h):
             raise ValueError("y must be [N, heads*d_h]")
     if gate is None:
@@ -422,3 +428,33 @@ def mlra_up_proj_allreduce(out_lat, w_uv, regions: torch.Tensor, rank: int, gate
                                           int(wait_limit_ns), _stream_ptr(stream, dev))
     _check(st, "mlra_up_proj_allreduce")
     return y
+
+
+def mlra_copy_ranges(pairs, stream=None, device: Optional[torch.device] = None) -> None:
+    """Copy each (src, dst) tensor pair (same byte size; device or pinned host
+    memory, 16-byte aligned, contiguous) in one launch of the SMs (see
+    mlra_copy_ranges in mlra.h)."""
+    pairs = list(pairs)
+    if not 1 <= len(pairs) <= 8:
+        raise ValueError("mlra_copy_ranges takes 1 to 8 pairs")
+    for k, (s_t, d_t) in enumerate(pairs):
+        if s_t.numel() * s_t.element_size() != d_t.numel() * d_t.element_size():
+            raise ValueError(f"mlra_copy_ranges: pair {k} differs in size")
+    pairs = [(s_t, d_t) for s_t, d_t in pairs if s_t.numel() > 0]  # empty ranges copy nothing
+    if not pairs:
+        return
+    n = len(pairs)
+    src, dst, nb = (ctypes.c_void_p * n)(), (ctypes.c_void_p * n)(), (ctypes.c_uint64 * n)()
+    dev = device
+    for k, (s_t, d_t) in enumerate(pairs):
+        for t, what in ((s_t, "src"), (d_t, "dst")):
+            if not t.is_contiguous():
+                raise ValueError(f"mlra_copy_ranges: {what} {k} must be contiguous")
+            if t.device.type == "cpu" and not t.is_pinned():
+                raise ValueError(f"mlra_copy_ranges: host {what} {k} must be pinned memory")
+            if t.device.type == "cuda" and dev is None:
+                dev = t.device
+        src[k], dst[k], nb[k] = _ptr(s_t), _ptr(d_t), s_t.numel() * s_t.element_size()
+    if dev is None:
+        dev = torch.device("cuda", torch.cuda.current_device())
+    _check(library().mlra_copy_ranges(n, src, dst, nb, _stream_ptr(stream, dev)), "mlra_copy_ranges")

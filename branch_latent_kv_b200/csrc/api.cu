@@ -147,6 +147,8 @@ mlra_status mlra_decode_simt(const mlra_dims* dims, const void* q_lat, const voi
 }
 
 namespace {
+const void* device_address(const void* p);
+
 mlra_status up_proj_impl(int32_t batch, int32_t heads, int32_t branches, int32_t d_c, int32_t d_h,
                          const void* out_lat, const void* w_uv, const void* gate, void* y, void* stream) {
     if (batch < 1 || heads < 1 || branches < 1 || d_c < 1 || d_h < 1) return MLRA_ERR_INVALID_ARG;
@@ -155,11 +157,13 @@ mlra_status up_proj_impl(int32_t batch, int32_t heads, int32_t branches, int32_t
     if ((int64_t)batch * heads * d_h > INT32_MAX) return MLRA_ERR_INVALID_ARG;
     const int K = branches * d_c;
     if (K % 64 != 0 || K > 512 || (d_h != 64 && d_h != 128)) return MLRA_ERR_UNSUPPORTED;
+    void* y_dev = const_cast<void*>(device_address(y));  // y may be mapped pinned host memory
+    if (y_dev == nullptr || !aligned16(y_dev)) return MLRA_ERR_INVALID_ARG;
     return cuda_status(launch_up_proj(batch, heads, branches, d_c, d_h,
                                       static_cast<const __nv_bfloat16*>(out_lat),
                                       static_cast<const __nv_bfloat16*>(w_uv),
                                       static_cast<const __nv_bfloat16*>(gate),
-                                      static_cast<__nv_bfloat16*>(y),
+                                      static_cast<__nv_bfloat16*>(y_dev),
                                       static_cast<cudaStream_t>(stream)));
 }
 }  // namespace
@@ -263,6 +267,57 @@ mlra_status mlra_up_proj_allreduce(int32_t batch, int32_t heads, int32_t branche
                                                static_cast<cudaStream_t>(stream));
     if (e == cudaErrorCooperativeLaunchTooLarge) return MLRA_ERR_UNSUPPORTED;
     return cuda_status(e);
+}
+
+namespace {
+// The address through which the device reaches `p` (device, managed or
+// mapped pinned host memory), or null for memory the device cannot address.
+const void* device_address(const void* p) {
+    if (p == nullptr) return nullptr;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();  // clear the error state the failed query leaves
+        return nullptr;
+    }
+    switch (at.type) {
+        case cudaMemoryTypeDevice:
+        case cudaMemoryTypeManaged:
+        case cudaMemoryTypeHost:
+            return at.devicePointer;
+        default:
+            return nullptr;
+    }
+}
+}  // namespace
+
+mlra_status mlra_copy_ranges(int32_t count, const void* const* src, void* const* dst, const uint64_t* bytes,
+                             void* stream) {
+    if (count < 1 || count > kMaxRanges || src == nullptr || dst == nullptr || bytes == nullptr)
+        return MLRA_ERR_INVALID_ARG;
+    CopyRanges r;
+    r.count = count;
+    for (int k = 0; k < count; ++k) {
+        if (!aligned16(src[k]) || !aligned16(dst[k])) return MLRA_ERR_INVALID_ARG;
+        const void* s_dev = device_address(src[k]);
+        void* d_dev = const_cast<void*>(device_address(dst[k]));
+        if (s_dev == nullptr || d_dev == nullptr || !aligned16(s_dev) || !aligned16(d_dev))
+            return MLRA_ERR_INVALID_ARG;
+        // no overlap between any destination and any range
+        r.src[k] = s_dev;
+        r.dst[k] = d_dev;
+        r.bytes[k] = (size_t)bytes[k];
+    }
+    for (int a = 0; a < count; ++a)
+        for (int c = 0; c < count; ++c) {
+            const uintptr_t d0 = reinterpret_cast<uintptr_t>(r.dst[a]), d1 = d0 + r.bytes[a];
+            const uintptr_t s0 = reinterpret_cast<uintptr_t>(r.src[c]), s1 = s0 + r.bytes[c];
+            const uintptr_t e0 = reinterpret_cast<uintptr_t>(r.dst[c]), e1 = e0 + r.bytes[c];
+            if (r.bytes[a] && r.bytes[c] && d0 < s1 && s0 < d1) return MLRA_ERR_INVALID_ARG;
+            if (a != c && r.bytes[a] && r.bytes[c] && d0 < e1 && e0 < d1) return MLRA_ERR_INVALID_ARG;
+        }
+    const int sms = device_sm_count();
+    if (sms <= 0) return MLRA_ERR_CUDA;
+    return cuda_status(launch_copy_ranges(r, sms, static_cast<cudaStream_t>(stream)));
 }
 
 mlra_status mlra_prepare(const mlra_dims* dims, int32_t d_h, const void* q_c, const void* q_r,

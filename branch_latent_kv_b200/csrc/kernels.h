@@ -92,6 +92,17 @@ cudaError_t launch_up_proj_xrank(int batch, int heads, int branches, int d_c, in
                                  const __nv_bfloat16* gate, __nv_bfloat16* y, const XRankArgs& xr,
                                  int ranks_in_launch, cudaStream_t stream);
 
+// Byte ranges copied by one launch of the SMs (device or mapped pinned host
+// memory, 16-byte aligned, validated on the host).
+constexpr int kMaxRanges = 8;
+struct CopyRanges {
+    const void* src[kMaxRanges];
+    void* dst[kMaxRanges];
+    size_t bytes[kMaxRanges];
+    int count;
+};
+cudaError_t launch_copy_ranges(const CopyRanges& r, int sms, cudaStream_t stream);
+
 // Arguments of the decode pre-step (validated on the host).
 struct PrepareArgs {
     const __nv_bfloat16* q_c;     // [N, H, d_h]

@@ -45,12 +45,14 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "peer.cuh"
 #include "sm100.cuh"
 
 namespace mlra {
 namespace {
 
 using namespace sm100;
+using namespace peer;
 
 constexpr int kThreads = 128;
 constexpr int kMaxChunks = 8;      // K <= 512

@@ -3,9 +3,11 @@
 A serving loop calls the same decode step every token with the same buffer
 shapes.  ``DecodeStep`` validates the arguments once (one eager call of
 ``mlra_decode`` and, when ``w_uv`` is given, ``mlra_up_proj``), then captures
-the step -- optionally with the host-to-device copies of its inputs and the
-device-to-host copy of its result -- into a CUDA graph, so each step costs
-one graph launch on the host.  All arithmetic is in the library's kernels;
+the step -- optionally with the host-to-device transfer of its inputs and the
+device-to-host transfer of its result -- into a CUDA graph, so each step costs
+one graph launch on the host.  The inputs cross PCIe in one launch of
+``mlra_copy_ranges`` (SM loads from the mapped pinned pages); with ``w_uv``
+the up-projection writes y straight into the pinned host output.  All arithmetic is in the library's kernels;
 this module only arranges launches.
 
 Buffers are bound at construction: write the next step's inputs into the
@@ -55,6 +57,10 @@ class DecodeStep:
                 raise ValueError(f"host_inputs[{name!r}] must be pinned CPU memory")
             if h.shape != d.shape or h.dtype != d.dtype:
                 raise ValueError(f"host_inputs[{name!r}] must match the device tensor's shape and dtype")
+            if not h.is_contiguous() or h.data_ptr() % 16 != 0:
+                raise ValueError(f"host_inputs[{name!r}] must be contiguous and 16-byte aligned")
+        if len(self.host_inputs) > 8:
+            raise ValueError("at most 8 host inputs")
         dims = b.decode_dims(q_lat, q_rope, latent_cache, block_table)
         self.workspace = workspace if workspace is not None else torch.zeros(
             b.mlra_decode_workspace_bytes(dims), dtype=torch.uint8, device=dev)
@@ -68,6 +74,8 @@ class DecodeStep:
         if host_output is not None:
             if host_output.device.type != "cpu" or not host_output.is_pinned():
                 raise ValueError("host_output must be pinned CPU memory")
+            if not host_output.is_contiguous() or host_output.data_ptr() % 16 != 0:
+                raise ValueError("host_output must be contiguous and 16-byte aligned")
             if host_output.shape != result.shape or host_output.dtype != result.dtype:
                 raise ValueError("host_output must match the result's shape and dtype")
         self.host_output = host_output
@@ -88,14 +96,19 @@ class DecodeStep:
 
     def _body(self, stream, copies: bool):
         with torch.cuda.stream(stream):
-            if copies:
-                for name, h in self.host_inputs.items():
-                    self.inputs[name].copy_(h, non_blocking=True)
+            if copies and self.host_inputs:
+                # every host input crosses PCIe in one launch (SM loads from
+                # the mapped pinned pages), not one DMA copy per tensor
+                b.mlra_copy_ranges([(h, self.inputs[name]) for name, h in self.host_inputs.items()],
+                                   stream=stream, device=self.device)
             b.mlra_decode(*self._args, out=self.out, workspace=self.workspace, stream=stream)
+            direct = copies and self.host_output is not None and self._w_uv is not None
             if self._w_uv is not None:
-                b.mlra_up_proj(self.out, self._w_uv, d_h=self._d_h, y=self.y, stream=stream)
-            if copies and self.host_output is not None:
-                self.host_output.copy_(self.y if self.y is not None else self.out, non_blocking=True)
+                # with a host output, the up-projection writes y straight into it
+                b.mlra_up_proj(self.out, self._w_uv, d_h=self._d_h, y=self.host_output if direct else self.y,
+                               stream=stream)
+            if copies and self.host_output is not None and not direct:
+                self.host_output.copy_(self.out, non_blocking=True)
 
     def __call__(self) -> torch.Tensor:
         self.graph.replay()

@@ -182,7 +182,9 @@ MLRA_API mlra_status mlra_decode_static_scratch(const mlra_dims* dims, const voi
  * fp32 accumulation, bf16 result.
  *   out_lat bf16 [batch, heads, branches, d_c]  (the output of mlra_decode)
  *   w_uv    bf16 [branches, d_c, heads * d_h]
- *   y       bf16 [batch, heads * d_h]           written
+ *   y       bf16 [batch, heads * d_h]           written; device memory or
+ *           pinned host memory the device can map (the kernel then writes
+ *           the result straight over PCIe, no separate copy)
  * Supported: branches * d_c in {64, 128, ..., 512} (a multiple of 64),
  * d_h in {64, 128}, any batch >= 1.
  */
@@ -321,6 +323,20 @@ MLRA_API mlra_status mlra_up_proj_allreduce(int32_t batch, int32_t heads, int32_
                                             const void* gate, void* y, void* const* regions, int32_t world,
                                             int32_t rank, int32_t ranks_in_launch, int32_t* device_status,
                                             uint64_t wait_limit_ns, void* stream);
+
+/*
+ * Copies `count` (1..8) byte ranges, dst[k] <- src[k] (bytes[k] bytes each),
+ * in one kernel launch whose SMs issue the loads and stores.  Every pointer
+ * is device memory, managed memory or pinned host memory the device can map
+ * (cudaHostAlloc / cudaMallocHost, or registered with cudaHostRegister),
+ * 16-byte aligned; no destination may overlap any range.  Host pointers are
+ * translated to their device addresses here.  For the host-to-device leg of
+ * a serving step: a few small input tensors cross PCIe in one launch instead
+ * of one DMA copy (and its setup latency) each.  Pageable host memory is
+ * rejected (MLRA_ERR_INVALID_ARG).  Asynchronous on `stream`.
+ */
+MLRA_API mlra_status mlra_copy_ranges(int32_t count, const void* const* src, void* const* dst,
+                                      const uint64_t* bytes, void* stream);
 
 /*
  * Synchronises `stream`, returns the first device-side error code recorded

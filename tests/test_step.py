@@ -61,3 +61,18 @@ def test_rejects_unpinned_host_buffers():
     with pytest.raises(ValueError):
         DecodeStep(x.q_lat, x.q_rope, x.latent_cache, x.rope_cache, x.block_table, x.seqlens,
                    x.scale, x.out_scale, host_inputs={"q_lat": x.q_lat.cpu()})
+
+
+def test_host_output_without_up_projection():
+    """Decode only: the latent output is copied to the pinned host buffer."""
+    x = make_inputs(WORKLOADS["decode_2p9b"].with_(batch=3, seqlen=700), seed=7).to("cuda")
+    h_in = {"q_lat": x.q_lat.cpu().pin_memory(), "q_rope": x.q_rope.cpu().pin_memory(),
+            "block_table": x.block_table.cpu().pin_memory(), "seqlens": x.seqlens.cpu().pin_memory()}
+    d_in = {k: torch.empty_like(v, device="cuda") for k, v in h_in.items()}
+    h_out = torch.empty(x.q_lat.shape, dtype=torch.bfloat16).pin_memory()
+    step = DecodeStep(d_in["q_lat"], d_in["q_rope"], x.latent_cache, x.rope_cache, d_in["block_table"],
+                      d_in["seqlens"], x.scale, x.out_scale, host_inputs=h_in, host_output=h_out)
+    step()
+    torch.cuda.synchronize()
+    out_ref, _ = _eager(x)
+    assert torch.equal(h_out, out_ref.cpu())
