@@ -458,6 +458,11 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
         fence_barrier_init();
     }
     if (warp == 0) {
+        // descriptor fetches overlap the loads of the lengths below
+        prefetch_tensormap(&maps.lat);
+        prefetch_tensormap(&maps.rope);
+        prefetch_tensormap(&maps.q);
+        prefetch_tensormap(&maps.qr);
         const int total = warp_cost_prefix(a.seqlens, a.batch, P, a.max_pages);
         const int chunk = plan_chunk(total, a.num_ctas);
         int n0 = a.batch, cum0 = total;
@@ -468,10 +473,6 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
             misc.plan[2] = n0;
             misc.plan[3] = cum0;
         }
-        prefetch_tensormap(&maps.lat);
-        prefetch_tensormap(&maps.rope);
-        prefetch_tensormap(&maps.q);
-        prefetch_tensormap(&maps.qr);
     }
     if (warp == 1) {
         tmem_alloc(&misc.tmem_base, C::TMEM_COLS);
@@ -493,6 +494,9 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
             int n = misc.plan[2], cum = misc.plan[3], next_len = first_len(a, n);
             int L, tiles, tb, te;
             uint32_t pc = 0, tc = 0, sc = 0;
+            // the cache is read once per step: its lines go first, and the
+            // block table, lengths, queries and partials stay in L2
+            const uint64_t stream_policy = l2_policy_evict_first();
             bool ok = true;
             while (ok && next_segment(a, n, cum, A0, A1, L, tiles, tb, te, next_len)) {
                 // the sequence's queries, once the previous range has finished
@@ -534,8 +538,8 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                     for (int q = 0; q < npages; ++q) {
                         const int page = __shfl_sync(0xffffffffu, win_val, page0 + q - win_base);
                         if (lane == 0)
-                            tma_load_2d(sm + C::OFF_ROPE + rs * C::ROPE_BYTES + q * P * C::ROPE_ROW, &maps.rope,
-                                        0, page * P, &misc.rope_full[rs]);
+                            tma_load_2d_hint(sm + C::OFF_ROPE + rs * C::ROPE_BYTES + q * P * C::ROPE_ROW, &maps.rope,
+                                             0, page * P, &misc.rope_full[rs], stream_policy);
                     }
                     ++tc;
                     for (int sp = 0; sp < C::NSTEP * C::PPS && ok; ++sp) {
@@ -551,9 +555,10 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                             const int page = __shfl_sync(0xffffffffu, win_val, page0 + q - win_base);
                             if (lane == 0) {
                                 uint8_t* dst = sm + C::OFF_PAIR + stage * C::PAIR_BYTES + q * P * 128;
-                                tma_load_2d(dst, &maps.lat, chunk0 * 64, page * P, &misc.pair_full[stage]);
-                                tma_load_2d(dst + C::CHUNK_BYTES, &maps.lat, chunk0 * 64 + 64, page * P,
-                                            &misc.pair_full[stage]);
+                                tma_load_2d_hint(dst, &maps.lat, chunk0 * 64, page * P, &misc.pair_full[stage],
+                                                 stream_policy);
+                                tma_load_2d_hint(dst + C::CHUNK_BYTES, &maps.lat, chunk0 * 64 + 64, page * P,
+                                                 &misc.pair_full[stage], stream_policy);
                             }
                         }
                         ++pc;
