@@ -7,11 +7,13 @@ softmax, value-absorbed output, split merge, out_scale) followed by the
 per-branch W_UV up-projection and branch sum (mlra_up_proj, one kernel).
 
 value: algorithmic KV bytes of all ranks' steps / device time (GB/s), the
-KV cache resident in HBM, each step one CUDA-graph replay of both kernels.
+KV cache resident in HBM, the steps replayed from a CUDA graph holding one
+step (both kernels) per KV copy.
 L2 cannot serve the cache: each step reads the next of k copies of the
 pools, k * KV bytes >= 4x the L2 size.
-roofline: the decode kernel alone, CUDA events around each of K decode-only
-graph replays (same rotation), algorithmic KV bytes / mean duration.
+roofline: the decode kernel alone, a graph of back-to-back decode launches
+(one per KV copy, same rotation) replayed until at least K launches, CUDA
+events around the region, algorithmic KV bytes / mean duration per launch.
 e2e: the same metric through the public Python API (DecodeStep: one graph
 launch per step) with the step's inputs (queries, block table, seqlens)
 brought in from pinned host memory (one mlra_copy_ranges launch) and the
@@ -53,7 +55,10 @@ FALLBACK_HBM_GBS = 6650.0
 # ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the
 # hash of the kernel sources it was taken on.  Reported as null whenever the
 # kernel sources differ from the captured ones.
-TRAFFIC_CAPTURE = {"sources_sha1": "98efd80ef51673f256d36a0e78337dc871473fb0", "bytes_per_launch": 151417600 + 4464128}
+# DRAM bytes (read + write) of one decode launch from the committed ncu
+# capture, valid only for that workload and those kernel sources
+TRAFFIC_CAPTURE = {"workload": "decode_2p9b", "sources_sha1": "98efd80ef51673f256d36a0e78337dc871473fb0",
+                   "bytes_per_launch": 151417600 + 4464128}
 KERNEL_SOURCES = ["branch_latent_kv_b200/csrc/decode_tc.cu", "branch_latent_kv_b200/csrc/sm100.cuh",
                   "branch_latent_kv_b200/csrc/common.cuh"]
 
@@ -339,27 +344,35 @@ def main():
             pg.destroy_process_group()
         return
 
-    # The device-resident step is replayed from CUDA graphs: one graph per KV
-    # copy holding both kernels of the step, so the up-projection (launched as
-    # a programmatic dependent) loads its weights on SMs the decode kernel has
-    # released while the decode kernel finishes.  The decode kernel's own
-    # duration (the roofline figure) is timed in a second region of
-    # decode-only graph replays with CUDA events around each launch.
+    # The device-resident steps are replayed from CUDA graphs.  One graph
+    # holds one step per KV copy (`copies` steps, both kernels each), the way
+    # a serving loop launches its kernels back to back from a graph rather
+    # than one graph launch per kernel; within a step the up-projection
+    # (launched as a programmatic dependent) loads its weights on SMs the
+    # decode kernel has released while the decode kernel finishes.  Steps
+    # left over when K is not a multiple of `copies` replay one-step graphs.
+    # The decode kernel's own duration (the roofline figure) is timed in a
+    # second region: a graph of `copies` decode launches, replayed until at
+    # least K launches, events around the region, divided by the launches.
     step(0)
     torch.cuda.synchronize(dev)
     cap = torch.cuda.Stream(dev)
     cap.wait_stream(stream)
-    step_graphs, decode_graphs = [], []
+    step_graphs = []
     for c in range(copies):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=cap):
             decode_call(c)
             up_call()
         step_graphs.append(g)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=cap):
+    chain_steps, chain_decode = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(chain_steps, stream=cap):
+        for c in range(copies):
             decode_call(c)
-        decode_graphs.append(g)
+            up_call()
+    with torch.cuda.graph(chain_decode, stream=cap):
+        for c in range(copies):
+            decode_call(c)
     torch.cuda.synchronize(dev)
 
     sampler = ClockSampler(local)
@@ -368,39 +381,43 @@ def main():
     t_warm = time.time()
     i = 0
     while i < args.warmup or time.time() - t_warm < 1.5:
-        step_graphs[i % copies].replay()
-        i += 1
-        if i % 256 == 0:
+        chain_steps.replay()
+        i += copies
+        if i % 256 < copies:
             torch.cuda.synchronize(dev)
     torch.cuda.synchronize(dev)
     if pg:
         pg.barrier()
     torch.cuda.synchronize(dev)
+    n_chain, n_rest = divmod(args.steps, copies)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
-    for k in range(args.steps):
-        step_graphs[(i + k) % copies].replay()
+    for _ in range(n_chain):
+        chain_steps.replay()
+    for k in range(n_rest):
+        step_graphs[k].replay()
     end.record(stream)
     torch.cuda.synchronize(dev)
     if pg:
         pg.barrier()
     torch.cuda.synchronize(dev)
     elapsed_ms = start.elapsed_time(end)
-    # decode kernel alone: events around each launch
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    for k in range(args.steps):
-        evs[k][0].record(stream)
-        decode_graphs[(i + k) % copies].replay()
-        evs[k][1].record(stream)
+    # decode kernel alone: at least K launches, events around the region
+    reps = -(-args.steps // copies)
+    d_start, d_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d_start.record(stream)
+    for _ in range(reps):
+        chain_decode.replay()
+    d_end.record(stream)
     torch.cuda.synchronize(dev)
     t_load1 = time.time()
     if pg:
         pg.barrier()
     torch.cuda.synchronize(dev)
-    decode_ms = sum(e0.elapsed_time(e1) for e0, e1 in evs) / args.steps
+    decode_launches = reps * copies
+    decode_ms = d_start.elapsed_time(d_end) / decode_launches
     elapsed_ms, decode_ms = max_over_ranks([elapsed_ms, decode_ms], pg, dev)
-    del step_graphs, decode_graphs
+    del step_graphs, chain_steps, chain_decode
 
     # end to end through the public API, host buffers: a DecodeStep per KV
     # copy (the same bound device inputs), each step one graph launch that
@@ -450,7 +467,7 @@ def main():
     gbs = kv * world * args.steps / (elapsed_ms / 1e3) / 1e9
     achieved = kv / (decode_ms / 1e3) / 1e9
     traffic = None
-    if TRAFFIC_CAPTURE["sources_sha1"] == kernel_sources_sha1():
+    if TRAFFIC_CAPTURE["workload"] == args.workload and TRAFFIC_CAPTURE["sources_sha1"] == kernel_sources_sha1():
         traffic = TRAFFIC_CAPTURE["bytes_per_launch"]
     line = {
         "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -463,8 +480,9 @@ def main():
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": traffic,
                      "kernel": "decode_tc_kernel (mlra_decode: split-KV decode with its in-kernel "
-                               "LSE merge), CUDA events around each of K decode-only graph launches "
-                               "timed after the step region, same KV rotation",
+                               "LSE merge), CUDA events around a region of >= K back-to-back decode "
+                               "launches (graphs of one launch per KV copy) timed after the step "
+                               "region, same KV rotation",
                      "peak_source": f"{peak_kind} hbm_gbs"},
         "e2e": {"value": kv * world * args.steps / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
