@@ -162,3 +162,64 @@ def test_plan_model_bounds_the_slowest_cta():
     flat = plan_model.plan([8192] * 16, 64, 128, 148)
     counts = [flat[4 * c + 1] - flat[4 * c] for c in range(148)]
     assert max(counts) == 7 and sum(counts) == 16 * 64
+
+
+def _up_grid_tiles(batch, heads, branches, d_c):
+    """Output tiles of the up-projection grid: K = branches * d_c split over a
+    cluster of ks CTAs (4, else 2, else 1 dividing K / 64), up to 64 sequences
+    (a multiple of 16) per CTA."""
+    nchunk = branches * d_c // 64
+    ks = 4 if nchunk % 4 == 0 else (2 if nchunk % 2 == 0 else 1)
+    nt = 64 if batch >= 64 else -(-batch // 16) * 16
+    return heads * ks * -(-batch // nt)
+
+
+@pytest.mark.parametrize("batch,heads,branches,d_c,d_h,world", [
+    (16, 16, 1, 128, 128, 4), (80, 4, 2, 256, 128, 2), (5, 8, 2, 64, 64, 2), (16, 16, 4, 128, 128, 1),
+])
+def test_exchange_bytes_follow_the_documented_layout(batch, heads, branches, d_c, d_h, world):
+    """epoch [tiles] u32, then data [2][world][batch][heads*d_h] u64, each
+    section rounded up to 256 bytes."""
+    up256 = lambda v: (v + 255) // 256 * 256
+    tiles = _up_grid_tiles(batch, heads, branches, d_c)
+    want = up256(tiles * 4) + up256(2 * world * batch * heads * d_h * 8)
+    assert b.mlra_exchange_bytes(batch, heads, branches, d_c, d_h, world) == want
+
+
+def test_exchange_and_allreduce_reject_bad_arguments_on_the_host():
+    lib = b.library()
+    assert lib.mlra_exchange_bytes(16, 16, 1, 128, 128, 0) == 0
+    assert lib.mlra_exchange_bytes(16, 16, 1, 128, 128, 9) == 0
+    assert lib.mlra_exchange_bytes(0, 16, 1, 128, 128, 2) == 0
+    assert lib.mlra_exchange_bytes(16, 16, 1, 96, 128, 2) == 0  # K not a multiple of 64
+    p = ctypes.c_void_p()
+    assert lib.mlra_exchange_alloc(0, ctypes.byref(p), None) == b.MLRA_ERR_INVALID_ARG
+    assert lib.mlra_exchange_alloc(4096, None, None) == b.MLRA_ERR_INVALID_ARG
+    assert lib.mlra_exchange_open(None, ctypes.byref(p)) == b.MLRA_ERR_INVALID_ARG
+    assert lib.mlra_exchange_close(None) == b.MLRA_ERR_INVALID_ARG
+    assert lib.mlra_exchange_free(None) == b.MLRA_ERR_INVALID_ARG
+    assert lib.mlra_exchange_reset(None, 4096, None) == b.MLRA_ERR_INVALID_ARG
+    ok = 1 << 20
+
+    def allreduce(batch=16, heads=16, branches=1, d_c=128, d_h=128, out=ok, w=ok, gate=None, y=ok,
+                  regions=ok, world=4, rank=0, k=1, status=None, limit=10**9):
+        return lib.mlra_up_proj_allreduce(batch, heads, branches, d_c, d_h, out, w, gate, y, regions, world,
+                                          rank, k, status, limit, None)
+    for kw in [dict(world=0), dict(world=9), dict(rank=4), dict(rank=-1), dict(rank=3, k=2), dict(k=0),
+               dict(out=ok + 8), dict(regions=None), dict(gate=ok + 1), dict(status=ok + 2), dict(limit=0),
+               dict(batch=0)]:
+        assert allreduce(**kw) == b.MLRA_ERR_INVALID_ARG, kw
+    assert allreduce(d_c=96) == b.MLRA_ERR_UNSUPPORTED      # K = 96
+    assert allreduce(d_h=96) == b.MLRA_ERR_UNSUPPORTED
+
+
+def test_copy_ranges_rejects_bad_arguments_on_the_host():
+    lib = b.library()
+    ok = 1 << 20
+    arr = lambda *v: (ctypes.c_void_p * len(v))(*v)
+    sizes = lambda *v: (ctypes.c_uint64 * len(v))(*v)
+    assert lib.mlra_copy_ranges(0, arr(ok), arr(ok + 4096), sizes(16), None) == b.MLRA_ERR_INVALID_ARG
+    assert lib.mlra_copy_ranges(9, arr(*[ok] * 9), arr(*[ok] * 9), sizes(*[16] * 9), None) == b.MLRA_ERR_INVALID_ARG
+    assert lib.mlra_copy_ranges(1, None, arr(ok), sizes(16), None) == b.MLRA_ERR_INVALID_ARG
+    assert lib.mlra_copy_ranges(1, arr(ok + 4), arr(ok + 4096), sizes(16), None) == b.MLRA_ERR_INVALID_ARG
+    assert lib.mlra_copy_ranges(1, arr(ok), arr(ok + 4104), sizes(16), None) == b.MLRA_ERR_INVALID_ARG

@@ -84,6 +84,9 @@ class _OracleBackend:
     def mlra_exchange_free(self, ptr):
         self.calls.append(("free", ptr))
 
+    def mlra_exchange_reset(self, ptr, nbytes, device=None):
+        self.calls.append(("reset", ptr, nbytes))
+
     def mlra_decode(self, q_lat, q_rope, latent_cache, rope_cache, block_table, seqlens, scale, out_scale):
         out, _, st = self.oracle.decode(q_lat, q_rope, latent_cache, rope_cache, block_table, seqlens,
                                         scale, out_scale)
@@ -149,9 +152,9 @@ def test_branch_shards_add_up_to_the_unsharded_step(oracle_lib, world):
 
 
 def _mutant_worker(rank, world, port, results):
-    """Planted mistake: each rank keeps ALL branches' W_UV but only its own
-    latents -- the up-projection then pairs branch b's output with the wrong
-    matrix, and the sum must miss the unsharded step."""
+    """Planted mistake: every rank takes rank 0's W_UV slice with its own
+    latents -- the up-projection then pairs a branch's output with another
+    branch's matrix, and the sum must miss the unsharded step."""
     sys.path.insert(0, ROOT)
     from branch_latent_kv_b200.inputs import WORKLOADS, make_inputs
     from oracle import oracle
@@ -181,3 +184,28 @@ def test_a_misassigned_w_uv_shard_is_caught(oracle_lib):
         mp.spawn(_mutant_worker, args=(2, _free_port(), results), nprocs=2, join=True)
         got = dict(results)
     assert min(got.values()) > 1e-2
+
+
+def _reset_worker(rank, world, port, results):
+    sys.path.insert(0, ROOT)
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        be = _OracleBackend(rank, 64)
+        ex = tp.ExchangeGroup(4, 8, 2, 64, 64, device=torch.device("cpu"), backend=be)
+        ex.reset()   # after a timeout: each rank zeroes only its own region, then the group meets
+        ex.close()
+        ex.close()   # a second close does nothing
+        results[rank] = be.calls
+    finally:
+        dist.destroy_process_group()
+
+
+def test_reset_zeroes_only_the_own_region_and_close_is_idempotent():
+    with mp.Manager() as manager:
+        results = manager.dict()
+        mp.spawn(_reset_worker, args=(2, _free_port(), results), nprocs=2, join=True)
+        got = dict(results)
+    for rank, calls in got.items():
+        assert [c for c in calls if c[0] == "reset"] == [("reset", 1000 + rank, 4096)]
+        assert [c for c in calls if c[0] == "free"] == [("free", 1000 + rank)]
+        assert [c for c in calls if c[0] == "close"] == [("close", 1000 + (1 - rank))]
