@@ -97,7 +97,12 @@ class ExchangeGroup:
         self.regions = torch.tensor(ptrs, dtype=torch.int64, device=self.device)
 
     def reset(self) -> None:
-        """Zero this rank's region and meet the group (after a timeout)."""
+        """Collective, after a timeout: once every rank's kernels have ended
+        (no peer can still write into a region), each rank zeroes its own
+        region, and the group meets again before the next call."""
+        if self.device.type == "cuda":
+            torch.cuda.synchronize(self.device)
+        dist.barrier(group=self.group)
         self.backend.mlra_exchange_reset(self.own, self.nbytes, device=self.device)
         if self.device.type == "cuda":
             torch.cuda.synchronize(self.device)

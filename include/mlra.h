@@ -289,8 +289,10 @@ MLRA_API mlra_status mlra_exchange_close(void* region);
 MLRA_API mlra_status mlra_exchange_free(void* region);
 
 /* Zeroes a region (asynchronously on `stream`).  After a timeout the ranks'
- * call counters disagree: every rank zeroes its region, the group meets at a
- * barrier, and the next call starts afresh. */
+ * call counters disagree.  To start afresh: every rank synchronises its
+ * device, the group meets at a barrier (no kernel can still write into a
+ * region), every rank zeroes its own region and synchronises, and the group
+ * meets again before the next call. */
 MLRA_API mlra_status mlra_exchange_reset(void* region, size_t bytes, void* stream);
 
 /*
