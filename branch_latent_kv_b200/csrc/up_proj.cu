@@ -32,15 +32,18 @@
 // can live on different GPUs, so under 4-way tensor parallelism each GPU loads
 // only its own branch's latents plus the shared RoPE key, 1.5 d_h per token
 // against 4.5 d_h for MLA).  Rank r then holds out_lat and W_UV of its
-// branches only, and the branch sum crosses the ranks.  In that mode the cluster's column slice is
-// not written as y: each CTA stores its fp32 slice into slot r of every
-// rank's exchange region (plain stores, to peer memory over NVLink), then
-// raises its flag there (release at system scope).  Each rank waits, with a
-// bound, for the flags of all ranks on its own region, adds the slots in rank
-// order (the same order on every rank, so every rank's y is bit-identical)
-// and applies the gate.  The call number of each tile, kept per tile in the
-// region, selects one of two buffers, so a rank that runs ahead into the next
-// call never overwrites data that a slower rank is still adding up.
+// branches only, and the branch sum crosses the ranks.  In that mode a CTA's
+// column slice is not written as y: each CTA stores every fp32 value of its
+// slice, paired with the call's tag (call + 1) in one 64-bit word, into slot
+// r of every rank's exchange region (plain stores, to peer memory over
+// NVLink).  Each rank then reads its own region's slots for the tile, polls
+// (with a bound) any word whose tag is not this call's, adds the slots in
+// rank order (the same order on every rank, so every rank's y is
+// bit-identical) and applies the gate.  The word is single-copy atomic, so a
+// reader that sees the tag sees the value: no flags, no fences.  The call
+// number of each tile, kept per tile in the region, selects one of two
+// buffers, so a rank that runs ahead into the next call never overwrites a
+// word that a slower rank has not yet read.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
