@@ -139,6 +139,17 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def replay_steps(steps, copies, chain_replay, step_replays):
+    """Replay exactly `steps` steps: whole graphs of `copies` steps (one per
+    KV copy), then the remainder as one-step graphs.  Returns the count."""
+    n_chain, n_rest = divmod(steps, copies)
+    for _ in range(n_chain):
+        chain_replay()
+    for k in range(n_rest):
+        step_replays[k]()
+    return n_chain * copies + n_rest
+
+
 def max_over_ranks(values, dist, device):
     """Element-wise max of a list of floats over all ranks (a no-op without a
     process group)."""
@@ -389,13 +400,9 @@ def main():
     if pg:
         pg.barrier()
     torch.cuda.synchronize(dev)
-    n_chain, n_rest = divmod(args.steps, copies)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
-    for _ in range(n_chain):
-        chain_steps.replay()
-    for k in range(n_rest):
-        step_graphs[k].replay()
+    replay_steps(args.steps, copies, chain_steps.replay, [g.replay for g in step_graphs])
     end.record(stream)
     torch.cuda.synchronize(dev)
     if pg:

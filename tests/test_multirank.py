@@ -66,3 +66,16 @@ def test_reference_arm_under_torchrun_prints_one_line_from_rank_zero(oracle_lib)
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["cpu_baseline"]["kind"] == "oracle" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+@pytest.mark.parametrize("steps,copies", [(200, 4), (201, 4), (3, 4), (1, 2), (7, 3), (0, 4)])
+def test_timed_region_replays_exactly_k_steps(steps, copies):
+    """The step region replays graphs of `copies` steps and then one-step
+    graphs: exactly K steps, each KV copy in turn."""
+    sys.path.insert(0, ROOT)
+    import bench
+    seen = []
+    n = bench.replay_steps(steps, copies, lambda: seen.extend(range(copies)),
+                           [lambda c=c: seen.append(c) for c in range(copies)])
+    assert n == steps == len(seen)
+    assert seen == [k % copies for k in range(steps)]
