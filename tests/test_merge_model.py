@@ -111,6 +111,17 @@ def _launches(rng, ctas):
 
 
 @pytest.mark.parametrize("ctas", [3, 7, 16, 148])
+def test_no_cta_has_more_than_two_split_sequences(ctas):
+    """The kernel keeps two pending arrivals per CTA (its range's first and
+    last sequence); a third would lose an arrival and stall that merge."""
+    rng = random.Random(100 + ctas)
+    for _ in range(200):
+        for seqlens in _launches(rng, ctas):
+            _, arrivals, _, _ = structure(seqlens, ctas)
+            assert max(len(v) for v in arrivals.values()) <= 2, seqlens
+
+
+@pytest.mark.parametrize("ctas", [3, 7, 16, 148])
 def test_merge_counters_are_exact_and_reset_between_launches(ctas):
     rng = random.Random(ctas)
     for seed in range(60):
