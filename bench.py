@@ -24,7 +24,10 @@ Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
        [--impl ours|reference]
 Under torchrun every rank runs the same workload on its own GPU (replicas,
 weak scaling); rank 0 prints one JSON line.  --impl reference times the fp64
-CPU oracle on a bounded sample of the same workload on the host cores.
+CPU oracle on the same workload on the host cores (the whole step unless
+W + K steps would exceed --ref-budget-s, then the first sequences).
+workloads (one GPU): the decode kernel alone on the other decode workloads,
+timed like the roofline region.
 """
 from __future__ import annotations
 
@@ -49,6 +52,10 @@ from branch_latent_kv_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
 from branch_latent_kv_b200.step import DecodeStep  # noqa: E402
 
 METRIC = "MLRA decode-attention KV GB/s and tokens/s at 1 B200; % of HBM roofline"
+# The other decode workloads whose decode-kernel figures ride along in the
+# line (the step itself is timed on --workload).
+OTHER_WORKLOADS = ["long_context", "ragged", "mla_equal_bytes", "mlra4_equal_bytes", "tp_shard",
+                   "mlra2_equal_bytes", "context_2m"]
 FALLBACK_HBM_GBS = 6650.0
 
 # DRAM traffic of the decode split kernel per launch on decode_2p9b, from one
@@ -171,8 +178,10 @@ def kv_bytes_of(x) -> int:
     return x.kv_bytes
 
 
-def reference_sample(w, n_seqs):
-    """The first n_seqs sequences of the workload (full lengths, same shapes)."""
+def reference_inputs(w, n_seqs=None):
+    """The workload's inputs on the host (all sequences, or the first n_seqs)."""
+    if n_seqs is None or n_seqs >= w.batch:
+        return make_inputs(w, with_w_uv=True)
     gen = torch.Generator(device="cpu").manual_seed(w.seed)
     from branch_latent_kv_b200.inputs import draw_seqlens
     seqlens = draw_seqlens(w, gen)[:n_seqs]
@@ -180,37 +189,64 @@ def reference_sample(w, n_seqs):
     return make_inputs(ws, seqlens=seqlens, with_w_uv=True)
 
 
+def l2_copies(kv_bytes):
+    """KV copies the GPU arm rotates over so that L2 cannot serve the cache."""
+    l2 = 126 * 1024 * 1024
+    if torch.cuda.is_available():
+        l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    return max(2, math.ceil(4 * l2 / kv_bytes))
+
+
 def run_reference(args, world, rank):
-    """fp64 oracle on the host cores; each step is a bounded sample of the
-    workload: its first --ref-sample-seqs sequences, decode + up-projection."""
+    """The fp64 oracle on the host cores, each step the whole workload
+    (decode + up-projection of every sequence), unless W + K such steps
+    would take longer than --ref-budget-s: then each step is the first
+    sequences of the workload, as many as fit."""
     if rank != 0:
         return
     from oracle import oracle
     w = WORKLOADS[args.workload]
     threads = len(os.sched_getaffinity(0))
     oracle.set_num_threads(threads)
-    x = reference_sample(w, args.ref_sample_seqs)
-    kv = x.kv_bytes
+    x = reference_inputs(w)
 
-    def step():
-        out, _, _ = oracle.decode(x.q_lat, x.q_rope, x.latent_cache, x.rope_cache, x.block_table,
-                                  x.seqlens, x.scale, x.out_scale)
-        oracle.up_proj(out, x.w_uv, w.d_h)
+    def make_step(xx):
+        def step():
+            out, _, _ = oracle.decode(xx.q_lat, xx.q_rope, xx.latent_cache, xx.rope_cache, xx.block_table,
+                                      xx.seqlens, xx.scale, xx.out_scale)
+            oracle.up_proj(out, xx.w_uv, w.d_h)
+        return step
 
-    for _ in range(args.warmup):
+    step = make_step(x)
+    t0 = time.perf_counter()
+    step()
+    one = time.perf_counter() - t0
+    n_steps = args.steps + max(args.warmup - 1, 0)
+    if one * n_steps > args.ref_budget_s:
+        keep = max(1, int(w.batch * args.ref_budget_s / (one * n_steps)))
+        x = reference_inputs(w, keep)
+        step = make_step(x)
+    for _ in range(max(args.warmup - 1, 0)):
         step()
     t0 = time.perf_counter()
     for _ in range(args.steps):
         step()
     dt = time.perf_counter() - t0
+    kv = x.kv_bytes
     gbs = kv * args.steps / dt / 1e9
-    sample = (f"first {x.workload.batch} of {w.batch} sequences of {w.name} "
-              f"({int(x.seqlens.sum())} tokens), decode + up-projection per step")
+    n = x.workload.batch
+    sample = (f"the whole {w.name} step (all {w.batch} sequences, {int(x.seqlens.sum())} tokens), "
+              f"decode + up-projection" if n == w.batch else
+              f"first {n} of {w.batch} sequences of {w.name} ({int(x.seqlens.sum())} tokens), "
+              f"decode + up-projection per step")
+    gen = torch.Generator(device="cpu").manual_seed(w.seed)
+    from branch_latent_kv_b200.inputs import draw_seqlens
+    full_kv = int(draw_seqlens(w, gen).to(torch.int64).sum()) * (w.branches * w.d_c + w.d_r) * 2
     line = {"impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": workload_config(w, None),
-            "tokens_per_s": x.workload.batch * args.steps / dt,
+            "data": "synthetic", "config": workload_config(w, l2_copies(full_kv)),
+            "tokens_per_s": n * args.steps / dt,
             "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -259,6 +295,56 @@ def prestep_time_us(x, w, dev, stream, steps):
     return e0.elapsed_time(e1) / (reps * per_graph) * 1e3
 
 
+def decode_only_figure(name, dev, stream, hbm_peak, min_launches=24):
+    """The decode kernel alone on another workload, timed like the roofline
+    region: a graph of one decode launch per KV copy (copies * KV bytes >= 4x
+    L2), replayed until at least min_launches launches, CUDA events around the
+    region."""
+    w = WORKLOADS[name]
+    x = make_inputs(w, device=str(dev), with_w_uv=False)
+    kv = x.kv_bytes
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    copies = max(2, math.ceil(4 * l2 / kv))
+    lat = [x.latent_cache] + [x.latent_cache.clone() for _ in range(copies - 1)]
+    rope = [x.rope_cache] + [x.rope_cache.clone() for _ in range(copies - 1)]
+    dims = b.decode_dims(x.q_lat, x.q_rope, x.latent_cache, x.block_table)
+    ws = torch.zeros(b.mlra_decode_workspace_bytes(dims), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(x.q_lat)
+
+    def call(i, st):
+        b.mlra_decode(x.q_lat, x.q_rope, lat[i], rope[i], x.block_table, x.seqlens, x.scale, x.out_scale,
+                      out=out, workspace=ws, stream=st)
+    call(0, stream)
+    torch.cuda.synchronize(dev)
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        for c in range(copies):
+            call(c, cap)
+    torch.cuda.synchronize(dev)
+    for _ in range(3):
+        g.replay()
+    reps = -(-min_launches // copies)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t1 = time.time()
+    us = e0.elapsed_time(e1) / (reps * copies) * 1e3
+    err = b.mlra_read_device_error(ws)
+    if err != 0:
+        raise RuntimeError(f"device error on {name}: {b.mlra_status_string(err)}")
+    del g
+    gbs = kv / (us * 1e-6) / 1e9
+    return {"tokens": int(x.seqlens.to(torch.int64).sum()), "kv_bytes_per_launch": kv,
+            "us_per_launch": us, "decode_gbs": gbs, "frac": gbs / hbm_peak,
+            "launches": reps * copies, "kv_copies": copies}, (t0, t1)
+
+
 def workload_config(w, copies):
     cfg = {"workload": w.name, "batch": w.batch, "heads": w.heads, "branches": w.branches,
            "d_c": w.d_c, "d_r": w.d_r, "page_size": w.page_size, "d_h": w.d_h,
@@ -300,7 +386,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="decode_2p9b", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--ref-sample-seqs", type=int, default=2)
+    ap.add_argument("--ref-budget-s", type=float, default=150.0,
+                    help="reference arm: longest oracle run before it falls back to a sample")
+    ap.add_argument("--workloads", default=",".join(OTHER_WORKLOADS),
+                    help="decode-kernel figures of these workloads in the line ('' for none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
                     help="run W + K device-resident steps only and print nothing (for profilers)")
@@ -458,19 +547,31 @@ def main():
     e_end.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms, = max_over_ranks([e_start.elapsed_time(e_end)], pg, dev)
-    sampler.stop()
 
     # the decode pre-step (query absorption, rotary embedding, append) on the
     # same batch, its own timed loop: events around each launch
     pre_us = prestep_time_us(x, w, dev, stream, args.steps)
+
+    peaks, peak_kind = measured_peaks()
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    # the decode kernel alone on the other workloads (one GPU runs only)
+    others = {}
+    names = [n for n in args.workloads.split(",") if n and n != args.workload] if world == 1 else []
+    if names:
+        del steps_e2e, lat, rope
+        torch.cuda.empty_cache()
+    for name in names:
+        fig, (t0, t1) = decode_only_figure(name, dev, stream, hbm_peak)
+        fig["sm_mhz"] = sampler.summary(t0, t1)["sm_mhz"]
+        others[name] = fig
+        torch.cuda.empty_cache()
+    sampler.stop()
 
     err = b.mlra_read_device_error(ws)
     if err != 0:
         raise RuntimeError(f"device error during the benchmark: {b.mlra_status_string(err)}")
 
     clocks = sampler.summary(t_warm, t_load1)
-    peaks, peak_kind = measured_peaks()
-    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     gbs = kv * world * args.steps / (elapsed_ms / 1e3) / 1e9
     achieved = kv / (decode_ms / 1e3) / 1e9
     traffic = None
@@ -500,6 +601,12 @@ def main():
                             "(back-to-back launches in a graph)"},
         "clocks": clocks,
     }
+    if others:
+        line["workloads"] = {
+            "what": "decode kernel alone (mlra_decode) on the other decode workloads: graphs of one "
+                    "launch per KV copy (copies x KV bytes >= 4x L2) replayed back to back, CUDA events "
+                    "around >= 24 launches; frac = decode_gbs / the same measured peak",
+            **others}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, x)
     if rank == 0:

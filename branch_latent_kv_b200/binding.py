@@ -261,8 +261,23 @@ def _up_proj(out_lat, w_uv, gate, d_h, y, stream) -> torch.Tensor:
     return y
 
 
-def mlra_read_device_error(workspace: torch.Tensor, stream=None) -> int:
-    """Synchronise the stream; return and clear the device error code."""
+def default_workspace(device: Optional[torch.device] = None) -> Optional[torch.Tensor]:
+    """The cached workspace that decode calls without an explicit workspace
+    use on `device` (None if none has been made yet)."""
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    return _ws_cache.get(key)
+
+
+def mlra_read_device_error(workspace: Optional[torch.Tensor] = None, stream=None) -> int:
+    """Synchronise the stream; return and clear the device error code of
+    `workspace` (default: the cached workspace of the current device).  A
+    reported MLRA_ERR_DEVICE_TIMEOUT also clears the workspace's split
+    counters, so the workspace serves the next call."""
+    if workspace is None:
+        workspace = default_workspace()
+        if workspace is None:
+            return MLRA_OK
     return int(library().mlra_read_device_error(_ptr(workspace),
                                                 _stream_ptr(stream, workspace.device)))
 

@@ -63,11 +63,12 @@ mlra_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MLRA_OK : MLR
 
 enum class Impl { kTensorCore, kSimt };
 
-mlra_status decode_impl(Impl impl, const mlra_dims* dims, const void* q_lat, const void* q_rope,
+// Host validation of a decode call and the kernel arguments it implies.
+mlra_status decode_args(Impl impl, const mlra_dims* dims, const void* q_lat, const void* q_rope,
                         const void* latent_cache, const void* rope_cache,
                         const int32_t* block_table, const int32_t* seqlens, float scale,
                         float out_scale, void* out, void* workspace, size_t workspace_bytes,
-                        void* stream) {
+                        DecodeArgs* a_out) {
     mlra_status s = check_dims(dims);
     if (s != MLRA_OK) return s;
     s = impl == Impl::kTensorCore ? check_tc_coverage(dims) : check_simt_coverage(dims);
@@ -85,7 +86,7 @@ mlra_status decode_impl(Impl impl, const mlra_dims* dims, const void* q_lat, con
         workspace_layout(dims->batch, dims->heads, dims->branches, dims->d_c, ctas);
     if (workspace_bytes < wl.total) return MLRA_ERR_WORKSPACE;
 
-    DecodeArgs a;
+    DecodeArgs& a = *a_out;
     a.q_lat = static_cast<const __nv_bfloat16*>(q_lat);
     a.q_rope = static_cast<const __nv_bfloat16*>(q_rope);
     a.latent = static_cast<const __nv_bfloat16*>(latent_cache);
@@ -109,7 +110,18 @@ mlra_status decode_impl(Impl impl, const mlra_dims* dims, const void* q_lat, con
     a.num_ctas = ctas;
     a.scale_log2 = scale * kLog2e;
     a.out_scale = out_scale;
+    return MLRA_OK;
+}
 
+mlra_status decode_impl(Impl impl, const mlra_dims* dims, const void* q_lat, const void* q_rope,
+                        const void* latent_cache, const void* rope_cache,
+                        const int32_t* block_table, const int32_t* seqlens, float scale,
+                        float out_scale, void* out, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+    DecodeArgs a;
+    const mlra_status s = decode_args(impl, dims, q_lat, q_rope, latent_cache, rope_cache, block_table,
+                                      seqlens, scale, out_scale, out, workspace, workspace_bytes, &a);
+    if (s != MLRA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (impl == Impl::kTensorCore) return cuda_status(launch_decode_tc(a, st));  // merges in-kernel
     mlra_status r = cuda_status(launch_decode_simt(a, st));
@@ -118,6 +130,16 @@ mlra_status decode_impl(Impl impl, const mlra_dims* dims, const void* q_lat, con
 }
 
 }  // namespace
+
+namespace mlra {
+mlra_status decode_tc_args(const mlra_dims* dims, const void* q_lat, const void* q_rope,
+                           const void* latent_cache, const void* rope_cache, const int32_t* block_table,
+                           const int32_t* seqlens, float scale, float out_scale, void* out, void* workspace,
+                           size_t workspace_bytes, DecodeArgs* a) {
+    return decode_args(Impl::kTensorCore, dims, q_lat, q_rope, latent_cache, rope_cache, block_table, seqlens,
+                       scale, out_scale, out, workspace, workspace_bytes, a);
+}
+}  // namespace mlra
 
 extern "C" {
 
@@ -370,7 +392,13 @@ mlra_status mlra_read_device_error(void* workspace, void* stream) {
     int code = 0;
     if (cudaMemcpy(&code, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
         return MLRA_ERR_CUDA;
-    if (code != 0 && cudaMemset(workspace, 0, sizeof(int)) != cudaSuccess) return MLRA_ERR_CUDA;
+    // A kernel that gave up on a bounded wait may leave split counters set;
+    // they sit at a fixed place for every dims (after the error word), so
+    // reporting the timeout also clears them and the workspace is usable again.
+    const size_t clear = code == MLRA_ERR_DEVICE_TIMEOUT
+                             ? workspace_layout(1, 1, 1, 1, 1).lse_off
+                             : (code != 0 ? sizeof(int) : 0);
+    if (clear != 0 && cudaMemset(workspace, 0, clear) != cudaSuccess) return MLRA_ERR_CUDA;
     return static_cast<mlra_status>(code);
 }
 

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "mlra.h"
+
 namespace mlra {
 
 // Arguments of the decode kernels (everything already validated on the host).
@@ -26,6 +28,13 @@ struct DecodeArgs {
     float scale_log2;             // scale * log2(e)
     float out_scale;
 };
+
+// Host validation of a tensor-core decode call (what mlra_decode checks);
+// fills the kernel arguments.  Defined in api.cu.
+mlra_status decode_tc_args(const mlra_dims* dims, const void* q_lat, const void* q_rope,
+                           const void* latent_cache, const void* rope_cache, const int32_t* block_table,
+                           const int32_t* seqlens, float scale, float out_scale, void* out, void* workspace,
+                           size_t workspace_bytes, DecodeArgs* a);
 
 // Split-KV decode on CUDA cores (fp32 FMA).  Writes final outputs of
 // single-split sequences and partials of the others.

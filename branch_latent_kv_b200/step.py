@@ -12,9 +12,11 @@ this module only arranges launches.
 
 Buffers are bound at construction: write the next step's inputs into the
 bound tensors (or into the pinned host tensors given as ``host_inputs``)
-before calling the step.  The graph keeps the kernels' arguments, including
-the TMA descriptors built from the bound pointers, so the bound tensors must
-stay alive and in place.
+before calling the step.  A replay is asynchronous and its copy kernel reads
+the pinned host inputs while it runs, so overwrite them only after the
+previous step has finished (synchronise its stream first).  The graph keeps
+the kernels' arguments, including the TMA descriptors built from the bound
+pointers, so the bound tensors must stay alive and in place.
 """
 from __future__ import annotations
 
@@ -82,10 +84,19 @@ class DecodeStep:
         self._args = (q_lat, q_rope, latent_cache, rope_cache, block_table, seqlens, scale, out_scale)
         self._w_uv, self._d_h = w_uv, d_h
 
-        # validation: one eager pass (raises on any argument error)
+        # validation: one eager pass (raises on any argument error) on the
+        # step's real inputs: the host inputs, if any, are brought in first,
+        # so the pass never reads uninitialised bound tensors
         stream = torch.cuda.current_stream(dev)
+        with torch.cuda.stream(stream):
+            for name, h in self.host_inputs.items():
+                self.inputs[name].copy_(h, non_blocking=True)
         self._body(stream, copies=False)
         torch.cuda.synchronize(dev)
+        # the validation pass's device findings are not a step's: reading
+        # clears the error word (and the split counters after a timeout), so
+        # the first replay reports only its own
+        b.mlra_read_device_error(self.workspace, stream)
         # capture on a side stream, ordered after the eager pass
         cap = torch.cuda.Stream(dev)
         cap.wait_stream(stream)

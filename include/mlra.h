@@ -84,8 +84,11 @@ typedef struct {
  * dims), the split-KV partial outputs (fp32) and their log-sum-exps.
  * Zero it once before first use (the error word and the counters must start
  * at 0).  Every call that ends without MLRA_ERR_DEVICE_TIMEOUT leaves the
- * counters at 0 again, so it never needs re-zeroing; after a timeout, zero it
- * before the next call.
+ * counters at 0 again, so it never needs re-zeroing.  A call whose kernel
+ * gave up on a bounded wait may leave counters set: mlra_read_device_error
+ * clears them when it reports the timeout; a caller that does not read the
+ * error must zero the first 256 KB + 256 bytes of the workspace before
+ * reusing it.
  */
 MLRA_API size_t mlra_decode_workspace_bytes(const mlra_dims* dims, int32_t num_ctas);
 
@@ -162,11 +165,12 @@ MLRA_API mlra_status mlra_decode_simt(const mlra_dims* dims, const void* q_lat, 
  * It allocates and frees nothing.  All calls on a device share the array:
  * calls that may overlap on the GPU race and corrupt each other's results,
  * so order them on one stream.  The array keeps the last call's contents;
- * the parts that must start at zero (the error word and the split counters)
- * start zeroed; the error word is cleared again at the end of every call and
- * the counters return to zero unless the call reports a device timeout.  The first call on each device
- * looks up the array's address with that device current; make it before any
- * stream capture starts.
+ * every call first clears, stream-ordered, the parts that must start at zero
+ * (the error word and its split counters), so no call inherits state from an
+ * earlier one, not even from one whose kernel gave up on a bounded wait.
+ * The first call in each CUDA context (on each device, and again after a
+ * cudaDeviceReset) looks up the array's address with that context current;
+ * make it before any stream capture starts.
  */
 MLRA_API mlra_status mlra_decode_static_scratch(const mlra_dims* dims, const void* q_lat,
                              const void* q_rope, const void* latent_cache,
@@ -343,7 +347,10 @@ MLRA_API mlra_status mlra_copy_ranges(int32_t count, const void* const* src, voi
 /*
  * Synchronises `stream`, returns the first device-side error code recorded
  * in `workspace` since the last read (MLRA_OK if none) and resets it to 0.
- * Returns MLRA_ERR_CUDA if the synchronisation or copy fails.
+ * When the code is MLRA_ERR_DEVICE_TIMEOUT it also clears the workspace's
+ * split counters (a kernel that gave up may have left them set), so the
+ * workspace serves the next call.  Returns MLRA_ERR_CUDA if the
+ * synchronisation or copy fails.
  */
 MLRA_API mlra_status mlra_read_device_error(void* workspace, void* stream);
 

@@ -49,12 +49,20 @@ def structure(seqlens, ctas):
     return multi, arrivals, merges, groups
 
 
-def run(seqlens_per_launch, ctas, seed, reset_at=0, wait_for=0):
+def run(seqlens_per_launch, ctas, seed, reset_at=0, wait_for=0, abort_launch=None,
+        clear_after_abort=True):
     """reset_at / wait_for: offsets planted into the reset threshold and the
-    wait target (0 = the protocol)."""
+    wait target (0 = the protocol).  abort_launch: index of a launch in which
+    some CTAs give up (a bounded wait that expired): each stops at a random
+    point of its program, and every wait that can then never be satisfied
+    expires too.  That launch's results are reported as a timeout and not
+    checked; with clear_after_abort the host then clears the counters (what
+    mlra_read_device_error does when it reports the timeout, and what the
+    static-scratch entry does before every call)."""
     rng = random.Random(seed)
     cnt = {}
-    for seqlens in seqlens_per_launch:
+    for li, seqlens in enumerate(seqlens_per_launch):
+        aborting = li == abort_launch
         multi, arrivals, merges, groups = structure(seqlens, ctas)
         arrived = {n: 0 for n in multi}
         merged = {n: [] for n in multi}
@@ -63,6 +71,9 @@ def run(seqlens_per_launch, ctas, seed, reset_at=0, wait_for=0):
         for c in range(ctas):
             if merges[c] is not None:
                 todo[c] += [("wait", merges[c]), ("depart", merges[c])]
+        if aborting:
+            for c in rng.sample(range(ctas), max(1, ctas // 4)):
+                todo[c] = todo[c][:rng.randrange(len(todo[c]) + 1)]
         while any(todo.values()):
             live = []
             for c, acts in todo.items():
@@ -73,6 +84,8 @@ def run(seqlens_per_launch, ctas, seed, reset_at=0, wait_for=0):
                     continue
                 live.append(c)
             if not live:
+                if aborting:
+                    break  # the remaining waits expire: those CTAs stop
                 return "deadlock"
             c = rng.choice(live)
             kind, n = todo[c].pop(0)
@@ -89,6 +102,10 @@ def run(seqlens_per_launch, ctas, seed, reset_at=0, wait_for=0):
                 cnt[n] = old + 1
                 if old == S + G - 1 + reset_at:
                     cnt[n] = 0
+        if aborting:
+            if clear_after_abort:
+                cnt = {}
+            continue
         for n in multi:
             if sorted(merged[n]) != list(range(len(groups[n]))):
                 return "rows not merged once"
@@ -126,6 +143,21 @@ def test_merge_counters_are_exact_and_reset_between_launches(ctas):
     rng = random.Random(ctas)
     for seed in range(60):
         assert run(_launches(rng, ctas), ctas, seed) == "ok", seed
+
+
+@pytest.mark.parametrize("ctas", [7, 16, 148])
+def test_a_launch_after_an_aborted_one_is_exact_once_counters_are_cleared(ctas):
+    """An aborted launch (some CTAs give up mid-protocol) followed by clean
+    ones: with the host-side clear that reporting the timeout performs, the
+    next launches merge exactly and leave every counter at zero; without it,
+    the stale counts let a later merge start early or stay set."""
+    rng = random.Random(500 + ctas)
+    uncleared = set()
+    for seed in range(60):
+        shapes = [[8192] * 16] + _launches(rng, ctas)
+        assert run(shapes, ctas, seed, abort_launch=0) == "ok", seed
+        uncleared.add(run(shapes, ctas, seed, abort_launch=0, clear_after_abort=False))
+    assert uncleared - {"ok"}, uncleared
 
 
 def test_planted_protocol_mistakes_are_caught():

@@ -57,7 +57,7 @@ def test_reference_arm_under_torchrun_prints_one_line_from_rank_zero(oracle_lib)
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
            "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
            "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0",
-           "--workload", "tiny", "--ref-sample-seqs", "1"]
+           "--workload", "tiny"]
     r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
@@ -66,6 +66,19 @@ def test_reference_arm_under_torchrun_prints_one_line_from_rank_zero(oracle_lib)
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["cpu_baseline"]["kind"] == "oracle" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["sample"].startswith("the whole tiny step")
+
+
+def test_reference_arm_falls_back_to_a_sample_beyond_its_budget(oracle_lib):
+    """With a budget too small for the whole step, each step is the first
+    sequences of the workload, and the line says so."""
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "2",
+           "--warmup", "3", "--workload", "ragged", "--ref-budget-s", "0.01"]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads([ln for ln in r.stdout.splitlines() if ln.startswith("{")][0])
+    assert line["cpu_baseline"]["sample"].startswith("first 1 of 64 sequences of ragged")
+    assert line["config"]["workload"] == "ragged"
 
 
 @pytest.mark.parametrize("steps,copies", [(200, 4), (201, 4), (3, 4), (1, 2), (7, 3), (0, 4)])

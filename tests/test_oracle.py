@@ -66,6 +66,27 @@ def test_matches_textbook_mqa(oracle_lib, B, d_c, d_r, P):
     assert np.isfinite(out).all()
 
 
+def test_mla_shape_matches_textbook_mqa(oracle_lib):
+    """The MLA special case at the equal-bytes comparison's own shape: one
+    branch of d_c = 512 plus the 64-wide RoPE key, page size 64, 16 heads,
+    scale 1/sqrt(576), out_scale 1.  With B = 1 the method is MLA's absorbed
+    decode, i.e. multi-query attention over keys [c ; k_r] and values c."""
+    rng = np.random.default_rng(512)
+    N, H, B, d_c, d_r, P = 2, 16, 1, 512, 64, 64
+    lengths = [300, 129]
+    lat, rope = _logical(rng, lengths, B, d_c, d_r)
+    q_lat, q_rope = _queries(rng, N, H, B, d_c, d_r, gain=500.0)
+    pool, rpool, table, seqlens = paged_from_logical(lat, rope, P, rng, slack_pages=2)
+    scale, out_scale = 1 / math.sqrt(d_c + d_r), 1.0
+    # the scores are far from flat (std about 3), so the weights matter
+    s0 = scale * (lat[0][:, 0, :] @ q_lat[0, 0, 0] + rope[0] @ q_rope[0, 0])
+    assert s0.std() > 2.0
+    out, lse, status = oracle_lib.decode(q_lat, q_rope, pool, rpool, table, seqlens, scale, out_scale)
+    assert status == 0
+    ref = _sdpa_reference(q_lat, q_rope, lat, rope, scale, out_scale)
+    np.testing.assert_allclose(out, ref, rtol=1e-11, atol=1e-14)
+
+
 def test_bruteforce_tiny(oracle_lib):
     """Enumerate every token with math.fsum and the max-free form
     p_t = 1 / sum_u exp(s_u - s_t)."""

@@ -4,10 +4,10 @@ memory pools, runtimes whose device memory is all owned by their own
 allocator, serving loops that forbid allocation after start-up).
 
 It is called here through the C ABI directly and must match mlra_decode
-(which uses a caller-provided workspace) within the parity tolerance on two
-calls in a row with different inputs, since every call reuses the same
-static scratch array.  This file runs last so that a failure here never
-hides the other GPU tests, and it needs nothing from them.
+(which uses a caller-provided workspace), and the fp64 oracle, within the
+parity tolerance on two calls in a row with different inputs, since every
+call reuses the same static scratch array.  This file runs last so that a
+failure here never hides the other GPU tests, and it needs nothing from them.
 """
 import ctypes
 
@@ -52,7 +52,7 @@ def _close(a, ref):
     return float(np.abs(d).max()), float(np.linalg.norm(d) / np.linalg.norm(r))
 
 
-def test_two_calls_in_a_row_match_mlra_decode(lib):
+def test_two_calls_in_a_row_match_mlra_decode(lib, oracle_lib):
     cases = [
         make_inputs(WORKLOADS["decode_2p9b"].with_(batch=6, seqlen=None), seed=21, device="cuda",
                     seqlens=torch.tensor([5000, 1, 777, 128, 4097, 2500], dtype=torch.int32)),
@@ -69,6 +69,13 @@ def test_two_calls_in_a_row_match_mlra_decode(lib):
         assert int(status.item()) == 0
         max_abs, rel = _close(out, ref)
         assert max_abs <= MAX_ABS and rel <= REL_L2, (max_abs, rel)
+        want, _, st_o = oracle_lib.decode(x.q_lat.cpu(), x.q_rope.cpu(), x.latent_cache.cpu(),
+                                          x.rope_cache.cpu(), x.block_table.cpu(), x.seqlens.cpu(),
+                                          x.scale, x.out_scale)
+        assert st_o == 0
+        d = out.float().cpu().double().numpy() - want
+        max_abs, rel = float(np.abs(d).max()), float(np.linalg.norm(d) / np.linalg.norm(want))
+        assert max_abs <= MAX_ABS and rel <= REL_L2, ("against the oracle", max_abs, rel)
 
 
 def test_device_errors_are_reported_and_cleared(lib):
