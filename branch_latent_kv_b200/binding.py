@@ -63,6 +63,9 @@ def library() -> ctypes.CDLL:
             lib.mlra_decode.argtypes = [dp, vp, vp, vp, vp, vp, vp, ctypes.c_float, ctypes.c_float,
                                         vp, vp, sz, vp]
             lib.mlra_decode.restype = ctypes.c_int
+            lib.mlra_decode_up_proj.argtypes = [dp, vp, vp, vp, vp, vp, vp, ctypes.c_float, ctypes.c_float,
+                                                vp, vp, i32, vp, vp, sz, vp]
+            lib.mlra_decode_up_proj.restype = ctypes.c_int
             lib.mlra_decode_simt.argtypes = lib.mlra_decode.argtypes
             lib.mlra_decode_simt.restype = ctypes.c_int
             lib.mlra_up_proj.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp]
@@ -161,6 +164,12 @@ def workspace_for(dims: mlra_dims, device: torch.device) -> torch.Tensor:
 
 def _decode(entry, q_lat, q_rope, latent_cache, rope_cache, block_table, seqlens, scale, out_scale,
             out=None, workspace=None, stream=None) -> torch.Tensor:
+    return _decode_call(lambda dims, *args: getattr(library(), entry)(dims, *args), entry, q_lat, q_rope,
+                        latent_cache, rope_cache, block_table, seqlens, scale, out_scale, out, workspace, stream)
+
+
+def _decode_call(call, name, q_lat, q_rope, latent_cache, rope_cache, block_table, seqlens, scale, out_scale,
+                 out=None, workspace=None, stream=None) -> torch.Tensor:
     dev = q_lat.device
     if dev.type != "cuda":
         raise ValueError("mlra_decode runs on CUDA tensors only")
@@ -184,12 +193,10 @@ def _decode(entry, q_lat, q_rope, latent_cache, rope_cache, block_table, seqlens
             raise ValueError("out must have the shape of q_lat")
     if workspace is None:
         workspace = workspace_for(dims, dev)
-    st = getattr(library(), entry)(ctypes.byref(dims), _ptr(q_lat), _ptr(q_rope), _ptr(latent_cache),
-                               _ptr(rope_cache), _ptr(block_table), _ptr(seqlens), float(scale),
-                               float(out_scale), _ptr(out), _ptr(workspace),
-                               workspace.numel() * workspace.element_size(),
-                               _stream_ptr(stream, dev))
-    _check(st, entry)
+    st = call(ctypes.byref(dims), _ptr(q_lat), _ptr(q_rope), _ptr(latent_cache), _ptr(rope_cache),
+              _ptr(block_table), _ptr(seqlens), float(scale), float(out_scale), _ptr(out), _ptr(workspace),
+              workspace.numel() * workspace.element_size(), _stream_ptr(stream, dev))
+    _check(st, name)
     return out
 
 
@@ -203,6 +210,40 @@ def mlra_decode(q_lat, q_rope, latent_cache, rope_cache, block_table, seqlens, s
     """
     return _decode("mlra_decode", q_lat, q_rope, latent_cache, rope_cache, block_table, seqlens,
                    scale, out_scale, out, workspace, stream)
+
+
+def mlra_decode_up_proj(q_lat, q_rope, latent_cache, rope_cache, block_table, seqlens, scale, out_scale,
+                        w_uv, d_h: Optional[int] = None, out=None, y=None, workspace=None, stream=None):
+    """The whole step in one launch (see mlra_decode_up_proj in mlra.h):
+    returns (out bf16 [N,H,B,d_c], y bf16 [N, H*d_h]).  y may be a pinned
+    host tensor (the kernel then writes it over PCIe)."""
+    dev = q_lat.device
+    if dev.type != "cuda":
+        raise ValueError("mlra_decode_up_proj runs on CUDA tensors only")
+    _require(w_uv, "w_uv", torch.bfloat16, 3, dev)
+    N, H, B, d_c = q_lat.shape
+    if w_uv.shape[0] != B or w_uv.shape[1] != d_c or w_uv.shape[2] % H != 0:
+        raise ValueError("w_uv must be [branches, d_c, heads*d_h]")
+    if d_h is None:
+        d_h = w_uv.shape[2] // H
+    if w_uv.shape[2] != H * d_h:
+        raise ValueError("w_uv last dimension must be heads*d_h")
+    if y is None:
+        y = torch.empty((N, H * d_h), dtype=torch.bfloat16, device=dev)
+    else:
+        _require(y, "y", torch.bfloat16, 2, y.device if y.device.type == "cpu" else dev)
+        if y.device.type == "cpu" and not y.is_pinned():
+            raise ValueError("a host y must be pinned memory")
+        if tuple(y.shape) != (N, H * d_h):
+            raise ValueError("y must be [N, heads*d_h]")
+    def entry(dims, *args):
+        # mlra_decode's arguments up to out, then w_uv, d_h, y, workspace, bytes, stream
+        head, tail = args[:9], args[9:]
+        return library().mlra_decode_up_proj(dims, *head, _ptr(w_uv), int(d_h), _ptr(y), *tail)
+
+    out = _decode_call(entry, "mlra_decode_up_proj", q_lat, q_rope, latent_cache, rope_cache, block_table,
+                       seqlens, scale, out_scale, out, workspace, stream)
+    return out, y
 
 
 def mlra_decode_simt(q_lat, q_rope, latent_cache, rope_cache, block_table, seqlens, scale,

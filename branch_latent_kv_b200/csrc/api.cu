@@ -61,6 +61,26 @@ int device_sm_count() {
 
 mlra_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MLRA_OK : MLRA_ERR_CUDA; }
 
+// The address through which the device reaches `p` (device, managed or
+// mapped pinned host memory), or null for memory the device cannot address.
+const void* device_address(const void* p) {
+    if (p == nullptr) return nullptr;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();  // clear the error state the failed query leaves
+        return nullptr;
+    }
+    switch (at.type) {
+        case cudaMemoryTypeDevice:
+        case cudaMemoryTypeManaged:
+        case cudaMemoryTypeHost:
+            return at.devicePointer;
+        default:
+            return nullptr;
+    }
+}
+
+
 enum class Impl { kTensorCore, kSimt };
 
 // Host validation of a decode call and the kernel arguments it implies.
@@ -110,6 +130,9 @@ mlra_status decode_args(Impl impl, const mlra_dims* dims, const void* q_lat, con
     a.num_ctas = ctas;
     a.scale_log2 = scale * kLog2e;
     a.out_scale = out_scale;
+    a.w_uv = nullptr;
+    a.y = nullptr;
+    a.d_h = 0;
     return MLRA_OK;
 }
 
@@ -159,6 +182,28 @@ mlra_status mlra_decode(const mlra_dims* dims, const void* q_lat, const void* q_
                        seqlens, scale, out_scale, out, workspace, workspace_bytes, stream);
 }
 
+mlra_status mlra_decode_up_proj(const mlra_dims* dims, const void* q_lat, const void* q_rope,
+                                const void* latent_cache, const void* rope_cache,
+                                const int32_t* block_table, const int32_t* seqlens, float scale,
+                                float out_scale, void* out, const void* w_uv, int32_t d_h, void* y,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+    DecodeArgs a;
+    mlra_status s = decode_args(Impl::kTensorCore, dims, q_lat, q_rope, latent_cache, rope_cache, block_table,
+                                seqlens, scale, out_scale, out, workspace, workspace_bytes, &a);
+    if (s != MLRA_OK) return s;
+    if (!aligned16(w_uv)) return MLRA_ERR_INVALID_ARG;
+    if (d_h != 64 && d_h != 128) return MLRA_ERR_UNSUPPORTED;
+    if (dims->batch > kUpProjFusedMaxBatch || dims->heads * d_h / 16 > a.num_ctas) return MLRA_ERR_UNSUPPORTED;
+    void* y_dev = const_cast<void*>(device_address(y));  // y may be mapped pinned host memory
+    if (y_dev == nullptr || !aligned16(y_dev)) return MLRA_ERR_INVALID_ARG;
+    a.w_uv = static_cast<const __nv_bfloat16*>(w_uv);
+    a.y = static_cast<__nv_bfloat16*>(y_dev);
+    a.d_h = d_h;
+    const cudaError_t e = launch_decode_tc(a, static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorInvalidConfiguration) return MLRA_ERR_UNSUPPORTED;  // staging does not fit
+    return cuda_status(e);
+}
+
 mlra_status mlra_decode_simt(const mlra_dims* dims, const void* q_lat, const void* q_rope,
                              const void* latent_cache, const void* rope_cache,
                              const int32_t* block_table, const int32_t* seqlens, float scale,
@@ -169,7 +214,6 @@ mlra_status mlra_decode_simt(const mlra_dims* dims, const void* q_lat, const voi
 }
 
 namespace {
-const void* device_address(const void* p);
 
 mlra_status up_proj_impl(int32_t batch, int32_t heads, int32_t branches, int32_t d_c, int32_t d_h,
                          const void* out_lat, const void* w_uv, const void* gate, void* y, void* stream) {
@@ -291,26 +335,7 @@ mlra_status mlra_up_proj_allreduce(int32_t batch, int32_t heads, int32_t branche
     return cuda_status(e);
 }
 
-namespace {
-// The address through which the device reaches `p` (device, managed or
-// mapped pinned host memory), or null for memory the device cannot address.
-const void* device_address(const void* p) {
-    if (p == nullptr) return nullptr;
-    cudaPointerAttributes at;
-    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
-        cudaGetLastError();  // clear the error state the failed query leaves
-        return nullptr;
-    }
-    switch (at.type) {
-        case cudaMemoryTypeDevice:
-        case cudaMemoryTypeManaged:
-        case cudaMemoryTypeHost:
-            return at.devicePointer;
-        default:
-            return nullptr;
-    }
-}
-}  // namespace
+
 
 mlra_status mlra_copy_ranges(int32_t count, const void* const* src, void* const* dst, const uint64_t* bytes,
                              void* stream) {

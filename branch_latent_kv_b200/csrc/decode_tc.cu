@@ -132,11 +132,12 @@ struct Misc {
     uint64_t p_full[3];   // its probabilities are in shared memory
     uint64_t p_empty[3];  // its output MMA finished (S and P slots free, O up to date)
     uint64_t q_full;      // sequence range r (phase r & 1): its queries are in shared memory
-    uint64_t q_empty;     // its score MMAs finished
+    uint64_t q_empty;     // the score MMAs of a range with a successor have finished
     uint64_t drain[2];
+    uint64_t merge_full;  // the split merge's bulk copies have landed
     uint32_t tmem_base;
     int abort_flag;
-    int plan[4];
+    int plan[4];      // -, chunk, first sequence, its cost start
     int last_seg[3];  // this CTA's last sequence range: sequence, cost start, tiles (-1: none)
     int merge_flag;   // merge: bit 0 a split met a bad page, bit 1 a wait expired
     float red_max[4][2 * kHP];
@@ -253,6 +254,30 @@ __device__ __forceinline__ void finish_segment(int& n, int& cum, int tiles) {
     ++n;
 }
 
+// The sequence of the CTA's next range after sequence n (cost start cum,
+// `tiles` tiles) in its window [A0, A1), or -1 if n is its last.
+__device__ __forceinline__ int next_range_seq(const DecodeArgs& a, int n, int cum, int tiles, int A0, int A1) {
+    int c = cum + tiles * kTileCost + kSeqCost;
+    for (int m = n + 1; m < a.batch && c < A1; ++m) {
+        const int t = seq_tiles(__ldg(a.seqlens + m), a.page_size, a.max_pages);
+        if (t > 0) {
+            if (first_tile_at(c, t, A0) < first_tile_at(c, t, A1)) return m;
+            c += t * kTileCost + kSeqCost;
+        }
+    }
+    return -1;
+}
+
+// One sequence's queries (latent and RoPE, 16 head rows each) into the
+// query buffer, completing `full`; issued by one thread.
+template <class C>
+__device__ __forceinline__ void load_queries(const Maps& maps, uint8_t* sm, uint64_t& full, int seq) {
+    uint8_t* qd = sm + C::OFF_Q;
+    mbar_arrive_expect_tx(&full, C::Q_BYTES + C::QR_BYTES);
+    for (int c = 0; c < C::NCHUNK; ++c) tma_load_3d(qd + c * C::Q_CHUNK_BYTES, &maps.q, c * 64, 0, seq, &full);
+    tma_load_3d(qd + C::Q_BYTES, &maps.qr, 0, 0, seq, &full);
+}
+
 // End of the kernel, all threads: the merge of split sequences and the
 // outputs of sequences with an invalid length.
 //
@@ -263,17 +288,20 @@ __device__ __forceinline__ void finish_segment(int& n, int& cum, int tiles) {
 // (branch, latent column) rows, i = c - c0, G the group size:
 //   o = out_scale * sum_s w_s o_s / sum_s w_s,  w_s = 2^(lse_s - max_s lse_s)
 // per (branch, head) -- the log-sum-exp merge of independent softmax
-// partitions.  Every split's log-sum-exp row and its slice of partial rows
-// are fetched together (one round of L2 loads).  The last of the S + G
-// counts returns seq_cnt[n] to zero.
+// partitions, summed in split order.  The S log-sum-exp rows (consecutive
+// slots) and each split's slice of partial rows (contiguous) arrive by bulk
+// copies.  A CTA leaves the count as soon as its wait is over (the count
+// guards only the wait; the partials stay in place until the next launch),
+// and the last of the S + G counts returns seq_cnt[n] to zero.  The arithmetic
+// is laid out for latency: every thread loads its values for up to 8 splits
+// at once before combining them.
 template <int NB, int DC>
 __device__ __forceinline__ void merge_tail(const DecodeArgs& a, int n, int cum, int tiles, int chunk,
-                                           float* w_s, float* red, int* flag) {
+                                           float* w_s, int* flag, uint64_t* bar) {
     constexpr int HB = NB * kHP;  // (branch, head) columns of a split's log-sum-exp row
     constexpr int R = NB * DC;    // (branch, latent column) rows
     const int tid = threadIdx.x;
     const int H = a.heads;
-    static_assert(kThreads >= HB && kThreads / HB * HB <= 4 * 64, "merge reduction scratch");
 
     // invalid lengths: zeros and an error code, sequence m by CTA m mod grid
     const int next_len = (n >= 0 && n + 1 < a.batch) ? __ldg(a.seqlens + n + 1) : 0;
@@ -301,114 +329,120 @@ __device__ __forceinline__ void merge_tail(const DecodeArgs& a, int n, int cum, 
     const int gi = blockIdx.x - c0;  // 0 <= gi < G: n is this CTA's last sequence
     const int r0 = (int)((long long)gi * R / G), r1 = (int)((long long)(gi + 1) * R / G);
     const int rows = r1 - r0;
+    float* part_s = w_s + S * HB;  // [S][rows][16 heads]
     // wait until every split of n has counted its partials
     if (tid == 0) {
         const uint64_t t0 = globaltimer_ns();
+        bool ok = true;
         while (ld_acquire_gpu(a.seq_cnt + n) < S) {
             if (globaltimer_ns() - t0 > 2000000000ull) {
-                *flag = 2;
-                record_error(a.err, MLRA_ERR_DEVICE_TIMEOUT);
+                ok = false;
                 break;
             }
             __nanosleep(32);
         }
+        if (!ok) {
+            *flag = 2;
+            record_error(a.err, MLRA_ERR_DEVICE_TIMEOUT);
+        }
     }
     __syncthreads();
     if (*flag & 2) return;
-
-    // shared memory: w_s [S][HB] log-sum-exps (then weights), part_s
-    // [S][rows][16 heads] partial rows; slot of split s = c0 + s + n.  Every
-    // thread copies 16-byte units with L2 loads, sixteen in flight at a time
-    // (many small rows: plain loads keep far more requests in flight than
-    // one bulk copy per row would).
-    float* part_s = w_s + S * HB;
-    {
-        constexpr int LQ = HB / 4;               // 16-byte units per log-sum-exp row
-        const int lse_units = S * LQ;
-        const int row_units = rows * (kHP / 4);  // 16-byte units of one split's slice
-        const int total = lse_units + S * row_units;
-        for (int e0 = tid; e0 < total; e0 += 16 * kThreads) {
-            float4 v[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int e = e0 + j * kThreads;
-                if (e < lse_units) {
-                    v[j] = __ldcg(reinterpret_cast<const float4*>(a.lse_part + (size_t)(c0 + n + e / LQ) * HB) + e % LQ);
-                } else if (e < total) {
-                    const int u = e - lse_units, sp = u / row_units, r = u % row_units;
-                    v[j] = __ldcg(reinterpret_cast<const float4*>(a.o_part + ((size_t)(c0 + n + sp) * R + r0) * kHP) + r);
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int e = e0 + j * kThreads;
-                if (e < total) reinterpret_cast<float4*>(w_s)[e] = v[j];  // part_s follows w_s contiguously
-            }
+    int departed = 0;
+    if (tid < 32) {
+        // the partials were published by generic stores and acquired by
+        // thread 0 (ordered before this warp by the barrier); the copies read
+        // them through the async proxy
+        fence_proxy_async_global();
+        if (tid == 0) {
+            mbar_arrive_expect_tx(bar, (uint32_t)(S * HB + S * rows * kHP) * 4u);
+            bulk_load(w_s, a.lse_part + (size_t)(c0 + n) * HB, (uint32_t)(S * HB) * 4u, bar);
         }
+        __syncwarp();
+        if (rows > 0)
+            for (int sp = tid; sp < S; sp += 32)
+                bulk_load(part_s + (size_t)sp * rows * kHP, a.o_part + ((size_t)(c0 + n + sp) * R + r0) * kHP,
+                          (uint32_t)rows * kHP * 4u, bar);
+        // this CTA leaves the count (its result is needed only at the end)
+        if (tid == 0) departed = atomicAdd(a.seq_cnt + n, 1);
     }
-    __syncthreads();
-    // weights out_scale * 2^(lse - max) / sum per (branch, head) column: TPC
-    // threads per column, each over every TPC-th split (consecutive threads
-    // take consecutive columns: conflict-free), partial maxima and sums
-    // combined through red[TPC][HB]
-    {
-        constexpr int TPC = kThreads / HB;
-        const int col = tid % HB, grp = tid / HB;
-        const bool act = grp < TPC;
+    if (!mbar_wait(bar, 0)) {
+        // never expected: report it, and give the copies a last bounded
+        // chance to land before this CTA's shared memory goes away
+        if (tid == 0) record_error(a.err, MLRA_ERR_DEVICE_TIMEOUT);
+        mbar_wait(bar, 0, 200000000ull);
+        return;
+    }
+    // weights out_scale * 2^(lse - max) / sum, two threads per (branch, head)
+    // column, each over every other split, eight splits' values in flight
+    static_assert(2 * HB <= kThreads && HB % 16 == 0, "two threads per column in whole warps");
+    if (tid < 2 * HB) {
+        const int col = tid >> 1, half = tid & 1;
         float mx = -INFINITY;
         bool bad = false;
-        if (act)
-            for (int sp = grp; sp < S; sp += TPC) {
-                const float l = w_s[sp * HB + col];
-                if (l == bad_split_marker()) bad = true; else mx = fmaxf(mx, l);
+        for (int s0 = half; s0 < S; s0 += 16) {
+            float v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = s0 + 2 * j < S ? w_s[(s0 + 2 * j) * HB + col] : -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                bad |= v[j] == bad_split_marker();
+                if (v[j] != bad_split_marker()) mx = fmaxf(mx, v[j]);
             }
-        if (act) red[grp * HB + col] = bad ? bad_split_marker() : mx;
-        __syncthreads();
-        float M = -INFINITY;
-        bool bad_col = false;
-        if (act)
-            for (int g = 0; g < TPC; ++g) {
-                const float v = red[g * HB + col];
-                if (v == bad_split_marker()) bad_col = true; else M = fmaxf(M, v);
-            }
-        __syncthreads();
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        bad = __shfl_xor_sync(0xffffffffu, (int)bad, 1) != 0 || bad;
         float sum = 0.f;
-        if (act) {
-            for (int sp = grp; sp < S; sp += TPC) {
-                const float w = bad_col ? 0.f : fast_exp2(w_s[sp * HB + col] - M);
-                w_s[sp * HB + col] = w;
-                sum += w;
+        for (int s0 = half; s0 < S; s0 += 16) {
+            float v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = s0 + 2 * j < S ? w_s[(s0 + 2 * j) * HB + col] : -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                v[j] = bad ? 0.f : fast_exp2(v[j] - mx);
+                sum += v[j];
             }
-            red[grp * HB + col] = sum;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (s0 + 2 * j < S) w_s[(s0 + 2 * j) * HB + col] = v[j];
         }
-        __syncthreads();
-        if (act) {
-            float total = 0.f;
-            for (int g = 0; g < TPC; ++g) total += red[g * HB + col];
-            const float norm = bad_col ? 0.f : a.out_scale / total;
-            for (int sp = grp; sp < S; sp += TPC) w_s[sp * HB + col] *= norm;
-            if (bad_col && grp == 0 && col % kHP < H) atomicOr(flag, 1);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        const float norm = bad ? 0.f : a.out_scale / sum;
+        for (int s0 = half; s0 < S; s0 += 16) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (s0 + 2 * j < S) w_s[(s0 + 2 * j) * HB + col] *= norm;
         }
+        if (bad && half == 0 && col % kHP < H) atomicOr(flag, 1);
     }
     __syncthreads();
     const bool bad = *flag & 1;
     if (bad && tid == 0) record_error(a.err, MLRA_ERR_DEVICE_BAD_INDEX);
 
-    // items (row, head quad), quads fastest: conflict-free 16-byte reads
+    // items (row, head quad), quads fastest: conflict-free 16-byte reads; the
+    // weighted sum over the splits in split order, eight splits' loads at once
     for (int e = tid; e < rows * 4; e += kThreads) {
-        const int lr = e / 4, q = e % 4, row = r0 + lr;
+        const int lr = e >> 2, q = e & 3, row = r0 + lr;
         const int b = row / DC, k = row % DC;
         const float* w = w_s + b * kHP + 4 * q;
         const float* src = part_s + lr * kHP + 4 * q;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-        for (int sp = 0; sp < S; ++sp) {
-            const float4 v = *reinterpret_cast<const float4*>(src + (size_t)sp * rows * kHP);
-            const float4 wv = *reinterpret_cast<const float4*>(w + sp * HB);
-            acc.x = fmaf(wv.x, v.x, acc.x);
-            acc.y = fmaf(wv.y, v.y, acc.y);
-            acc.z = fmaf(wv.z, v.z, acc.z);
-            acc.w = fmaf(wv.w, v.w, acc.w);
+        for (int s0 = 0; s0 < S; s0 += 8) {
+            float4 v[8], wv[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const bool in = s0 + j < S;
+                v[j] = in ? *reinterpret_cast<const float4*>(src + (size_t)(s0 + j) * rows * kHP)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                wv[j] = in ? *reinterpret_cast<const float4*>(w + (s0 + j) * HB) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                acc.x = fmaf(wv[j].x, v[j].x, acc.x);
+                acc.y = fmaf(wv[j].y, v[j].y, acc.y);
+                acc.z = fmaf(wv[j].z, v[j].z, acc.z);
+                acc.w = fmaf(wv[j].w, v[j].w, acc.w);
+            }
         }
         if (bad) acc = make_float4(0.f, 0.f, 0.f, 0.f);
         __nv_bfloat16* dst = a.out + ((size_t)n * H * NB + b) * DC + k;
@@ -417,9 +451,144 @@ __device__ __forceinline__ void merge_tail(const DecodeArgs& a, int n, int cum, 
         for (int j = 0; j < 4; ++j)
             if (4 * q + j < H) dst[(size_t)(4 * q + j) * NB * DC] = to_bf16(v4[j]);
     }
+    if (tid == 0 && departed == S + G - 1) a.seq_cnt[n] = 0;
+}
+
+// ------------------------------------------------------------------ fused up-projection
+// The fused step (mlra_decode_up_proj): after the launch's merges, CTA c below
+// H d_h / 16 computes the 16 output columns [16 c, 16 c + 16) of
+//   y[n, h d_h + j] = sum_b sum_k out[n, h, b, k] W_UV[b][k][h d_h + j]
+// for every sequence n: the per-branch up-projection summed over the
+// branches is one K = B d_c reduction ("The Core Insight" section of the
+// wispaper.ai MLRA page: each branch is up-projected by its own matrix and
+// the branch outputs are summed).  Every CTA counts itself into a grid
+// counter once its merge duty is done (the spare word after the split
+// counters); the up-projection CTAs wait (bounded) for all of them, read the
+// latent output of their head for every sequence (rows padded to a multiple
+// of 16 with zeros) and multiply it on the warp-level tensor cores
+// (m16n8k16, fp32 accumulate) with K split over the warps; the warps' sums
+// meet in shared memory, in warp order.  The weight columns are staged
+// before the wait, transposed so that K is contiguous.
+constexpr int kUpMaxBatch = kUpProjFusedMaxBatch;
+
+template <int K>
+struct UpTile {
+    static constexpr int KP = K + 8;                       // row stride (bf16): conflict-free fragment reads
+    static constexpr int W_BYTES = 16 * KP * 2;            // the 16 weight columns, [16][KP]
+    static constexpr int X_BYTES = kUpMaxBatch * KP * 2;   // latent rows, [N padded][KP]
+    static constexpr int RED_BYTES = (kThreads / 32) * kUpMaxBatch * 16 * 4;
+    static constexpr int BYTES = W_BYTES + X_BYTES + RED_BYTES;
+};
+
+// The CTA's 16 weight columns into wt [16][KP] (at the end of the ring).
+template <int NB, int DC>
+__device__ __forceinline__ void up_stage_weights(const DecodeArgs& a, __nv_bfloat16* wt) {
+    constexpr int K = NB * DC;
+    using T = UpTile<K>;
+    const int cols = a.heads * a.d_h;
+    const int cb = blockIdx.x, h = cb / (a.d_h / 16), j0 = (cb % (a.d_h / 16)) * 16;
+    const __nv_bfloat16* src = a.w_uv + (size_t)h * a.d_h + j0;
+    for (int e = threadIdx.x; e < 2 * K; e += kThreads) {
+        const int k = e >> 1, half = e & 1;
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + (size_t)k * cols) + half);
+        const __nv_bfloat16* v8 = reinterpret_cast<const __nv_bfloat16*>(&v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) wt[(8 * half + i) * T::KP + k] = v8[i];
+    }
+}
+
+template <int NB, int DC>
+__device__ __forceinline__ void up_proj_tail(const DecodeArgs& a, uint8_t* ring, __nv_bfloat16* wt, int* flag) {
+    constexpr int K = NB * DC;
+    using T = UpTile<K>;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int N = a.batch, H = a.heads, ncb = H * a.d_h / 16;
+    const bool worker = (int)blockIdx.x < ncb;
+    int* gcnt = a.seq_cnt + kMaxBatch;
+    __syncthreads();  // the CTA's merge is done (and its weight columns staged)
+    if (tid == 0) red_add_release_gpu(gcnt, 1);
+    if (!worker) return;
+    int departed = 0;
+    if (tid == 0) {
+        const uint64_t t0 = globaltimer_ns();
+        bool ok = true;
+        while (ld_acquire_gpu(gcnt) < a.num_ctas) {
+            if (globaltimer_ns() - t0 > 2000000000ull) {
+                ok = false;
+                break;
+            }
+            __nanosleep(32);
+        }
+        if (ok) departed = atomicAdd(gcnt, 1);  // (the counter guards only this wait)
+        else {
+            *flag |= 4;
+            record_error(a.err, MLRA_ERR_DEVICE_TIMEOUT);
+        }
+    }
     __syncthreads();
-    // the last of the S arrivals and G departures resets the counter
-    if (tid == 0 && atomicAdd(a.seq_cnt + n, 1) == S + G - 1) a.seq_cnt[n] = 0;
+    if (*flag & 4) return;
+    const int h = blockIdx.x / (a.d_h / 16), j0 = (blockIdx.x % (a.d_h / 16)) * 16;
+    const int Np = (N + 15) & ~15;
+    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(ring);
+    float* red = reinterpret_cast<float*>(ring + T::X_BYTES);
+    // out[n][h][0..K) for every sequence, 16-byte units (rows past N zero)
+    for (int e = tid; e < Np * (K / 8); e += kThreads) {
+        const int n = e / (K / 8), u = e % (K / 8);
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (n < N) v = __ldcg(reinterpret_cast<const uint4*>(a.out + ((size_t)n * H + h) * K) + u);
+        *reinterpret_cast<uint4*>(xs + n * T::KP + 8 * u) = v;
+    }
+    __syncthreads();
+    const int g = lane >> 2, tg = lane & 3;
+    float acc[4][2][4];
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[mt][t][i] = 0.f;
+    for (int ks = warp; ks < K / 16; ks += kThreads / 32) {
+        const int kb = 16 * ks + 2 * tg;
+        uint32_t b[2][2];
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            b[t][0] = *reinterpret_cast<const uint32_t*>(wt + (8 * t + g) * T::KP + kb);
+            b[t][1] = *reinterpret_cast<const uint32_t*>(wt + (8 * t + g) * T::KP + kb + 8);
+        }
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+            if (16 * mt >= Np) break;
+            const __nv_bfloat16* x0 = xs + (16 * mt + g) * T::KP + kb;
+            const uint32_t af[4] = {*reinterpret_cast<const uint32_t*>(x0),
+                                    *reinterpret_cast<const uint32_t*>(x0 + 8 * T::KP),
+                                    *reinterpret_cast<const uint32_t*>(x0 + 8),
+                                    *reinterpret_cast<const uint32_t*>(x0 + 8 * T::KP + 8)};
+#pragma unroll
+            for (int t = 0; t < 2; ++t) mma_m16n8k16_bf16(acc[mt][t], af, b[t][0], b[t][1]);
+        }
+    }
+    // the warps' partial sums: red[warp][row][16 columns]
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+        if (16 * mt >= Np) break;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            float* r = red + ((size_t)warp * kUpMaxBatch + 16 * mt + g) * 16 + 8 * t + 2 * tg;
+            r[0] = acc[mt][t][0];
+            r[1] = acc[mt][t][1];
+            r[8 * 16] = acc[mt][t][2];
+            r[8 * 16 + 1] = acc[mt][t][3];
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < N * 16; e += kThreads) {
+        const int n = e >> 4, j = e & 15;
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < kThreads / 32; ++w) v += red[((size_t)w * kUpMaxBatch + n) * 16 + j];
+        a.y[(size_t)n * H * a.d_h + h * a.d_h + j0 + j] = to_bf16(v);
+    }
+    if (tid == 0 && departed == a.num_ctas + ncb - 1) *gcnt = 0;
 }
 
 template <int NB, int DC, int DR>
@@ -434,6 +603,10 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int P = a.page_size;
 
+    if (warp == 0 && lane < 4) {
+        // descriptor fetches overlap the set-up below
+        prefetch_tensormap(lane == 0 ? &maps.lat : lane == 1 ? &maps.rope : lane == 2 ? &maps.q : &maps.qr);
+    }
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::NSTAGE; ++i) {
             mbar_init(&misc.pair_full[i], 1);
@@ -451,47 +624,53 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
             mbar_init(&misc.p_empty[i], 1);
         }
         mbar_init(&misc.q_full, 1);
+        mbar_init(&misc.merge_full, 1);
         mbar_init(&misc.q_empty, 1);
         misc.abort_flag = 0;
         misc.last_seg[0] = -1;
         misc.merge_flag = 0;
         fence_barrier_init();
     }
+    launch_dependents();  // a dependent kernel may be scheduled as CTAs retire
+    // Warp 0 computes the plan and goes straight on to its copies; the other
+    // warps allocate TMEM and meet it (named barrier 2) for the plan.
+    int n_first, cum_first;
     if (warp == 0) {
-        // descriptor fetches overlap the loads of the lengths below
-        prefetch_tensormap(&maps.lat);
-        prefetch_tensormap(&maps.rope);
-        prefetch_tensormap(&maps.q);
-        prefetch_tensormap(&maps.qr);
+        // the inputs may come from the preceding kernel (programmatic launch)
+        wait_prerequisite_grid();
         const int total = warp_cost_prefix(a.seqlens, a.batch, P, a.max_pages);
         const int chunk = plan_chunk(total, a.num_ctas);
-        int n0 = a.batch, cum0 = total;
+        n_first = a.batch;
+        cum_first = total;
         if ((long long)blockIdx.x * chunk < total)
-            warp_find_seq(a.seqlens, a.batch, P, a.max_pages, blockIdx.x * chunk, &n0, &cum0);
+            warp_find_seq(a.seqlens, a.batch, P, a.max_pages, blockIdx.x * chunk, &n_first, &cum_first);
         if (lane == 0) {
             misc.plan[1] = chunk;
-            misc.plan[2] = n0;
-            misc.plan[3] = cum0;
+            misc.plan[2] = n_first;
+            misc.plan[3] = cum_first;
         }
+        __syncwarp();
+        named_bar_arrive<2, kThreads>();
+    } else {
+        if (warp == 1) {
+            tmem_alloc(&misc.tmem_base, C::TMEM_COLS);
+            tmem_relinquish();
+        }
+        tc_fence_before();
+        named_bar_sync<2, kThreads>();
+        tc_fence_after();
+        n_first = misc.plan[2];
+        cum_first = misc.plan[3];
     }
-    if (warp == 1) {
-        tmem_alloc(&misc.tmem_base, C::TMEM_COLS);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
-    launch_dependents();  // the combine kernel may be scheduled as CTAs retire
     const int chunk = misc.plan[1];
     const int A0 = blockIdx.x * chunk, A1 = A0 + chunk;  // this CTA's cost window
-    const uint32_t tmem = misc.tmem_base;
+    const uint32_t tmem = misc.tmem_base;                // (warp 0 never uses it)
     volatile int* abort_flag = &misc.abort_flag;
 
-    if (misc.plan[2] < a.batch) {
+    if (n_first < a.batch) {
         if (warp == 0) {
             // ------------------------------------------------------------ producer
-            int n = misc.plan[2], cum = misc.plan[3], next_len = first_len(a, n);
+            int n = n_first, cum = cum_first, next_len = first_len(a, n);
             int L, tiles, tb, te;
             uint32_t pc = 0, tc = 0, sc = 0;
             // the cache is read once per step: its lines go first, and the
@@ -499,19 +678,10 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
             const uint64_t stream_policy = l2_policy_evict_first();
             bool ok = true;
             while (ok && next_segment(a, n, cum, A0, A1, L, tiles, tb, te, next_len)) {
-                // the sequence's queries, once the previous range has finished
-                // its score MMAs
-                if (lane == 0) {
-                    if (sc >= 1) ok = mbar_wait(&misc.q_empty, (sc - 1) & 1);
-                    if (ok) {
-                        uint64_t* qb = &misc.q_full;
-                        uint8_t* qd = sm + C::OFF_Q;
-                        mbar_arrive_expect_tx(qb, C::Q_BYTES + C::QR_BYTES);
-                        for (int c = 0; c < C::NCHUNK; ++c)
-                            tma_load_3d(qd + c * C::Q_CHUNK_BYTES, &maps.q, c * 64, 0, n, qb);
-                        tma_load_3d(qd + C::Q_BYTES, &maps.qr, 0, 0, n, qb);
-                    }
-                }
+                // the first range's queries; a later range's are loaded by the
+                // score MMA warp once the range before has its last scores, so
+                // the copies of the cache never wait for the query buffer
+                if (lane == 0 && sc == 0) load_queries<C>(maps, sm, misc.q_full, n);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 ++sc;
@@ -598,9 +768,9 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
             const uint64_t dQ = smem_desc(sm_base + C::OFF_Q, 16, 1024, kLayoutSw128);
             const uint64_t dQR = rope_desc<DR>(sm_base + C::OFF_QR);
             const uint64_t dR = rope_desc<DR>(sm_base + C::OFF_ROPE);
-            int n = misc.plan[2], cum = misc.plan[3], next_len = first_len(a, n);
+            int n = n_first, cum = cum_first, next_len = first_len(a, n);
             int L, tiles, tb, te;
-            uint32_t gs = 0, tc = 0, sc = 0;
+            uint32_t gs = 0, tc = 0, sc = 0, qe = 0;
             uint32_t stage = 0, phase = 0;  // ring position of the next pair to consume
             bool ok = true;
             while (ok && next_segment(a, n, cum, A0, A1, L, tiles, tb, te, next_len)) {
@@ -666,9 +836,17 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                     ++tc;
                     if (__shfl_sync(0xffffffffu, *abort_flag, 0)) ok = false;
                 }
-                // the queries' slot is free once this range's score MMAs finish
-                if (ok && elect_one()) mma_commit(&misc.q_empty);
-                __syncwarp();
+                // a next range: its queries replace these once this range's
+                // score MMAs have finished
+                const int nn = next_range_seq(a, n, cum, tiles, A0, A1);
+                if (ok && nn >= 0) {
+                    if (elect_one()) mma_commit(&misc.q_empty);
+                    __syncwarp();
+                    ok = mbar_wait_warp(&misc.q_empty, qe & 1);
+                    ++qe;
+                    if (ok && elect_one()) load_queries<C>(maps, sm, misc.q_full, nn);
+                    __syncwarp();
+                }
                 ++sc;
                 finish_segment(n, cum, tiles);
             }
@@ -687,7 +865,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
             const uint32_t sm_base = smem_u32(sm);
             const uint64_t dA_pv = smem_desc(sm_base + C::OFF_PAIR, C::CHUNK_BYTES, 1024, kLayoutSw128);  // MN-major
             const uint64_t dP = smem_desc(sm_base + C::OFF_P, 128, 2048, kLayoutNone);
-            int n = misc.plan[2], cum = misc.plan[3], next_len = first_len(a, n);
+            int n = n_first, cum = cum_first, next_len = first_len(a, n);
             int L, tiles, tb, te;
             uint32_t gs = 0;
             uint32_t stage = 0;  // ring position of the step's first pair
@@ -746,7 +924,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
             const int stid = threadIdx.x - 64;         // 0..127 within the group
             const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
             const int H = a.heads;
-            int n = misc.plan[2], cum = misc.plan[3], next_len = first_len(a, n);
+            int n = n_first, cum = cum_first, next_len = first_len(a, n);
             int L, tiles, tb, te;
             uint32_t gs = 0, sc = 0, tcnt = 0;  // steps, ranges, tiles so far
             // This thread's share of the softmax denominators, one row per
@@ -777,6 +955,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                         const uint32_t slot = gs % C::NSP;
                         const bool ok = mbar_wait(&misc.s_full[slot], (gs / C::NSP) & 1);
                         tc_fence_after();
+
                         float x[C::SBR][kHP];
                         if (st == 0) tmem_ld16(tmem + lane_off + C::R_COL0 + (tcnt % C::NRS) * kHP, r);
 #pragma unroll
@@ -951,9 +1130,8 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                     }
                 }
                 bad = named_bar_or<1, 128>(bad);  // also publishes red_sum
-                int first_cta, last_cta;
-                seq_owners(cum, tiles, chunk, &first_cta, &last_cta);
-                const bool single = first_cta == last_cta;
+                // one window holds every tile of the sequence: no split
+                const bool single = cum >= A0 && cum + (tiles - 1) * kTileCost < A1;
                 const size_t slot = (size_t)blockIdx.x + n;
                 if (stid < NB * kHP) {
                     const float lt = misc.red_sum[0][stid] + misc.red_sum[1][stid] + misc.red_sum[2][stid] +
@@ -997,11 +1175,13 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                         for (int i = 0; i < kHP; ++i)
                             if (i < H) dst[(size_t)i * NB * DC] = to_bf16(o[blk][i] * a.out_scale);
                     } else {
-                        // partial layout [slot][branch][k][16 heads]: 64 contiguous bytes per row
-                        float4* dst = reinterpret_cast<float4*>(a.o_part + (((slot * NB + b) * DC + k) * kHP));
-#pragma unroll
-                        for (int i = 0; i < kHP; i += 4)
-                            dst[i / 4] = make_float4(o[blk][i], o[blk][i + 1], o[blk][i + 2], o[blk][i + 3]);
+                        // partial layout [slot][branch][k][16 heads]: one 64-byte
+                        // row per thread, two 32-byte stores
+                        float* dst = a.o_part + ((slot * NB + b) * DC + k) * kHP;
+                        st_global_v8(dst, o[blk][0], o[blk][1], o[blk][2], o[blk][3], o[blk][4], o[blk][5],
+                                     o[blk][6], o[blk][7]);
+                        st_global_v8(dst + 8, o[blk][8], o[blk][9], o[blk][10], o[blk][11], o[blk][12],
+                                     o[blk][13], o[blk][14], o[blk][15]);
                     }
                 }
                 if (bad && stid == 0) record_error(a.err, MLRA_ERR_DEVICE_BAD_INDEX);
@@ -1027,7 +1207,9 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                 *abort_flag = 1;
             }
             if (!dead && stid == 0 && pend_a >= 0) {
-                __threadfence();
+                // the partial stores of all 128 threads precede the named
+                // barrier that ended their epilogue; the release makes them
+                // visible with the count
                 red_add_release_gpu(a.seq_cnt + pend_a, 1);
                 if (pend_b >= 0) red_add_release_gpu(a.seq_cnt + pend_b, 1);
             }
@@ -1040,9 +1222,15 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
     if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
     if (*abort_flag) return;
     // the ring's shared memory is free from here on: the merge stages its
-    // weights there
+    // partials at its start, the fused up-projection its weight columns at
+    // its end
+    __nv_bfloat16* wt = reinterpret_cast<__nv_bfloat16*>(sm + C::OFF_PAIR + C::NSTAGE * C::PAIR_BYTES -
+                                                         UpTile<NB * DC>::W_BYTES);
+    const bool fused = a.w_uv != nullptr;
+    if (fused && (int)blockIdx.x < a.heads * a.d_h / 16) up_stage_weights<NB, DC>(a, wt);
     merge_tail<NB, DC>(a, misc.last_seg[0], misc.last_seg[1], misc.last_seg[2], chunk,
-                       reinterpret_cast<float*>(sm + C::OFF_PAIR), &misc.red_sum[0][0], &misc.merge_flag);
+                       reinterpret_cast<float*>(sm + C::OFF_PAIR), &misc.merge_flag, &misc.merge_full);
+    if (fused) up_proj_tail<NB, DC>(a, sm + C::OFF_PAIR, wt, &misc.merge_flag);
 }
 
 // ------------------------------------------------------------------ host side
@@ -1102,12 +1290,16 @@ cudaError_t launch_cfg(const DecodeArgs& a, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     // the merge stages in the ring: for all S <= grid splits of a sequence the
-    // log-sum-exp rows (S NB 16 floats), S row slices of at most
-    // R / (S - 1) + 1 rows of 16 floats (at most 2 R + S rows in all), the
-    // column partials (2 kThreads floats at most) and factors (NB 16 floats)
-    const size_t merge_bytes = sizeof(float) * ((size_t)a.num_ctas * NB * kHP + (2 * (size_t)C::W + a.num_ctas) * kHP +
-                                                2 * (size_t)kThreads + NB * kHP);
-    if (merge_bytes > (size_t)C::NSTAGE * C::PAIR_BYTES) return cudaErrorInvalidConfiguration;
+    // log-sum-exp rows (S NB 16 floats) and S row slices of at most
+    // R / (S - 1) + 1 rows of 16 floats (at most 2 R + S rows in all)
+    const size_t merge_bytes = sizeof(float) * ((size_t)a.num_ctas * NB * kHP + (2 * (size_t)C::W + a.num_ctas) * kHP);
+    const size_t ring = (size_t)C::NSTAGE * C::PAIR_BYTES;
+    if (merge_bytes > ring) return cudaErrorInvalidConfiguration;
+    // the fused up-projection: weight columns at the ring's end (staged while
+    // the merge uses its start), then its rows and sums from the start
+    if (a.w_uv != nullptr &&
+        (merge_bytes + UpTile<NB * DC>::W_BYTES > ring || (size_t)UpTile<NB * DC>::BYTES > ring))
+        return cudaErrorInvalidConfiguration;
     // Cooperative: every CTA is resident at once, so the merge's wait for the
     // other splits of a sequence always ends.
     cudaLaunchConfig_t cfg = {};
@@ -1115,11 +1307,16 @@ cudaError_t launch_cfg(const DecodeArgs& a, cudaStream_t stream) {
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    // Programmatic: the CTAs of this launch may set up (barriers, TMEM) on SMs
+    // the preceding kernel has released, and wait for its completion only
+    // before reading inputs.
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kernel, maps, a);
 }
 

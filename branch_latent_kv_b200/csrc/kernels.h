@@ -27,6 +27,11 @@ struct DecodeArgs {
     int num_ctas;                 // grid of the split kernel (partial slots = num_ctas + batch)
     float scale_log2;             // scale * log2(e)
     float out_scale;
+    // the fused step (mlra_decode_up_proj): after the merges the same launch
+    // up-projects the latent output; w_uv null: no up-projection
+    const __nv_bfloat16* w_uv;    // [B, d_c, H * d_h]
+    __nv_bfloat16* y;             // [N, H * d_h] (device address)
+    int d_h;
 };
 
 // Host validation of a tensor-core decode call (what mlra_decode checks);
@@ -35,6 +40,10 @@ mlra_status decode_tc_args(const mlra_dims* dims, const void* q_lat, const void*
                            const void* latent_cache, const void* rope_cache, const int32_t* block_table,
                            const int32_t* seqlens, float scale, float out_scale, void* out, void* workspace,
                            size_t workspace_bytes, DecodeArgs* a);
+
+// Largest batch of the fused decode + up-projection (its latent rows of one
+// head for every sequence are staged in shared memory).
+constexpr int kUpProjFusedMaxBatch = 64;
 
 // Split-KV decode on CUDA cores (fp32 FMA).  Writes final outputs of
 // single-split sequences and partials of the others.

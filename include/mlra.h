@@ -132,6 +132,32 @@ MLRA_API mlra_status mlra_decode(const mlra_dims* dims, const void* q_lat, const
                         void* stream);
 
 /*
+ * The whole decode step in one launch: mlra_decode's attention and split
+ * merge, then the per-branch W_UV up-projection and branch sum of its output
+ * (what mlra_up_proj computes; "The Core Insight" section of the blog page:
+ * each branch is up-projected by its own matrix and the branch outputs are
+ * summed):
+ *   y[n, h*d_h + j] = sum_b sum_k out[n,h,b,k] * w_uv[b][k][h*d_h + j]
+ * Arguments as mlra_decode, plus
+ *   w_uv  bf16 [branches, d_c, heads * d_h]
+ *   d_h   64 or 128
+ *   y     bf16 [batch, heads * d_h], written; device memory or pinned host
+ *         memory the device can map
+ * `out` is written exactly as mlra_decode writes it (the same bits).  After
+ * the launch's merges the CTAs meet once (a bounded grid-wide wait, reported
+ * as MLRA_ERR_DEVICE_TIMEOUT if it expires) and heads * d_h / 16 of them form
+ * 16 output columns each, in fp32 on the warp-level tensor cores.
+ * Supported: the shapes of mlra_decode with batch <= 64 and
+ * heads * d_h / 16 <= the SM count; other calls return MLRA_ERR_UNSUPPORTED
+ * (use mlra_decode and mlra_up_proj).
+ */
+MLRA_API mlra_status mlra_decode_up_proj(const mlra_dims* dims, const void* q_lat, const void* q_rope,
+                                         const void* latent_cache, const void* rope_cache,
+                                         const int32_t* block_table, const int32_t* seqlens, float scale,
+                                         float out_scale, void* out, const void* w_uv, int32_t d_h, void* y,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * The same operation as mlra_decode, computed by a split-KV kernel on the
  * CUDA cores (fp32 FMA) instead of the tensor cores: same arguments, same
  * workspace, same outputs within the stated tolerance.  It covers more

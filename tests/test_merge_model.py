@@ -6,9 +6,11 @@ splits owned by CTAs c0..c1 (the plan of `plan_model`):
     seq_cnt[n] (an arrival; a CTA has at most two split sequences, the first
     and the last of its range);
   - the CTAs whose range ends in n (c0..c1-1, and c1 when n is its last
-    sequence: G of them) wait until seq_cnt[n] >= S, merge their share of the
-    rows, then add 1 (a departure); the one whose add sees S + G - 1 returns
-    the counter to zero for the next launch.
+    sequence: G of them) wait until seq_cnt[n] >= S, then add 1 (a
+    departure) and merge their share of the rows; the one whose add sees
+    S + G - 1 returns the counter to zero for the next launch.  (The count
+    guards only the wait: the partials a member reads after leaving it stay
+    in place until the next launch, which starts after this one completes.)
 CTAs interleave arbitrarily within a launch; launches follow each other.
 
 The model draws lengths and grid sizes, derives the splits and groups from
