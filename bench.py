@@ -350,7 +350,8 @@ def workload_config(w, copies):
            "d_c": w.d_c, "d_r": w.d_r, "page_size": w.page_size, "d_h": w.d_h,
            "seq_len": w.seqlen if w.seqlen is not None else f"U{{{w.seqlen_range[0]}..{w.seqlen_range[1]}}}",
            "page_order": w.page_order, "parallelism": "replicas (one independent step per GPU)",
-           "step": "mlra_decode (split-KV kernel with in-kernel LSE merge) + mlra_up_proj"}
+           "step": "mlra_decode_up_proj (one launch: split-KV attention, in-kernel LSE merge, per-branch "
+                   "W_UV up-projection and branch sum); batch > 64: mlra_decode + mlra_up_proj"}
     if copies is not None:
         cfg["l2"] = f"inputs larger than L2: {copies} rotating copies of the KV pools"
     return cfg
@@ -391,6 +392,8 @@ def main():
     ap.add_argument("--workloads", default=",".join(OTHER_WORKLOADS),
                     help="decode-kernel figures of these workloads in the line ('' for none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--two-kernel-step", action="store_true",
+                    help="time the step as mlra_decode + mlra_up_proj (two launches) instead of the fused launch")
     ap.add_argument("--profile", action="store_true",
                     help="run W + K device-resident steps only and print nothing (for profilers)")
     args = ap.parse_args()
@@ -432,9 +435,17 @@ def main():
     def up_call():
         b.mlra_up_proj(out, x.w_uv, y=y)
 
+    # the step: one launch of the fused decode + up-projection where it covers
+    # the shape (batch <= 64), else the two kernels
+    fused = w.batch <= 64 and not args.two_kernel_step
+
     def step(i):
-        decode_call(i)
-        up_call()
+        if fused:
+            b.mlra_decode_up_proj(x.q_lat, x.q_rope, lat[i % copies], rope[i % copies], x.block_table,
+                                  x.seqlens, x.scale, x.out_scale, x.w_uv, out=out, y=y, workspace=ws)
+        else:
+            decode_call(i)
+            up_call()
 
     if args.profile:
         for i in range(args.warmup + args.steps):
@@ -462,14 +473,12 @@ def main():
     for c in range(copies):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=cap):
-            decode_call(c)
-            up_call()
+            step(c)
         step_graphs.append(g)
     chain_steps, chain_decode = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     with torch.cuda.graph(chain_steps, stream=cap):
         for c in range(copies):
-            decode_call(c)
-            up_call()
+            step(c)
     with torch.cuda.graph(chain_decode, stream=cap):
         for c in range(copies):
             decode_call(c)
@@ -594,7 +603,8 @@ def main():
                      "peak_source": f"{peak_kind} hbm_gbs"},
         "e2e": {"value": kv * world * args.steps / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 2 * args.steps,  # per step: the decode kernel and the up-projection
+        # per step: the fused decode + up-projection kernel, or the two kernels
+        "gpu_launches": (1 if fused else 2) * args.steps,
         "prestep": {"kernel": "prepare_kernel (mlra_prepare: query absorption, rotary embedding, "
                               "append of the new token)", "us_per_launch": pre_us,
                     "note": "not part of the step above; timed in its own loop on the same batch "

@@ -138,7 +138,7 @@ struct Misc {
     uint32_t tmem_base;
     int abort_flag;
     int plan[4];      // -, chunk, first sequence, its cost start
-    int last_seg[3];  // this CTA's last sequence range: sequence, cost start, tiles (-1: none)
+    int last_seg[4];  // this CTA's last sequence range: sequence, cost start, tiles (-1: none), c1 merges
     int merge_flag;   // merge: bit 0 a split met a bad page, bit 1 a wait expired
     float red_max[4][2 * kHP];
     float red_sum[4][4 * kHP];
@@ -278,8 +278,7 @@ __device__ __forceinline__ void load_queries(const Maps& maps, uint8_t* sm, uint
     tma_load_3d(qd + C::Q_BYTES, &maps.qr, 0, 0, seq, &full);
 }
 
-// End of the kernel, all threads: the merge of split sequences and the
-// outputs of sequences with an invalid length.
+// End of the kernel, all threads: the merge of split sequences.
 //
 // Sequence n with S > 1 splits (CTAs c0..c1) is merged by the CTAs whose
 // range ends in it: c0..c1-1 always, c1 when n is also its last sequence.
@@ -296,35 +295,20 @@ __device__ __forceinline__ void load_queries(const Maps& maps, uint8_t* sm, uint
 // is laid out for latency: every thread loads its values for up to 8 splits
 // at once before combining them.
 template <int NB, int DC>
-__device__ __forceinline__ void merge_tail(const DecodeArgs& a, int n, int cum, int tiles, int chunk,
-                                           float* w_s, int* flag, uint64_t* bar) {
+__device__ __forceinline__ void merge_tail(const DecodeArgs& a, int n, int cum, int tiles, bool c1_member,
+                                           int chunk, float* w_s, int* flag, uint64_t* bar) {
     constexpr int HB = NB * kHP;  // (branch, head) columns of a split's log-sum-exp row
     constexpr int R = NB * DC;    // (branch, latent column) rows
     const int tid = threadIdx.x;
     const int H = a.heads;
 
-    // invalid lengths: zeros and an error code, sequence m by CTA m mod grid
-    const int next_len = (n >= 0 && n + 1 < a.batch) ? __ldg(a.seqlens + n + 1) : 0;
-    for (int m = blockIdx.x; m < a.batch; m += a.num_ctas) {
-        if (seq_tiles(__ldg(a.seqlens + m), a.page_size, a.max_pages) > 0) continue;
-        __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(a.out + (size_t)m * H * R);
-        for (int e = tid; e < H * R / 2; e += kThreads) dst[e] = __floats2bfloat162_rn(0.f, 0.f);
-        if (tid == 0) record_error(a.err, MLRA_ERR_DEVICE_BAD_SEQLEN);
-    }
     if (n < 0) return;
     int c0, c1;
     seq_owners(cum, tiles, chunk, &c0, &c1);
     const int S = c1 - c0 + 1;
     if (S == 1) return;  // written by the epilogue
-    // c1 belongs to the group when no later tile is its own: the next valid
-    // sequence starts at cum + cost_n, owned by c1 or a later CTA
-    bool c1_member = true;
-    for (int m = n + 1; m < a.batch; ++m) {
-        const int Lm = m == n + 1 ? next_len : __ldg(a.seqlens + m);
-        if (seq_tiles(Lm, a.page_size, a.max_pages) == 0) continue;
-        c1_member = (cum + tiles * kTileCost + kSeqCost) / chunk != c1;
-        break;
-    }
+    // c1 belongs to the group when no later tile is its own (the next valid
+    // sequence starts in a later window); worked out at the range's start
     const int G = c1_member ? S : S - 1;
     const int gi = blockIdx.x - c0;  // 0 <= gi < G: n is this CTA's last sequence
     const int r0 = (int)((long long)gi * R / G), r1 = (int)((long long)(gi + 1) * R / G);
@@ -661,6 +645,18 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
         tc_fence_after();
         n_first = misc.plan[2];
         cum_first = misc.plan[3];
+        if (warp == 6) {
+            // sequences with an invalid length: zeros and an error code,
+            // sequence m by CTA m mod grid (this warp is idle until the first
+            // probabilities of its CTA are ready)
+            const int R = NB * DC;
+            for (int m = blockIdx.x; m < a.batch; m += a.num_ctas) {
+                if (seq_tiles(__ldg(a.seqlens + m), P, a.max_pages) > 0) continue;
+                __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(a.out + (size_t)m * a.heads * R);
+                for (int e = lane; e < a.heads * R / 2; e += 32) dst[e] = __floats2bfloat162_rn(0.f, 0.f);
+                if (lane == 0) record_error(a.err, MLRA_ERR_DEVICE_BAD_SEQLEN);
+            }
+        }
     }
     const int chunk = misc.plan[1];
     const int A0 = blockIdx.x * chunk, A1 = A0 + chunk;  // this CTA's cost window
@@ -940,6 +936,18 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                 // issued at the tile's start and consumed at its end)
                 bool bad = false;
                 const int32_t* bt = a.block_table + (size_t)n * a.max_pages;
+                // for the merge at the kernel's end: whether the CTA owning
+                // this sequence's last tile also merges it (no later sequence
+                // starts in its window); worked out now, off the critical path
+                int c1_member = 1;
+                if (stid == 0) {
+                    const int c1 = (cum + (tiles - 1) * kTileCost) / chunk;
+                    for (int m = n + 1; m < a.batch; ++m) {
+                        if (seq_tiles(__ldg(a.seqlens + m), a.page_size, a.max_pages) == 0) continue;
+                        c1_member = (cum + tiles * kTileCost + kSeqCost) / chunk != c1;
+                        break;
+                    }
+                }
 #pragma unroll
                 for (int b = 0; b < NB; ++b)
 #pragma unroll
@@ -1198,6 +1206,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                     misc.last_seg[0] = n;
                     misc.last_seg[1] = cum;
                     misc.last_seg[2] = tiles;
+                    misc.last_seg[3] = c1_member;
                 }
                 ++sc;
                 finish_segment(n, cum, tiles);
@@ -1208,10 +1217,11 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
             }
             if (!dead && stid == 0 && pend_a >= 0) {
                 // the partial stores of all 128 threads precede the named
-                // barrier that ended their epilogue; the release makes them
-                // visible with the count
-                red_add_release_gpu(a.seq_cnt + pend_a, 1);
-                if (pend_b >= 0) red_add_release_gpu(a.seq_cnt + pend_b, 1);
+                // barrier that ended their epilogue; one release fence makes
+                // them visible before both counts
+                fence_acq_rel_gpu();
+                red_add_relaxed_gpu(a.seq_cnt + pend_a, 1);
+                if (pend_b >= 0) red_add_relaxed_gpu(a.seq_cnt + pend_b, 1);
             }
         }
     }
@@ -1228,7 +1238,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                                                          UpTile<NB * DC>::W_BYTES);
     const bool fused = a.w_uv != nullptr;
     if (fused && (int)blockIdx.x < a.heads * a.d_h / 16) up_stage_weights<NB, DC>(a, wt);
-    merge_tail<NB, DC>(a, misc.last_seg[0], misc.last_seg[1], misc.last_seg[2], chunk,
+    merge_tail<NB, DC>(a, misc.last_seg[0], misc.last_seg[1], misc.last_seg[2], misc.last_seg[3] != 0, chunk,
                        reinterpret_cast<float*>(sm + C::OFF_PAIR), &misc.merge_flag, &misc.merge_full);
     if (fused) up_proj_tail<NB, DC>(a, sm + C::OFF_PAIR, wt, &misc.merge_flag);
 }

@@ -323,6 +323,13 @@ __device__ __forceinline__ void wait_prerequisite_grid() { asm volatile("griddep
 __device__ __forceinline__ void red_add_release_gpu(int* p, int v) {
     asm volatile("red.release.gpu.global.add.s32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
 }
+// A release fence at GPU scope followed by relaxed adds: one fence publishes
+// every earlier write (this thread's, and those ordered before it by a CTA
+// barrier) before all the adds that follow.
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+__device__ __forceinline__ void red_add_relaxed_gpu(int* p, int v) {
+    asm volatile("red.relaxed.gpu.global.add.s32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
 __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
     int v;
     asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");

@@ -2,7 +2,9 @@
 
 A serving loop calls the same decode step every token with the same buffer
 shapes.  ``DecodeStep`` validates the arguments once (one eager call of
-``mlra_decode`` and, when ``w_uv`` is given, ``mlra_up_proj``), then captures
+``mlra_decode`` or, when ``w_uv`` is given, ``mlra_decode_up_proj``: the
+whole step in one launch; batches above 64 use ``mlra_decode`` and
+``mlra_up_proj``), then captures
 the step -- optionally with the host-to-device transfer of its inputs and the
 device-to-host transfer of its result -- into a CUDA graph, so each step costs
 one graph launch on the host.  The inputs cross PCIe in one launch of
@@ -83,6 +85,9 @@ class DecodeStep:
         self.host_output = host_output
         self._args = (q_lat, q_rope, latent_cache, rope_cache, block_table, seqlens, scale, out_scale)
         self._w_uv, self._d_h = w_uv, d_h
+        # decode and up-projection in one launch where that kernel covers the
+        # shape (batch <= 64), else the two launches
+        self._fused = w_uv is not None and q_lat.shape[0] <= 64
 
         # validation: one eager pass (raises on any argument error) on the
         # step's real inputs: the host inputs, if any, are brought in first,
@@ -112,12 +117,16 @@ class DecodeStep:
                 # the mapped pinned pages), not one DMA copy per tensor
                 b.mlra_copy_ranges([(h, self.inputs[name]) for name, h in self.host_inputs.items()],
                                    stream=stream, device=self.device)
-            b.mlra_decode(*self._args, out=self.out, workspace=self.workspace, stream=stream)
             direct = copies and self.host_output is not None and self._w_uv is not None
-            if self._w_uv is not None:
-                # with a host output, the up-projection writes y straight into it
-                b.mlra_up_proj(self.out, self._w_uv, d_h=self._d_h, y=self.host_output if direct else self.y,
-                               stream=stream)
+            y_dst = self.host_output if direct else self.y  # a host output is written straight from the kernel
+            if self._w_uv is not None and self._fused:
+                # the whole step in one launch
+                b.mlra_decode_up_proj(*self._args, self._w_uv, d_h=self._d_h, out=self.out, y=y_dst,
+                                      workspace=self.workspace, stream=stream)
+            else:
+                b.mlra_decode(*self._args, out=self.out, workspace=self.workspace, stream=stream)
+                if self._w_uv is not None:
+                    b.mlra_up_proj(self.out, self._w_uv, d_h=self._d_h, y=y_dst, stream=stream)
             if copies and self.host_output is not None and not direct:
                 self.host_output.copy_(self.out, non_blocking=True)
 

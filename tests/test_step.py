@@ -1,5 +1,7 @@
 """DecodeStep: a decode step bound to fixed buffers and replayed from a CUDA
-graph gives the same bits as the eager calls, including its host copies."""
+graph gives the same bits as the eager calls it stands for (the fused
+decode + up-projection launch for batches up to 64), including its host
+copies."""
 import pytest
 import torch
 
@@ -17,9 +19,9 @@ def _cuda():
 
 
 def _eager(x, q_lat=None):
-    out = b.mlra_decode(q_lat if q_lat is not None else x.q_lat, x.q_rope, x.latent_cache,
-                        x.rope_cache, x.block_table, x.seqlens, x.scale, x.out_scale)
-    return out, b.mlra_up_proj(out, x.w_uv)
+    """The eager step: the fused launch (the batches here are <= 64)."""
+    return b.mlra_decode_up_proj(q_lat if q_lat is not None else x.q_lat, x.q_rope, x.latent_cache,
+                                 x.rope_cache, x.block_table, x.seqlens, x.scale, x.out_scale, x.w_uv)
 
 
 def test_replay_matches_eager_calls():
@@ -32,6 +34,12 @@ def test_replay_matches_eager_calls():
         torch.cuda.synchronize()
         assert torch.equal(y, y_ref)
         assert torch.equal(step.out, out_ref)
+    # the same latent output as mlra_decode, and the same up-projection as
+    # mlra_up_proj of it within the parity tolerance
+    assert torch.equal(out_ref, b.mlra_decode(x.q_lat, x.q_rope, x.latent_cache, x.rope_cache, x.block_table,
+                                              x.seqlens, x.scale, x.out_scale))
+    y2 = b.mlra_up_proj(out_ref, x.w_uv).float()
+    assert ((y.float() - y2).norm() / y2.norm()).item() <= 5e-3
 
 
 def test_host_copies_follow_the_pinned_buffers():
