@@ -451,33 +451,31 @@ __device__ __forceinline__ void merge_tail(const DecodeArgs& a, int n, int cum, 
 // latent output of their head for every sequence (rows padded to a multiple
 // of 16 with zeros) and multiply it on the warp-level tensor cores
 // (m16n8k16, fp32 accumulate) with K split over the warps; the warps' sums
-// meet in shared memory, in warp order.  The weight columns are staged
-// before the wait, transposed so that K is contiguous.
+// meet in shared memory, in warp order.  The weight columns are copied
+// asynchronously before the CTA's merge and waited for after the wait.
 constexpr int kUpMaxBatch = kUpProjFusedMaxBatch;
 
 template <int K>
 struct UpTile {
     static constexpr int KP = K + 8;                       // row stride (bf16): conflict-free fragment reads
-    static constexpr int W_BYTES = 16 * KP * 2;            // the 16 weight columns, [16][KP]
+    static constexpr int W_BYTES = K * 16 * 2;             // the 16 weight columns, [K][16]
     static constexpr int X_BYTES = kUpMaxBatch * KP * 2;   // latent rows, [N padded][KP]
     static constexpr int RED_BYTES = (kThreads / 32) * kUpMaxBatch * 16 * 4;
     static constexpr int BYTES = W_BYTES + X_BYTES + RED_BYTES;
 };
 
-// The CTA's 16 weight columns into wt [16][KP] (at the end of the ring).
+// The CTA's 16 weight columns into wt [K][16] (at the end of the ring), by
+// asynchronous 16-byte copies that land while the merge runs (waited for in
+// up_proj_tail).
 template <int NB, int DC>
 __device__ __forceinline__ void up_stage_weights(const DecodeArgs& a, __nv_bfloat16* wt) {
     constexpr int K = NB * DC;
-    using T = UpTile<K>;
     const int cols = a.heads * a.d_h;
     const int cb = blockIdx.x, h = cb / (a.d_h / 16), j0 = (cb % (a.d_h / 16)) * 16;
     const __nv_bfloat16* src = a.w_uv + (size_t)h * a.d_h + j0;
     for (int e = threadIdx.x; e < 2 * K; e += kThreads) {
         const int k = e >> 1, half = e & 1;
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + (size_t)k * cols) + half);
-        const __nv_bfloat16* v8 = reinterpret_cast<const __nv_bfloat16*>(&v);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) wt[(8 * half + i) * T::KP + k] = v8[i];
+        cp_async16(wt + k * 16 + 8 * half, src + (size_t)k * cols + 8 * half);
     }
 }
 
@@ -509,19 +507,23 @@ __device__ __forceinline__ void up_proj_tail(const DecodeArgs& a, uint8_t* ring,
             record_error(a.err, MLRA_ERR_DEVICE_TIMEOUT);
         }
     }
+    cp_async_wait_all();  // this thread's weight copies (issued before the merge)
     __syncthreads();
     if (*flag & 4) return;
     const int h = blockIdx.x / (a.d_h / 16), j0 = (blockIdx.x % (a.d_h / 16)) * 16;
     const int Np = (N + 15) & ~15;
     __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(ring);
     float* red = reinterpret_cast<float*>(ring + T::X_BYTES);
-    // out[n][h][0..K) for every sequence, 16-byte units (rows past N zero)
+    // out[n][h][0..K) for every sequence: asynchronous 16-byte copies, all
+    // in flight at once (rows past N zero)
     for (int e = tid; e < Np * (K / 8); e += kThreads) {
         const int n = e / (K / 8), u = e % (K / 8);
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (n < N) v = __ldcg(reinterpret_cast<const uint4*>(a.out + ((size_t)n * H + h) * K) + u);
-        *reinterpret_cast<uint4*>(xs + n * T::KP + 8 * u) = v;
+        if (n < N)
+            cp_async16(xs + n * T::KP + 8 * u, a.out + ((size_t)n * H + h) * K + 8 * u);
+        else
+            *reinterpret_cast<uint4*>(xs + n * T::KP + 8 * u) = make_uint4(0u, 0u, 0u, 0u);
     }
+    cp_async_wait_all();
     __syncthreads();
     const int g = lane >> 2, tg = lane & 3;
     float acc[4][2][4];
@@ -533,11 +535,15 @@ __device__ __forceinline__ void up_proj_tail(const DecodeArgs& a, uint8_t* ring,
             for (int i = 0; i < 4; ++i) acc[mt][t][i] = 0.f;
     for (int ks = warp; ks < K / 16; ks += kThreads / 32) {
         const int kb = 16 * ks + 2 * tg;
+        // B (K x 8, column n = output column 8 t + g): rows kb, kb + 1 and
+        // kb + 8, kb + 9 of the [K][16] weight tile, packed in pairs
         uint32_t b[2][2];
+        const uint16_t* wt16 = reinterpret_cast<const uint16_t*>(wt);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-            b[t][0] = *reinterpret_cast<const uint32_t*>(wt + (8 * t + g) * T::KP + kb);
-            b[t][1] = *reinterpret_cast<const uint32_t*>(wt + (8 * t + g) * T::KP + kb + 8);
+            const int col = 8 * t + g;
+            b[t][0] = (uint32_t)wt16[kb * 16 + col] | ((uint32_t)wt16[(kb + 1) * 16 + col] << 16);
+            b[t][1] = (uint32_t)wt16[(kb + 8) * 16 + col] | ((uint32_t)wt16[(kb + 9) * 16 + col] << 16);
         }
 #pragma unroll
         for (int mt = 0; mt < 4; ++mt) {
