@@ -55,7 +55,7 @@ METRIC = "MLRA decode-attention KV GB/s and tokens/s at 1 B200; % of HBM rooflin
 # The other decode workloads whose decode-kernel figures ride along in the
 # line (the step itself is timed on --workload).
 OTHER_WORKLOADS = ["long_context", "ragged", "mla_equal_bytes", "mlra4_equal_bytes", "tp_shard",
-                   "mlra2_equal_bytes", "context_2m"]
+                   "mlra2_equal_bytes", "context_2m", "heads_64"]
 FALLBACK_HBM_GBS = 6650.0
 
 # DRAM traffic of the decode split kernel per launch on decode_2p9b, from one

@@ -36,6 +36,8 @@ mlra_status check_dims(const mlra_dims* d) {
 mlra_status check_tc_coverage(const mlra_dims* d) {
     if (!is_pow2_in(d->page_size, 16, 128)) return MLRA_ERR_UNSUPPORTED;
     if (!decode_tc_supported(d->branches, d->d_c, d->d_r, d->heads)) return MLRA_ERR_UNSUPPORTED;
+    // one block of split counters per head group
+    if ((int64_t)d->batch * tc_head_groups(d->heads) > kMaxBatch) return MLRA_ERR_UNSUPPORTED;
     return MLRA_OK;
 }
 
@@ -193,7 +195,7 @@ mlra_status mlra_decode_up_proj(const mlra_dims* dims, const void* q_lat, const 
     if (s != MLRA_OK) return s;
     if (!aligned16(w_uv)) return MLRA_ERR_INVALID_ARG;
     if (d_h != 64 && d_h != 128) return MLRA_ERR_UNSUPPORTED;
-    if (dims->batch > kUpProjFusedMaxBatch || dims->heads * d_h / 16 > a.num_ctas) return MLRA_ERR_UNSUPPORTED;
+    if (dims->batch > kUpProjFusedMaxBatch) return MLRA_ERR_UNSUPPORTED;
     void* y_dev = const_cast<void*>(device_address(y));  // y may be mapped pinned host memory
     if (y_dev == nullptr || !aligned16(y_dev)) return MLRA_ERR_INVALID_ARG;
     a.w_uv = static_cast<const __nv_bfloat16*>(w_uv);

@@ -22,12 +22,15 @@ constexpr float kLog2e = 1.4426950408889634f;
 // Workspace layout (byte offsets, each region 256-byte aligned):
 //   [0, 256)        int32 error word (first device-side error code, else 0)
 //   split counters  int32 [kMaxBatch + 1]              (fixed place)
-//   lse partials    fp32 [slots][branches][HP]         (log2 domain; HP = 16,
-//                   or the head count when above 16: 64-byte rows)
-//   o partials      fp32 [slots][branches][d_c][16]    (normalised per split;
-//                   heads innermost, padded to 16: one 64-byte row per column)
+//   lse partials    fp32 [slots][branches][HP]         (log2 domain; HP = the
+//                   head count rounded up to a multiple of 16)
+//   o partials      fp32 [slots][branches][d_c][HP]    (normalised per split;
+//                   heads innermost)
 // slots = num_ctas + batch: the partial of CTA c for sequence n lives in slot
-// c + n (unique because CTA ranges are contiguous and ordered).
+// c + n (unique because CTA ranges are contiguous and ordered).  The
+// tensor-core kernel writes rows of 16 heads: with G = HP / 16 head groups,
+// group g owns the G-th part of the bytes, cpg + batch slots of 16-wide rows
+// (cpg = num_ctas / G), and split counters [g batch, (g + 1) batch).
 // ---------------------------------------------------------------------------
 struct WorkspaceLayout {
     size_t err_off, lse_off, o_off, cnt_off, total;
@@ -39,6 +42,10 @@ __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_
 // Largest batch the library accepts (int32 sequence ids, 16-bit grid rows).
 constexpr int kMaxBatch = 65535;
 
+// Heads the tensor-core kernel takes: groups of 16 (its MMA's N), at most 8.
+constexpr int kMaxTcHeads = 128;
+__host__ __device__ inline int tc_head_groups(int heads) { return (heads + 15) / 16; }
+
 __host__ __device__ inline WorkspaceLayout workspace_layout(int batch, int heads, int branches,
                                                             int d_c, int num_ctas) {
     WorkspaceLayout w;
@@ -49,7 +56,7 @@ __host__ __device__ inline WorkspaceLayout workspace_layout(int batch, int heads
     // that reuse the workspace find them where they left them (at zero)
     w.cnt_off = 256;
     w.lse_off = align256(w.cnt_off + sizeof(int) * (size_t)(kMaxBatch + 1));
-    const size_t hp = heads <= 16 ? 16 : (size_t)heads;  // heads padded to 16 (more for the CUDA-core kernel)
+    const size_t hp = 16 * (size_t)tc_head_groups(heads);  // heads padded to a multiple of 16
     w.o_off = align256(w.lse_off + sizeof(float) * (size_t)w.slots * branches * hp);
     w.total = align256(w.o_off + sizeof(float) * (size_t)w.slots * branches * d_c * hp);
     return w;

@@ -122,11 +122,12 @@ mlra_status mlra_decode_static_scratch(const mlra_dims* dims, const void* q_lat,
                                                seqlens, scale, out_scale, out, scratch, kStaticScratchBytes, &a);
     if (s != MLRA_OK) return s;
     // Clear the error word and this call's split counters (the first
-    // 256 + 4 * batch bytes of the workspace layout) before the kernel, so
+    // 256 + 4 * batch * head groups bytes of the workspace layout) before the kernel, so
     // that no earlier call's state -- a stale count left by a kernel that gave
     // up on a bounded wait -- reaches this one.  Stream-ordered, no allocation.
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const size_t clear = reinterpret_cast<char*>(a.seq_cnt + dims->batch) - static_cast<char*>(scratch);
+    const size_t clear = reinterpret_cast<char*>(a.seq_cnt + (size_t)dims->batch * mlra::tc_head_groups(dims->heads)) -
+                         static_cast<char*>(scratch);
     if (cudaMemsetAsync(scratch, 0, clear, st) != cudaSuccess) return MLRA_ERR_CUDA;
     if (mlra::launch_decode_tc(a, st) != cudaSuccess) return MLRA_ERR_CUDA;
     // the error word (offset 0) goes to the caller, stream-ordered

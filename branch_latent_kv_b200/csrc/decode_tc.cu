@@ -10,7 +10,7 @@
 // (abstract of "Multi-Head Low-Rank Attention"), so the kernel streams each
 // token's latent and RoPE row through shared memory exactly once.
 //
-// Organisation (one persistent CTA per SM, 224 threads):
+// Organisation (one persistent CTA per SM, 352 threads):
 //   warp 0     TMA producer: per 128-token tile, the RoPE tile and, per
 //              "pair" of 64-column chunks (128 latent columns), the paged
 //              latent rows (one 2-D box per page) into a ring of stages.
@@ -24,8 +24,10 @@
 //              score MMA and the MN-major A operand of the output MMA).  An
 //              MMA issue stalls the issuing warp for about one MMA's duration,
 //              so two issuers keep the tensor pipe busy while either waits.
-//   warps 2-5  softmax and epilogue: thread t owns token t of the tile (a
-//              TMEM lane); scores are base-2 logits; each (head, branch) has
+//   warps 2-5  softmax and epilogue, heads 0-7, and
+//   warps 7-10 the same for heads 8-15 (two warps per scheduler, so that
+//              each hides the other's latency): a thread owns one token of
+//              the tile (a TMEM lane); scores are base-2 logits; each (head, branch) has
 //              its own running max, rescaled only when a score exceeds it by
 //              more than 2^8 (then the exact column max is reduced and the
 //              TMEM accumulator is rescaled); P is written as bf16 to shared
@@ -48,8 +50,9 @@ namespace {
 using namespace sm100;
 
 constexpr int kHP = 16;             // heads padded to the MMA N
+constexpr int kHG = kHP / 2;        // heads of one softmax group
 constexpr int kT = kTileTokens;     // tokens per tile = MMA M
-constexpr int kThreads = 224;
+constexpr int kThreads = 352;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kSmemLimit = 232448;  // max dynamic shared memory per CTA on sm_100
 
@@ -156,6 +159,36 @@ struct Maps {
     CUtensorMap qr;    // q_rope [batch][H][d_r]
 };
 
+// Head groups.  The MMAs take 16 heads (N = 16); H > 16 heads run as
+// ceil(H / 16) groups side by side.  CTA g * cpg + i (cpg = grid / groups)
+// runs window i of one cost plan over cpg windows for heads
+// [16 g, 16 g + 16), so the groups stream the same tokens at about the same
+// time and every read of a cache line after the first hits L2 (the latents
+// are shared by all heads).  Each group has its own partial slots (a block
+// of cpg + batch) and split counters (a block of batch); CTAs past
+// groups * cpg only take part in the fused up-projection.
+struct HeadGroup {
+    int ci, cpg;   // window of this CTA, windows (CTAs) per group
+    int h0, hn;    // first head of the group, heads in it
+    int slot0;     // first partial slot of the group
+    int cnt0;      // first split counter of the group
+    bool idle;     // no group: beyond groups * cpg
+};
+
+__device__ __forceinline__ HeadGroup head_group(const DecodeArgs& a) {
+    HeadGroup hg;
+    const int groups = tc_head_groups(a.heads);
+    hg.cpg = a.num_ctas / groups;
+    const int g = (int)blockIdx.x / hg.cpg;
+    hg.ci = (int)blockIdx.x - g * hg.cpg;
+    hg.idle = g >= groups;
+    hg.h0 = g * kHP;
+    hg.hn = hg.idle ? 0 : min(kHP, a.heads - hg.h0);
+    hg.slot0 = g * (hg.cpg + a.batch);
+    hg.cnt0 = g * a.batch;
+    return hg;
+}
+
 // 2^x on the special-function unit (ex2.approx, flush-to-zero: results below
 // 2^-126 become 0, which only affects probabilities that are negligible).
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -164,31 +197,26 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return y;
 }
 
-// Max over the 32 lanes of a warp of each of 16 values, reduce-scattered:
-// the result for column c ends up in lanes 2c and 2c+1.  16 shuffles.
-__device__ __forceinline__ float warp_colmax16(const float (&v)[16], int lane) {
-    float a8[8], a4[4], a2[2];
+// Max over the 32 lanes of a warp of each of 8 values, reduce-scattered:
+// the result for column c ends up in lanes 4c..4c+3.  9 shuffles.
+__device__ __forceinline__ float warp_colmax8(const float (&v)[8], int lane) {
+    float a4[4], a2[2];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {  // lanes with bit 4 keep columns 8..15
+    for (int i = 0; i < 4; ++i) {  // lanes with bit 4 keep columns 4..7
         const bool hi = lane & 16;
-        const float keep = hi ? v[i + 8] : v[i], send = hi ? v[i] : v[i + 8];
-        a8[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 16));
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const bool hi = lane & 8;
-        const float keep = hi ? a8[i + 4] : a8[i], send = hi ? a8[i] : a8[i + 4];
-        a4[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+        const float keep = hi ? v[i + 4] : v[i], send = hi ? v[i] : v[i + 4];
+        a4[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 16));
     }
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-        const bool hi = lane & 4;
+        const bool hi = lane & 8;
         const float keep = hi ? a4[i + 2] : a4[i], send = hi ? a4[i] : a4[i + 2];
-        a2[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+        a2[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 8));
     }
-    const bool hi = lane & 2;
+    const bool hi = lane & 4;
     const float keep = hi ? a2[1] : a2[0], send = hi ? a2[0] : a2[1];
-    const float a1 = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
+    float a1 = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+    a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 2));
     return fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
 }
 
@@ -268,14 +296,15 @@ __device__ __forceinline__ int next_range_seq(const DecodeArgs& a, int n, int cu
     return -1;
 }
 
-// One sequence's queries (latent and RoPE, 16 head rows each) into the
-// query buffer, completing `full`; issued by one thread.
+// One sequence's queries (latent and RoPE, the 16 head rows from h0; rows
+// past the last head read as zero) into the query buffer, completing `full`;
+// issued by one thread.
 template <class C>
-__device__ __forceinline__ void load_queries(const Maps& maps, uint8_t* sm, uint64_t& full, int seq) {
+__device__ __forceinline__ void load_queries(const Maps& maps, uint8_t* sm, uint64_t& full, int seq, int h0) {
     uint8_t* qd = sm + C::OFF_Q;
     mbar_arrive_expect_tx(&full, C::Q_BYTES + C::QR_BYTES);
-    for (int c = 0; c < C::NCHUNK; ++c) tma_load_3d(qd + c * C::Q_CHUNK_BYTES, &maps.q, c * 64, 0, seq, &full);
-    tma_load_3d(qd + C::Q_BYTES, &maps.qr, 0, 0, seq, &full);
+    for (int c = 0; c < C::NCHUNK; ++c) tma_load_3d(qd + c * C::Q_CHUNK_BYTES, &maps.q, c * 64, h0, seq, &full);
+    tma_load_3d(qd + C::Q_BYTES, &maps.qr, 0, h0, seq, &full);
 }
 
 // End of the kernel, all threads: the merge of split sequences.
@@ -295,8 +324,8 @@ __device__ __forceinline__ void load_queries(const Maps& maps, uint8_t* sm, uint
 // is laid out for latency: every thread loads its values for up to 8 splits
 // at once before combining them.
 template <int NB, int DC>
-__device__ __forceinline__ void merge_tail(const DecodeArgs& a, int n, int cum, int tiles, bool c1_member,
-                                           int chunk, float* w_s, int* flag, uint64_t* bar) {
+__device__ __forceinline__ void merge_tail(const DecodeArgs& a, const HeadGroup& grp, int n, int cum, int tiles,
+                                           bool c1_member, int chunk, float* w_s, int* flag, uint64_t* bar) {
     constexpr int HB = NB * kHP;  // (branch, head) columns of a split's log-sum-exp row
     constexpr int R = NB * DC;    // (branch, latent column) rows
     const int tid = threadIdx.x;
@@ -310,15 +339,17 @@ __device__ __forceinline__ void merge_tail(const DecodeArgs& a, int n, int cum, 
     // c1 belongs to the group when no later tile is its own (the next valid
     // sequence starts in a later window); worked out at the range's start
     const int G = c1_member ? S : S - 1;
-    const int gi = blockIdx.x - c0;  // 0 <= gi < G: n is this CTA's last sequence
+    const int gi = grp.ci - c0;  // 0 <= gi < G: n is this CTA's last sequence
     const int r0 = (int)((long long)gi * R / G), r1 = (int)((long long)(gi + 1) * R / G);
     const int rows = r1 - r0;
+    const size_t slot_c0 = (size_t)grp.slot0 + c0 + n;  // the partial slot of split 0
+    int* cnt = a.seq_cnt + grp.cnt0 + n;
     float* part_s = w_s + S * HB;  // [S][rows][16 heads]
     // wait until every split of n has counted its partials
     if (tid == 0) {
         const uint64_t t0 = globaltimer_ns();
         bool ok = true;
-        while (ld_acquire_gpu(a.seq_cnt + n) < S) {
+        while (ld_acquire_gpu(cnt) < S) {
             if (globaltimer_ns() - t0 > 2000000000ull) {
                 ok = false;
                 break;
@@ -340,15 +371,15 @@ __device__ __forceinline__ void merge_tail(const DecodeArgs& a, int n, int cum, 
         fence_proxy_async_global();
         if (tid == 0) {
             mbar_arrive_expect_tx(bar, (uint32_t)(S * HB + S * rows * kHP) * 4u);
-            bulk_load(w_s, a.lse_part + (size_t)(c0 + n) * HB, (uint32_t)(S * HB) * 4u, bar);
+            bulk_load(w_s, a.lse_part + slot_c0 * HB, (uint32_t)(S * HB) * 4u, bar);
         }
         __syncwarp();
         if (rows > 0)
             for (int sp = tid; sp < S; sp += 32)
-                bulk_load(part_s + (size_t)sp * rows * kHP, a.o_part + ((size_t)(c0 + n + sp) * R + r0) * kHP,
+                bulk_load(part_s + (size_t)sp * rows * kHP, a.o_part + ((slot_c0 + sp) * R + r0) * kHP,
                           (uint32_t)rows * kHP * 4u, bar);
         // this CTA leaves the count (its result is needed only at the end)
-        if (tid == 0) departed = atomicAdd(a.seq_cnt + n, 1);
+        if (tid == 0) departed = atomicAdd(cnt, 1);
     }
     if (!mbar_wait(bar, 0)) {
         // never expected: report it, and give the copies a last bounded
@@ -397,7 +428,7 @@ __device__ __forceinline__ void merge_tail(const DecodeArgs& a, int n, int cum, 
             for (int j = 0; j < 8; ++j)
                 if (s0 + 2 * j < S) w_s[(s0 + 2 * j) * HB + col] *= norm;
         }
-        if (bad && half == 0 && col % kHP < H) atomicOr(flag, 1);
+        if (bad && half == 0 && col % kHP < grp.hn) atomicOr(flag, 1);
     }
     __syncthreads();
     const bool bad = *flag & 1;
@@ -429,18 +460,19 @@ __device__ __forceinline__ void merge_tail(const DecodeArgs& a, int n, int cum, 
             }
         }
         if (bad) acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        __nv_bfloat16* dst = a.out + ((size_t)n * H * NB + b) * DC + k;
+        __nv_bfloat16* dst = a.out + (((size_t)n * H + grp.h0) * NB + b) * DC + k;
         const float v4[4] = {acc.x, acc.y, acc.z, acc.w};
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-            if (4 * q + j < H) dst[(size_t)(4 * q + j) * NB * DC] = to_bf16(v4[j]);
+            if (4 * q + j < grp.hn) dst[(size_t)(4 * q + j) * NB * DC] = to_bf16(v4[j]);
     }
-    if (tid == 0 && departed == S + G - 1) a.seq_cnt[n] = 0;
+    if (tid == 0 && departed == S + G - 1) *cnt = 0;
 }
 
 // ------------------------------------------------------------------ fused up-projection
-// The fused step (mlra_decode_up_proj): after the launch's merges, CTA c below
-// H d_h / 16 computes the 16 output columns [16 c, 16 c + 16) of
+// The fused step (mlra_decode_up_proj): after the launch's merges, CTA c
+// computes the 16 output columns [16 cb, 16 cb + 16) of each column block
+// cb = c, c + grid, ... below H d_h / 16 of
 //   y[n, h d_h + j] = sum_b sum_k out[n, h, b, k] W_UV[b][k][h d_h + j]
 // for every sequence n: the per-branch up-projection summed over the
 // branches is one K = B d_c reduction ("The Core Insight" section of the
@@ -448,11 +480,13 @@ __device__ __forceinline__ void merge_tail(const DecodeArgs& a, int n, int cum, 
 // the branch outputs are summed).  Every CTA counts itself into a grid
 // counter once its merge duty is done (the spare word after the split
 // counters); the up-projection CTAs wait (bounded) for all of them, read the
-// latent output of their head for every sequence (rows padded to a multiple
-// of 16 with zeros) and multiply it on the warp-level tensor cores
+// latent output of the block's head for every sequence (rows padded to a
+// multiple of 16 with zeros) and multiply it on the warp-level tensor cores
 // (m16n8k16, fp32 accumulate) with K split over the warps; the warps' sums
-// meet in shared memory, in warp order.  The weight columns are copied
-// asynchronously before the CTA's merge and waited for after the wait.
+// meet in shared memory, in warp order.  The first block's weight columns are
+// copied asynchronously before the CTA's merge and waited for after the wait
+// (a further block's, when there are more blocks than CTAs, after the block
+// before it).
 constexpr int kUpMaxBatch = kUpProjFusedMaxBatch;
 
 template <int K>
@@ -468,10 +502,10 @@ struct UpTile {
 // asynchronous 16-byte copies that land while the merge runs (waited for in
 // up_proj_tail).
 template <int NB, int DC>
-__device__ __forceinline__ void up_stage_weights(const DecodeArgs& a, __nv_bfloat16* wt) {
+__device__ __forceinline__ void up_stage_weights(const DecodeArgs& a, __nv_bfloat16* wt, int cb) {
     constexpr int K = NB * DC;
     const int cols = a.heads * a.d_h;
-    const int cb = blockIdx.x, h = cb / (a.d_h / 16), j0 = (cb % (a.d_h / 16)) * 16;
+    const int h = cb / (a.d_h / 16), j0 = (cb % (a.d_h / 16)) * 16;
     const __nv_bfloat16* src = a.w_uv + (size_t)h * a.d_h + j0;
     for (int e = threadIdx.x; e < 2 * K; e += kThreads) {
         const int k = e >> 1, half = e & 1;
@@ -485,11 +519,11 @@ __device__ __forceinline__ void up_proj_tail(const DecodeArgs& a, uint8_t* ring,
     using T = UpTile<K>;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int N = a.batch, H = a.heads, ncb = H * a.d_h / 16;
-    const bool worker = (int)blockIdx.x < ncb;
+    const int workers = ncb < a.num_ctas ? ncb : a.num_ctas;
     int* gcnt = a.seq_cnt + kMaxBatch;
     __syncthreads();  // the CTA's merge is done (and its weight columns staged)
     if (tid == 0) red_add_release_gpu(gcnt, 1);
-    if (!worker) return;
+    if ((int)blockIdx.x >= ncb) return;
     int departed = 0;
     if (tid == 0) {
         const uint64_t t0 = globaltimer_ns();
@@ -507,78 +541,86 @@ __device__ __forceinline__ void up_proj_tail(const DecodeArgs& a, uint8_t* ring,
             record_error(a.err, MLRA_ERR_DEVICE_TIMEOUT);
         }
     }
-    cp_async_wait_all();  // this thread's weight copies (issued before the merge)
-    __syncthreads();
-    if (*flag & 4) return;
-    const int h = blockIdx.x / (a.d_h / 16), j0 = (blockIdx.x % (a.d_h / 16)) * 16;
     const int Np = (N + 15) & ~15;
     __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(ring);
     float* red = reinterpret_cast<float*>(ring + T::X_BYTES);
-    // out[n][h][0..K) for every sequence: asynchronous 16-byte copies, all
-    // in flight at once (rows past N zero)
-    for (int e = tid; e < Np * (K / 8); e += kThreads) {
-        const int n = e / (K / 8), u = e % (K / 8);
-        if (n < N)
-            cp_async16(xs + n * T::KP + 8 * u, a.out + ((size_t)n * H + h) * K + 8 * u);
-        else
-            *reinterpret_cast<uint4*>(xs + n * T::KP + 8 * u) = make_uint4(0u, 0u, 0u, 0u);
-    }
-    cp_async_wait_all();
-    __syncthreads();
-    const int g = lane >> 2, tg = lane & 3;
-    float acc[4][2][4];
-#pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[mt][t][i] = 0.f;
-    for (int ks = warp; ks < K / 16; ks += kThreads / 32) {
-        const int kb = 16 * ks + 2 * tg;
-        // B (K x 8, column n = output column 8 t + g): rows kb, kb + 1 and
-        // kb + 8, kb + 9 of the [K][16] weight tile, packed in pairs
-        uint32_t b[2][2];
-        const uint16_t* wt16 = reinterpret_cast<const uint16_t*>(wt);
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            const int col = 8 * t + g;
-            b[t][0] = (uint32_t)wt16[kb * 16 + col] | ((uint32_t)wt16[(kb + 1) * 16 + col] << 16);
-            b[t][1] = (uint32_t)wt16[(kb + 8) * 16 + col] | ((uint32_t)wt16[(kb + 9) * 16 + col] << 16);
+    for (int cb = blockIdx.x; cb < ncb; cb += a.num_ctas) {
+        if (cb != (int)blockIdx.x) {
+            __syncthreads();  // the block before is done with wt, xs and red
+            up_stage_weights<NB, DC>(a, wt, cb);
         }
+        const int h = cb / (a.d_h / 16), j0 = (cb % (a.d_h / 16)) * 16;
+        if (cb == (int)blockIdx.x) {
+            cp_async_wait_all();  // this thread's weight copies (issued before the merge)
+            __syncthreads();
+            if (*flag & 4) return;
+        }
+        // out[n][h][0..K) for every sequence: asynchronous 16-byte copies, all
+        // in flight at once (rows past N zero)
+        for (int e = tid; e < Np * (K / 8); e += kThreads) {
+            const int n = e / (K / 8), u = e % (K / 8);
+            if (n < N)
+                cp_async16(xs + n * T::KP + 8 * u, a.out + ((size_t)n * H + h) * K + 8 * u);
+            else
+                *reinterpret_cast<uint4*>(xs + n * T::KP + 8 * u) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        cp_async_wait_all();
+        __syncthreads();
+        const int g = lane >> 2, tg = lane & 3;
+        float acc[4][2][4];
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[mt][t][i] = 0.f;
+        for (int ks = warp; ks < K / 16; ks += kThreads / 32) {
+            const int kb = 16 * ks + 2 * tg;
+            // B (K x 8, column n = output column 8 t + g): rows kb, kb + 1 and
+            // kb + 8, kb + 9 of the [K][16] weight tile, packed in pairs
+            uint32_t bf[2][2];
+            const uint16_t* wt16 = reinterpret_cast<const uint16_t*>(wt);
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const int col = 8 * t + g;
+                bf[t][0] = (uint32_t)wt16[kb * 16 + col] | ((uint32_t)wt16[(kb + 1) * 16 + col] << 16);
+                bf[t][1] = (uint32_t)wt16[(kb + 8) * 16 + col] | ((uint32_t)wt16[(kb + 9) * 16 + col] << 16);
+            }
+#pragma unroll
+            for (int mt = 0; mt < 4; ++mt) {
+                if (16 * mt >= Np) break;
+                const __nv_bfloat16* x0 = xs + (16 * mt + g) * T::KP + kb;
+                const uint32_t af[4] = {*reinterpret_cast<const uint32_t*>(x0),
+                                        *reinterpret_cast<const uint32_t*>(x0 + 8 * T::KP),
+                                        *reinterpret_cast<const uint32_t*>(x0 + 8),
+                                        *reinterpret_cast<const uint32_t*>(x0 + 8 * T::KP + 8)};
+#pragma unroll
+                for (int t = 0; t < 2; ++t) mma_m16n8k16_bf16(acc[mt][t], af, bf[t][0], bf[t][1]);
+            }
+        }
+        // the warps' partial sums: red[warp][row][16 columns]
 #pragma unroll
         for (int mt = 0; mt < 4; ++mt) {
             if (16 * mt >= Np) break;
-            const __nv_bfloat16* x0 = xs + (16 * mt + g) * T::KP + kb;
-            const uint32_t af[4] = {*reinterpret_cast<const uint32_t*>(x0),
-                                    *reinterpret_cast<const uint32_t*>(x0 + 8 * T::KP),
-                                    *reinterpret_cast<const uint32_t*>(x0 + 8),
-                                    *reinterpret_cast<const uint32_t*>(x0 + 8 * T::KP + 8)};
 #pragma unroll
-            for (int t = 0; t < 2; ++t) mma_m16n8k16_bf16(acc[mt][t], af, b[t][0], b[t][1]);
+            for (int t = 0; t < 2; ++t) {
+                float* r = red + ((size_t)warp * kUpMaxBatch + 16 * mt + g) * 16 + 8 * t + 2 * tg;
+                r[0] = acc[mt][t][0];
+                r[1] = acc[mt][t][1];
+                r[8 * 16] = acc[mt][t][2];
+                r[8 * 16 + 1] = acc[mt][t][3];
+            }
+        }
+        __syncthreads();
+        for (int e = tid; e < N * 16; e += kThreads) {
+            const int n = e >> 4, j = e & 15;
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < kThreads / 32; ++w) v += red[((size_t)w * kUpMaxBatch + n) * 16 + j];
+            a.y[(size_t)n * H * a.d_h + h * a.d_h + j0 + j] = to_bf16(v);
         }
     }
-    // the warps' partial sums: red[warp][row][16 columns]
-#pragma unroll
-    for (int mt = 0; mt < 4; ++mt) {
-        if (16 * mt >= Np) break;
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            float* r = red + ((size_t)warp * kUpMaxBatch + 16 * mt + g) * 16 + 8 * t + 2 * tg;
-            r[0] = acc[mt][t][0];
-            r[1] = acc[mt][t][1];
-            r[8 * 16] = acc[mt][t][2];
-            r[8 * 16 + 1] = acc[mt][t][3];
-        }
-    }
-    __syncthreads();
-    for (int e = tid; e < N * 16; e += kThreads) {
-        const int n = e >> 4, j = e & 15;
-        float v = 0.f;
-#pragma unroll
-        for (int w = 0; w < kThreads / 32; ++w) v += red[((size_t)w * kUpMaxBatch + n) * 16 + j];
-        a.y[(size_t)n * H * a.d_h + h * a.d_h + j0 + j] = to_bf16(v);
-    }
-    if (tid == 0 && departed == a.num_ctas + ncb - 1) *gcnt = 0;
+    if (tid == 0 && departed == a.num_ctas + workers - 1) *gcnt = 0;
 }
 
 template <int NB, int DC, int DR>
@@ -592,6 +634,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
     M& misc = *reinterpret_cast<M*>(sm + C::OFF_MISC);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int P = a.page_size;
+    const HeadGroup grp = head_group(a);
 
     if (warp == 0 && lane < 4) {
         // descriptor fetches overlap the set-up below
@@ -610,7 +653,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
         mbar_init(&misc.drain[1], 1);
         for (int i = 0; i < C::NSP; ++i) {
             mbar_init(&misc.s_full[i], 1);
-            mbar_init(&misc.p_full[i], 4);
+            mbar_init(&misc.p_full[i], 8);  // the eight softmax warps
             mbar_init(&misc.p_empty[i], 1);
         }
         mbar_init(&misc.q_full, 1);
@@ -629,11 +672,11 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
         // the inputs may come from the preceding kernel (programmatic launch)
         wait_prerequisite_grid();
         const int total = warp_cost_prefix(a.seqlens, a.batch, P, a.max_pages);
-        const int chunk = plan_chunk(total, a.num_ctas);
+        const int chunk = plan_chunk(total, grp.cpg);
         n_first = a.batch;
         cum_first = total;
-        if ((long long)blockIdx.x * chunk < total)
-            warp_find_seq(a.seqlens, a.batch, P, a.max_pages, blockIdx.x * chunk, &n_first, &cum_first);
+        if (!grp.idle && (long long)grp.ci * chunk < total)
+            warp_find_seq(a.seqlens, a.batch, P, a.max_pages, grp.ci * chunk, &n_first, &cum_first);
         if (lane == 0) {
             misc.plan[1] = chunk;
             misc.plan[2] = n_first;
@@ -665,7 +708,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
         }
     }
     const int chunk = misc.plan[1];
-    const int A0 = blockIdx.x * chunk, A1 = A0 + chunk;  // this CTA's cost window
+    const int A0 = grp.ci * chunk, A1 = A0 + chunk;  // this CTA's cost window
     const uint32_t tmem = misc.tmem_base;                // (warp 0 never uses it)
     volatile int* abort_flag = &misc.abort_flag;
 
@@ -676,14 +719,16 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
             int L, tiles, tb, te;
             uint32_t pc = 0, tc = 0, sc = 0;
             // the cache is read once per step: its lines go first, and the
-            // block table, lengths, queries and partials stay in L2
-            const uint64_t stream_policy = l2_policy_evict_first();
+            // block table, lengths, queries and partials stay in L2 (with
+            // head groups every line is read once per group, at about the
+            // same time: normal priority)
+            const uint64_t stream_policy = grp.cpg == a.num_ctas ? l2_policy_evict_first() : l2_policy_evict_normal();
             bool ok = true;
             while (ok && next_segment(a, n, cum, A0, A1, L, tiles, tb, te, next_len)) {
                 // the first range's queries; a later range's are loaded by the
                 // score MMA warp once the range before has its last scores, so
                 // the copies of the cache never wait for the query buffer
-                if (lane == 0 && sc == 0) load_queries<C>(maps, sm, misc.q_full, n);
+                if (lane == 0 && sc == 0) load_queries<C>(maps, sm, misc.q_full, n, grp.h0);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 ++sc;
@@ -846,7 +891,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                     __syncwarp();
                     ok = mbar_wait_warp(&misc.q_empty, qe & 1);
                     ++qe;
-                    if (ok && elect_one()) load_queries<C>(maps, sm, misc.q_full, nn);
+                    if (ok && elect_one()) load_queries<C>(maps, sm, misc.q_full, nn, grp.h0);
                     __syncwarp();
                 }
                 ++sc;
@@ -921,9 +966,19 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
             __syncwarp();
         } else {
             // ------------------------------------------------------------ softmax + epilogue
-            const int quad = warp & 3;                 // TMEM lane quadrant of this warp
-            const int row = quad * 32 + lane;          // token (S) / latent row (O)
-            const int stid = threadIdx.x - 64;         // 0..127 within the group
+            // Two groups of four warps (warps 2-5 and 7-10), one warp of each
+            // per TMEM lane quadrant: group sg owns heads [8 sg, 8 sg + 8) of
+            // every score and output column block.  The groups share no
+            // running max, denominator or rescale (those are per head); they
+            // meet only in a P slot (each writes its 8 heads of a token's row
+            // and arrives on p_full) and at the kernel's end.  Two warps per
+            // scheduler hide each other's latency chains.
+            const int sg = warp >= 7;                        // softmax group
+            const int hoff = kHG * sg;                       // its first head column
+            const uint32_t gbar = 3 + sg;                    // its named barrier (128 threads)
+            const int quad = warp & 3;                       // TMEM lane quadrant of this warp
+            const int row = quad * 32 + lane;                // token (S) / latent row (O)
+            const int stid = (warp - (sg ? 7 : 2)) * 32 + lane;  // 0..127 within the group
             const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
             const int H = a.heads;
             int n = n_first, cum = cum_first, next_len = first_len(a, n);
@@ -932,7 +987,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
             // This thread's share of the softmax denominators, one row per
             // branch.  The step loop is not unrolled: after each step the rows
             // rotate by G so that the current step's branches are rows 0..G-1.
-            float l[NB][kHP];
+            float l[NB][kHG];
             bool dead = false;
             int pend_a = -1, pend_b = -1;  // split ranges not yet counted (thread stid 0)
 
@@ -946,7 +1001,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                 // this sequence's last tile also merges it (no later sequence
                 // starts in its window); worked out now, off the critical path
                 int c1_member = 1;
-                if (stid == 0) {
+                if (sg == 0 && stid == 0) {
                     const int c1 = (cum + (tiles - 1) * kTileCost) / chunk;
                     for (int m = n + 1; m < a.batch; ++m) {
                         if (seq_tiles(__ldg(a.seqlens + m), a.page_size, a.max_pages) == 0) continue;
@@ -957,31 +1012,31 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
 #pragma unroll
                 for (int b = 0; b < NB; ++b)
 #pragma unroll
-                    for (int i = 0; i < kHP; ++i) l[b][i] = 0.f;
+                    for (int i = 0; i < kHG; ++i) l[b][i] = 0.f;
 
                 for (int j = tb; j < te && !dead; ++j) {
                     const int valid = min(kT, L - j * kT);
                     const bool masked = row >= valid;
                     const int page = masked ? 0 : __ldg(bt + (j * kT + row) / P);
-                    float r[kHP];  // this token's RoPE score per head, shared by the tile's branches
+                    float r[kHG];  // this token's RoPE score per head, shared by the tile's branches
 #pragma unroll 1
                     for (int st = 0; st < C::NSTEP; ++st) {
                         const uint32_t slot = gs % C::NSP;
                         const bool ok = mbar_wait(&misc.s_full[slot], (gs / C::NSP) & 1);
                         tc_fence_after();
 
-                        float x[C::SBR][kHP];
-                        if (st == 0) tmem_ld16(tmem + lane_off + C::R_COL0 + (tcnt % C::NRS) * kHP, r);
+                        float x[C::SBR][kHG];
+                        if (st == 0) tmem_ld8(tmem + lane_off + C::R_COL0 + (tcnt % C::NRS) * kHP + hoff, r);
 #pragma unroll
                         for (int g = 0; g < C::SBR; ++g)
-                            tmem_ld16(tmem + lane_off + C::S_COL0 + slot * C::S_SLOT_COLS + g * kHP, x[g]);
+                            tmem_ld8(tmem + lane_off + C::S_COL0 + slot * C::S_SLOT_COLS + g * kHP + hoff, x[g]);
                         tmem_wait_ld();
 #pragma unroll
                         for (int g = 0; g < C::SBR; ++g)
 #pragma unroll
-                            for (int i = 0; i < kHP; ++i)
+                            for (int i = 0; i < kHG; ++i)
                                 x[g][i] = masked ? -INFINITY : (x[g][i] + r[i]) * a.scale_log2;
-                        float* m_step = &misc.m_run[st * C::SBR * kHP];
+                        float* m_step = &misc.m_run[st * C::SBR * kHP + hoff];  // [g * kHP + i]
                         if (j == tb) {
                             // first tile of the range: token 0 (always valid) sets the
                             // reference maxima; larger scores take the exact path below
@@ -989,15 +1044,15 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
 #pragma unroll
                                 for (int g = 0; g < C::SBR; ++g)
 #pragma unroll
-                                    for (int i = 0; i < kHP; ++i) m_step[g * kHP + i] = x[g][i];
+                                    for (int i = 0; i < kHG; ++i) m_step[g * kHP + i] = x[g][i];
                             }
-                            named_bar_sync<1, 128>();
+                            named_bar_sync_id<128>(gbar);
                         }
-                        float m[C::SBR][kHP];
+                        float m[C::SBR][kHG];
 #pragma unroll
                         for (int g = 0; g < C::SBR; ++g)
 #pragma unroll
-                            for (int i = 0; i < kHP; i += 4) {
+                            for (int i = 0; i < kHG; i += 4) {
                                 const float4 v = *reinterpret_cast<const float4*>(m_step + g * kHP + i);
                                 m[g][i] = v.x;
                                 m[g][i + 1] = v.y;
@@ -1008,27 +1063,28 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
 #pragma unroll
                         for (int g = 0; g < C::SBR; ++g)
 #pragma unroll
-                            for (int i = 0; i < kHP; ++i) need |= x[g][i] > m[g][i] + kRescaleLog2;
-                        if (named_bar_or<1, 128>(need || !ok)) {
-                            if (named_bar_or<1, 128>(!ok)) {
+                            for (int i = 0; i < kHG; ++i) need |= x[g][i] > m[g][i] + kRescaleLog2;
+                        if (named_bar_or_id<128>(gbar, need || !ok)) {
+                            if (named_bar_or_id<128>(gbar, !ok)) {
                                 dead = true;
                                 break;
                             }
                             // exact column max over the tile's 128 tokens: a warp
-                            // reduce-scatter leaves column (lane >> 1) in each lane
+                            // reduce-scatter leaves column (lane >> 2) in each lane
 #pragma unroll
                             for (int g = 0; g < C::SBR; ++g) {
-                                const float v = warp_colmax16(x[g], lane);
-                                if ((lane & 1) == 0) misc.red_max[quad][g * kHP + (lane >> 1)] = v;
+                                const float v = warp_colmax8(x[g], lane);
+                                if ((lane & 3) == 0) misc.red_max[quad][g * kHP + hoff + (lane >> 2)] = v;
                             }
-                            named_bar_sync<1, 128>();
-                            float alpha[C::SBR][kHP];
+                            named_bar_sync_id<128>(gbar);
+                            float alpha[C::SBR][kHG];
 #pragma unroll
                             for (int g = 0; g < C::SBR; ++g)
 #pragma unroll
-                                for (int i = 0; i < kHP; ++i) {
-                                    const float tmax = fmaxf(fmaxf(misc.red_max[0][g * kHP + i], misc.red_max[1][g * kHP + i]),
-                                                             fmaxf(misc.red_max[2][g * kHP + i], misc.red_max[3][g * kHP + i]));
+                                for (int i = 0; i < kHG; ++i) {
+                                    const int c = g * kHP + hoff + i;
+                                    const float tmax = fmaxf(fmaxf(misc.red_max[0][c], misc.red_max[1][c]),
+                                                             fmaxf(misc.red_max[2][c], misc.red_max[3][c]));
                                     const float mnew = fmaxf(m[g][i], tmax);
                                     alpha[g][i] = fast_exp2(m[g][i] - mnew);
                                     m[g][i] = mnew;
@@ -1040,14 +1096,14 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
 #pragma unroll
                                 for (int g = 0; g < C::SBR; ++g)
 #pragma unroll
-                                    for (int i = 0; i < kHP; ++i) m_step[g * kHP + i] = m[g][i];
+                                    for (int i = 0; i < kHG; ++i) m_step[g * kHP + i] = m[g][i];
                             }
-                            named_bar_sync<1, 128>();
+                            named_bar_sync_id<128>(gbar);
                             if (j > tb) {
-                                // O holds earlier tiles of this range: rescale it once the
-                                // previous output MMA has finished
+                                // O holds earlier tiles of this range: rescale this
+                                // group's columns once the previous output MMA has finished
                                 const bool ok2 = mbar_wait(&misc.p_empty[(gs - 1) % C::NSP], ((gs - 1) / C::NSP) & 1);
-                                if (named_bar_or<1, 128>(!ok2)) {
+                                if (named_bar_or_id<128>(gbar, !ok2)) {
                                     dead = true;
                                     break;
                                 }
@@ -1057,24 +1113,25 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
 #pragma unroll
                                     for (int g2 = 0; g2 < C::BPP; ++g2) {
                                         const int gl = DC >= 128 ? p * 128 / DC : p * C::BPP + g2;
-                                        const uint32_t col = ((st * C::PPS + p) * C::BPP + g2) * kHP;
-                                        float o[kHP];
-                                        tmem_ld16(tmem + lane_off + col, o);
+                                        const uint32_t col = ((st * C::PPS + p) * C::BPP + g2) * kHP + hoff;
+                                        float o[kHG];
+                                        tmem_ld8(tmem + lane_off + col, o);
                                         tmem_wait_ld();
 #pragma unroll
-                                        for (int i = 0; i < kHP; ++i) o[i] *= alpha[gl][i];
-                                        tmem_st16(tmem + lane_off + col, o);
+                                        for (int i = 0; i < kHG; ++i) o[i] *= alpha[gl][i];
+                                        tmem_st8(tmem + lane_off + col, o);
                                     }
                                 tmem_wait_st();
                             }
                         }
-                        // probabilities -> bf16 P (MN-major, 8x8 core matrices)
+                        // probabilities -> bf16 P (MN-major, 8x8 core matrices; this
+                        // group's 8 heads are the core matrix at + 2048 sg)
                         uint8_t* p_slot = sm + C::OFF_P + slot * C::P_BYTES;
 #pragma unroll
                         for (int g = 0; g < C::SBR; ++g) {
-                            uint32_t packed[kHP / 2];
+                            uint32_t packed[kHG / 2];
 #pragma unroll
-                            for (int i = 0; i < kHP; i += 2) {
+                            for (int i = 0; i < kHG; i += 2) {
                                 const float p0 = fast_exp2(x[g][i] - m[g][i]);
                                 const float p1 = fast_exp2(x[g][i + 1] - m[g][i + 1]);
                                 l[g][i] += p0;
@@ -1082,22 +1139,20 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                                 __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
                                 packed[i / 2] = *reinterpret_cast<uint32_t*>(&pr);
                             }
-                            uint8_t* dst = p_slot + g * C::P_BRANCH_BYTES + (row >> 3) * 128 + (row & 7) * 16;
+                            uint8_t* dst = p_slot + g * C::P_BRANCH_BYTES + (row >> 3) * 128 + (row & 7) * 16 + sg * 2048;
                             *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                            *reinterpret_cast<uint4*>(dst + 2048) = make_uint4(packed[4], packed[5], packed[6], packed[7]);
                         }
                         // rows past the end of the sequence (stale or poisoned data)
-                        // become zero before the output MMA reads them
+                        // become zero before the output MMA reads them: this group
+                        // clears chunk sg of each of the step's pairs
                         if (masked) {
 #pragma unroll
                             for (int p = 0; p < C::PPS; ++p) {
                                 uint8_t* pair = sm + C::OFF_PAIR + ((gs * C::PPS + p) % C::NSTAGE) * C::PAIR_BYTES;
 #pragma unroll
-                                for (int h2 = 0; h2 < 2; ++h2)
-#pragma unroll
-                                    for (int u = 0; u < 8; ++u)
-                                        *reinterpret_cast<uint4*>(pair + h2 * C::CHUNK_BYTES + row * 128 + u * 16) =
-                                            make_uint4(0, 0, 0, 0);
+                                for (int u = 0; u < 8; ++u)
+                                    *reinterpret_cast<uint4*>(pair + sg * C::CHUNK_BYTES + row * 128 + u * 16) =
+                                        make_uint4(0, 0, 0, 0);
                             }
                         }
                         fence_proxy_async_smem();
@@ -1106,16 +1161,16 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                         if (lane == 0) mbar_arrive(&misc.p_full[slot]);
                         // rotate the denominator rows: the next step's branches first
 #pragma unroll
-                        for (int r = 0; r < C::SBR; ++r) {
-                            float t[kHP];
+                        for (int r2 = 0; r2 < C::SBR; ++r2) {
+                            float t[kHG];
 #pragma unroll
-                            for (int i = 0; i < kHP; ++i) t[i] = l[0][i];
+                            for (int i = 0; i < kHG; ++i) t[i] = l[0][i];
 #pragma unroll
                             for (int b = 0; b + 1 < NB; ++b)
 #pragma unroll
-                                for (int i = 0; i < kHP; ++i) l[b][i] = l[b + 1][i];
+                                for (int i = 0; i < kHG; ++i) l[b][i] = l[b + 1][i];
 #pragma unroll
-                            for (int i = 0; i < kHP; ++i) l[NB - 1][i] = t[i];
+                            for (int i = 0; i < kHG; ++i) l[NB - 1][i] = t[i];
                         }
                         ++gs;
                     }
@@ -1126,51 +1181,50 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
 
                 // ---------------------------------------------------- epilogue
                 // denominators (final once the last probabilities are written):
-                // warp reduce-scatter, then the four warps through shared memory,
-                // while the range's last output MMA may still run
+                // warp reduce-scatter, then the four warps through shared memory
+                // (this group's 32 columns of red_sum), while the range's last
+                // output MMA may still run
+                constexpr int NV = NB * kHG;  // (branch, head) values of the group
+                static_assert(NV <= 32, "a group's denominators fit its half of red_sum");
                 {
-                    constexpr int NV = NB * kHP;
                     float f[NV];
 #pragma unroll
                     for (int b = 0; b < NB; ++b)
 #pragma unroll
-                        for (int i = 0; i < kHP; ++i) f[b * kHP + i] = l[b][i];
+                        for (int i = 0; i < kHG; ++i) f[b * kHG + i] = l[b][i];
                     warp_sum_scatter<NV, 16, NV>(f, lane);
-                    if constexpr (NV >= 32) {
-#pragma unroll
-                        for (int r = 0; r < NV / 32; ++r) misc.red_sum[quad][(NV / 32) * lane + r] = f[r];
-                    } else {
-                        if ((lane & 1) == 0) misc.red_sum[quad][lane >> 1] = f[0];
-                    }
+                    constexpr int SPAN = 32 / NV;  // lanes holding one value's total
+                    if ((lane & (SPAN - 1)) == 0) misc.red_sum[quad][32 * sg + lane / SPAN] = f[0];
                 }
-                bad = named_bar_or<1, 128>(bad);  // also publishes red_sum
+                bad = named_bar_or_id<128>(gbar, bad);  // also publishes red_sum
                 // one window holds every tile of the sequence: no split
                 const bool single = cum >= A0 && cum + (tiles - 1) * kTileCost < A1;
-                const size_t slot = (size_t)blockIdx.x + n;
-                if (stid < NB * kHP) {
-                    const float lt = misc.red_sum[0][stid] + misc.red_sum[1][stid] + misc.red_sum[2][stid] +
-                                     misc.red_sum[3][stid];
-                    misc.inv_l[stid] = 1.0f / lt;
-                    const int b = stid / kHP, i = stid % kHP;
+                const size_t slot = (size_t)grp.slot0 + grp.ci + n;
+                if (stid < NV) {
+                    const int c = 32 * sg + stid;
+                    const float lt = misc.red_sum[0][c] + misc.red_sum[1][c] + misc.red_sum[2][c] + misc.red_sum[3][c];
+                    const int b = stid / kHG, i = hoff + stid % kHG;
+                    misc.inv_l[b * kHP + i] = 1.0f / lt;
                     if (!single)  // all 16 columns (padded heads too): the merge reads whole rows
-                        a.lse_part[(slot * NB + b) * kHP + i] = bad ? bad_split_marker() : misc.m_run[stid] + __log2f(lt);
+                        a.lse_part[(slot * NB + b) * kHP + i] =
+                            bad ? bad_split_marker() : misc.m_run[b * kHP + i] + __log2f(lt);
                 }
                 // the range's last output MMA (the barrier below also publishes inv_l)
                 {
                     const bool ok = mbar_wait(&misc.p_empty[(gs - 1) % C::NSP], ((gs - 1) / C::NSP) & 1);
-                    if (named_bar_or<1, 128>(!ok)) {
+                    if (named_bar_or_id<128>(gbar, !ok)) {
                         dead = true;
                         break;
                     }
                 }
                 tc_fence_after();
                 // outputs: a block of TMEM holds 128 latent rows x 16 heads of one
-                // branch (or two branches of 64 rows when DC = 64); all blocks are
-                // read before a single wait
+                // branch (or two branches of 64 rows when DC = 64); this group
+                // reads its 8 heads of every block before a single wait
                 constexpr int WIDTH = DC >= 128 ? 128 : DC;  // valid rows per block
-                float o[C::O_BLOCKS][kHP];
+                float o[C::O_BLOCKS][kHG];
 #pragma unroll
-                for (int blk = 0; blk < C::O_BLOCKS; ++blk) tmem_ld16(tmem + lane_off + blk * kHP, o[blk]);
+                for (int blk = 0; blk < C::O_BLOCKS; ++blk) tmem_ld8(tmem + lane_off + blk * kHP + hoff, o[blk]);
                 tmem_wait_ld();
 #pragma unroll
                 for (int blk = 0; blk < C::O_BLOCKS; ++blk) {
@@ -1180,27 +1234,25 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                     const int k = (gp * 128 + row0) % DC + (row - row0);  // latent column of this row
                     const bool mine = row >= row0 && row < row0 + WIDTH;
                     if (!mine) continue;
-                    const float* inv = &misc.inv_l[b * kHP];
+                    const float* inv = &misc.inv_l[b * kHP + hoff];
 #pragma unroll
-                    for (int i = 0; i < kHP; ++i) o[blk][i] = bad ? 0.f : o[blk][i] * inv[i];
+                    for (int i = 0; i < kHG; ++i) o[blk][i] = bad ? 0.f : o[blk][i] * inv[i];
                     if (single) {
-                        __nv_bfloat16* dst = a.out + ((size_t)n * H * NB + b) * DC + k;
+                        __nv_bfloat16* dst = a.out + (((size_t)n * H + grp.h0 + hoff) * NB + b) * DC + k;
 #pragma unroll
-                        for (int i = 0; i < kHP; ++i)
-                            if (i < H) dst[(size_t)i * NB * DC] = to_bf16(o[blk][i] * a.out_scale);
+                        for (int i = 0; i < kHG; ++i)
+                            if (hoff + i < grp.hn) dst[(size_t)i * NB * DC] = to_bf16(o[blk][i] * a.out_scale);
                     } else {
-                        // partial layout [slot][branch][k][16 heads]: one 64-byte
-                        // row per thread, two 32-byte stores
-                        float* dst = a.o_part + ((slot * NB + b) * DC + k) * kHP;
+                        // partial layout [slot][branch][k][16 heads]: this group's
+                        // 8 heads are one 32-byte store
+                        float* dst = a.o_part + ((slot * NB + b) * DC + k) * kHP + hoff;
                         st_global_v8(dst, o[blk][0], o[blk][1], o[blk][2], o[blk][3], o[blk][4], o[blk][5],
                                      o[blk][6], o[blk][7]);
-                        st_global_v8(dst + 8, o[blk][8], o[blk][9], o[blk][10], o[blk][11], o[blk][12],
-                                     o[blk][13], o[blk][14], o[blk][15]);
                     }
                 }
                 if (bad && stid == 0) record_error(a.err, MLRA_ERR_DEVICE_BAD_INDEX);
                 tc_fence_before();
-                named_bar_sync<1, 128>();  // inv_l and red_sum are reused by the next range
+                named_bar_sync_id<128>(gbar);  // inv_l and red_sum are reused by the next range
                 if (stid == 0) {
                     // a split's partials are complete: counted for the merge when
                     // this CTA's work ends (only its first and last ranges can be
@@ -1209,10 +1261,12 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                     if (!single) {
                         if (pend_a < 0) pend_a = n; else pend_b = n;
                     }
-                    misc.last_seg[0] = n;
-                    misc.last_seg[1] = cum;
-                    misc.last_seg[2] = tiles;
-                    misc.last_seg[3] = c1_member;
+                    if (sg == 0) {
+                        misc.last_seg[0] = n;
+                        misc.last_seg[1] = cum;
+                        misc.last_seg[2] = tiles;
+                        misc.last_seg[3] = c1_member;
+                    }
                 }
                 ++sc;
                 finish_segment(n, cum, tiles);
@@ -1221,13 +1275,14 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                 record_error(a.err, MLRA_ERR_DEVICE_TIMEOUT);
                 *abort_flag = 1;
             }
-            if (!dead && stid == 0 && pend_a >= 0) {
-                // the partial stores of all 128 threads precede the named
-                // barrier that ended their epilogue; one release fence makes
-                // them visible before both counts
+            // both groups' partial stores precede this barrier; then one
+            // release fence makes them visible before both counts (none when
+            // either group gave up: the CTA then skips its merges too)
+            const bool any_dead = named_bar_or<5, 2 * 128>(dead);
+            if (!any_dead && sg == 0 && stid == 0 && pend_a >= 0) {
                 fence_acq_rel_gpu();
-                red_add_relaxed_gpu(a.seq_cnt + pend_a, 1);
-                if (pend_b >= 0) red_add_relaxed_gpu(a.seq_cnt + pend_b, 1);
+                red_add_relaxed_gpu(a.seq_cnt + grp.cnt0 + pend_a, 1);
+                if (pend_b >= 0) red_add_relaxed_gpu(a.seq_cnt + grp.cnt0 + pend_b, 1);
             }
         }
     }
@@ -1243,8 +1298,8 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
     __nv_bfloat16* wt = reinterpret_cast<__nv_bfloat16*>(sm + C::OFF_PAIR + C::NSTAGE * C::PAIR_BYTES -
                                                          UpTile<NB * DC>::W_BYTES);
     const bool fused = a.w_uv != nullptr;
-    if (fused && (int)blockIdx.x < a.heads * a.d_h / 16) up_stage_weights<NB, DC>(a, wt);
-    merge_tail<NB, DC>(a, misc.last_seg[0], misc.last_seg[1], misc.last_seg[2], misc.last_seg[3] != 0, chunk,
+    if (fused && (int)blockIdx.x < a.heads * a.d_h / 16) up_stage_weights<NB, DC>(a, wt, blockIdx.x);
+    merge_tail<NB, DC>(a, grp, misc.last_seg[0], misc.last_seg[1], misc.last_seg[2], misc.last_seg[3] != 0, chunk,
                        reinterpret_cast<float*>(sm + C::OFF_PAIR), &misc.merge_flag, &misc.merge_full);
     if (fused) up_proj_tail<NB, DC>(a, sm + C::OFF_PAIR, wt, &misc.merge_flag);
 }
@@ -1339,7 +1394,7 @@ cudaError_t launch_cfg(const DecodeArgs& a, cudaStream_t stream) {
 }  // namespace
 
 bool decode_tc_supported(int branches, int d_c, int d_r, int heads) {
-    if (heads > kHP || (d_r != 32 && d_r != 64)) return false;
+    if (heads > kMaxTcHeads || (d_r != 32 && d_r != 64)) return false;
     switch (d_c) {
         case 64: return branches == 2 || branches == 4;
         case 128: return branches == 1 || branches == 2 || branches == 4;

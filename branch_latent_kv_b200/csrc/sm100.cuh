@@ -102,6 +102,12 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
     return p;
 }
+// L2 policy: normal priority (lines that other CTAs read again soon)
+__device__ __forceinline__ uint64_t l2_policy_evict_normal() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
 __device__ __forceinline__ void tma_load_2d_hint(void* smem_dst, const CUtensorMap* map, int32_t x,
                                                  int32_t y, uint64_t* bar, uint64_t policy) {
     asm volatile(
@@ -227,6 +233,25 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
                  : "r"(taddr));
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 32 lanes x 8 columns of 32-bit (as tmem_ld16, columns col..col+7).
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7])
+                 : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                 ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])),
+                   "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])),
+                   "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
+                 : "memory");
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
@@ -372,6 +397,23 @@ __device__ __forceinline__ bool named_bar_or(bool pred) {
                  "selp.u32 %0, 1, 0, p;\n\t}"
                  : "=r"(r) : "r"((uint32_t)pred), "n"(ID), "n"(COUNT) : "memory");
     return r != 0;
+}
+
+// The same with the barrier id in a register (COUNT fixed).
+template <int COUNT>
+__device__ __forceinline__ bool named_bar_or_id(uint32_t id, bool pred) {
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.u32 p, %1, 0;\n\t"
+                 "barrier.cta.red.or.pred p, %2, %3, p;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(r) : "r"((uint32_t)pred), "r"(id), "n"(COUNT) : "memory");
+    return r != 0;
+}
+
+template <int COUNT>
+__device__ __forceinline__ void named_bar_sync_id(uint32_t id) {
+    asm volatile("barrier.cta.sync %0, %1;" ::"r"(id), "n"(COUNT) : "memory");
 }
 
 template <int ID, int COUNT>

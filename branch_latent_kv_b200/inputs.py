@@ -78,6 +78,10 @@ WORKLOADS = {
                                   d_r=64, page_size=64, seqlen=16384),
     "context_2m": Workload("context_2m", batch=1, heads=16, branches=4, d_c=128, d_r=64,
                            page_size=64, seqlen=2097152, page_order="permuted"),
+    # Many query heads on one latent cache (every head reads the same
+    # latents, as in MLA's large models): the 2.9B cache read by 64 heads.
+    "heads_64": Workload("heads_64", batch=16, heads=64, branches=4, d_c=128, d_r=64,
+                         page_size=64, seqlen=8192, d_h=64),
 }
 
 

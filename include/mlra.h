@@ -118,8 +118,12 @@ MLRA_API size_t mlra_decode_workspace_bytes(const mlra_dims* dims, int32_t num_c
  *
  * Runs on the tensor cores (tcgen05, operands staged by TMA) as one
  * cooperative kernel (one CTA per SM, all resident; the CTAs that share a
- * sequence merge their partials at the end).  Supported
- * shapes: heads <= 16; (branches, d_c) in {(2,64), (4,64), (1,128), (2,128),
+ * sequence merge their partials at the end).  The MMAs take 16 heads at a
+ * time: more heads run as ceil(heads / 16) groups on as many equal parts of
+ * the grid, which walk the same tokens together so that the cache crosses
+ * HBM about once (the repeat reads of a line hit L2).  Supported
+ * shapes: heads <= 128 with batch * ceil(heads / 16) <= 65535;
+ * (branches, d_c) in {(2,64), (4,64), (1,128), (2,128),
  * (4,128), (1,256), (2,256), (1,512)}; d_r in {32, 64}; page_size in
  * {16, 32, 64, 128}.  Other shapes return MLRA_ERR_UNSUPPORTED
  * (mlra_decode_simt covers more).
@@ -145,11 +149,11 @@ MLRA_API mlra_status mlra_decode(const mlra_dims* dims, const void* q_lat, const
  *         memory the device can map
  * `out` is written exactly as mlra_decode writes it (the same bits).  After
  * the launch's merges the CTAs meet once (a bounded grid-wide wait, reported
- * as MLRA_ERR_DEVICE_TIMEOUT if it expires) and heads * d_h / 16 of them form
- * 16 output columns each, in fp32 on the warp-level tensor cores.
- * Supported: the shapes of mlra_decode with batch <= 64 and
- * heads * d_h / 16 <= the SM count; other calls return MLRA_ERR_UNSUPPORTED
- * (use mlra_decode and mlra_up_proj).
+ * as MLRA_ERR_DEVICE_TIMEOUT if it expires) and form the heads * d_h / 16
+ * blocks of 16 output columns (CTA c takes blocks c, c + grid, ...) in fp32
+ * on the warp-level tensor cores.
+ * Supported: the shapes of mlra_decode with batch <= 64; other batches
+ * return MLRA_ERR_UNSUPPORTED (use mlra_decode and mlra_up_proj).
  */
 MLRA_API mlra_status mlra_decode_up_proj(const mlra_dims* dims, const void* q_lat, const void* q_rope,
                                          const void* latent_cache, const void* rope_cache,

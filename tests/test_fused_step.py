@@ -94,3 +94,29 @@ def test_fused_step_rejects_what_it_does_not_cover():
     with pytest.raises(b.MlraError) as e:
         b.mlra_decode_up_proj(*_args(x), x.w_uv)
     assert e.value.status == b.MLRA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("heads,d_h", [(32, 128), (48, 64), (128, 128)])
+def test_fused_step_head_groups(oracle_lib, heads, d_h):
+    """Groups of 16 heads in the attention, and in the up-projection more
+    16-column blocks than CTAs (32 x 128 / 16 = 256, 128 x 128 / 16 = 1024
+    blocks on 148 CTAs): each CTA takes blocks c, c + grid, ...  Two calls on
+    one workspace: the grid-wide counter returns to zero."""
+    w = Workload("fused_groups", batch=8, heads=heads, branches=4, d_c=128, d_r=64, page_size=64, d_h=d_h,
+                 page_order="permuted")
+    g = torch.Generator().manual_seed(heads)
+    seqlens = torch.randint(1, 3000, (8,), generator=g, dtype=torch.int32)
+    x = make_inputs(w, seed=heads, seqlens=seqlens, device="cuda")
+    out_ref = b.mlra_decode(*_args(x))
+    ws = torch.zeros(b.mlra_decode_workspace_bytes(b.decode_dims(x.q_lat, x.q_rope, x.latent_cache,
+                                                                  x.block_table)), dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        out, y = b.mlra_decode_up_proj(*_args(x), x.w_uv, workspace=ws)
+        assert torch.equal(out, out_ref)
+        assert b.mlra_read_device_error(ws) == b.MLRA_OK
+    lat, _, st = oracle_lib.decode(x.q_lat.cpu(), x.q_rope.cpu(), x.latent_cache.cpu(), x.rope_cache.cpu(),
+                                   x.block_table.cpu(), x.seqlens.cpu(), x.scale, x.out_scale)
+    assert st == 0
+    y_ref = oracle_lib.up_proj(lat, x.w_uv.cpu(), d_h)
+    max_abs, rel = _close(y, y_ref)
+    assert max_abs <= MAX_ABS and rel <= REL_L2, (heads, d_h, max_abs, rel)
