@@ -1,6 +1,7 @@
 // api.cu -- the C ABI declared in include/mlra.h: host-side validation,
 // workspace sizing and kernel launches.  No allocation, no synchronisation
 // (except mlra_read_device_error), no exceptions across the boundary.
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 
@@ -408,7 +409,10 @@ mlra_status mlra_prepare(const mlra_dims* dims, int32_t d_h, const void* q_c, co
     a.page_size = dims->page_size;
     a.max_pages = dims->max_pages_per_seq;
     a.num_pages = dims->num_pages;
-    a.rope_base = rope_base;
+    for (int i = 0; i < 32; ++i)
+        a.rope_turns[i] = 2 * i < dims->d_r
+                              ? std::pow((double)rope_base, -2.0 * i / dims->d_r) / (2.0 * 3.14159265358979323846)
+                              : 0.0;
     return cuda_status(launch_prepare(a, static_cast<cudaStream_t>(stream)));
 }
 

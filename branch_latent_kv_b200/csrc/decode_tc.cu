@@ -92,7 +92,7 @@ struct Cfg {
     // TMEM slot t % NRS: the score MMA of a tile's first step waits for the
     // output MMA NSP steps back, so the softmax has read every RoPE score
     // more than ceil(NSP / NSTEP) tiles back.
-    static constexpr int NSP = 3;
+    static constexpr int NSP = NPAIR == 1 ? 4 : 3;
     static constexpr int NROPE = NPAIR == 1 ? 4 : NPAIR == 2 ? 3 : 2;
     static constexpr int NRS = (NSP + NSTEP - 1) / NSTEP > 2 ? (NSP + NSTEP - 1) / NSTEP : 2;
     static constexpr int FIXED = NROPE * ROPE_BYTES + QSET_BYTES + NSP * P_BYTES + MISC_BYTES;
@@ -131,9 +131,9 @@ struct Misc {
     uint64_t pair_empty[NSTAGE];
     uint64_t rope_full[4];  // tile t in RoPE slot t % NROPE: its RoPE keys are in shared memory
     uint64_t rope_empty[4];  // its RoPE score MMA finished
-    uint64_t s_full[3];   // step g in slot g % NSP: its scores are in TMEM
-    uint64_t p_full[3];   // its probabilities are in shared memory
-    uint64_t p_empty[3];  // its output MMA finished (S and P slots free, O up to date)
+    uint64_t s_full[4];   // step g in slot g % NSP: its scores are in TMEM
+    uint64_t p_full[4];   // its probabilities are in shared memory
+    uint64_t p_empty[4];  // its output MMA finished (S and P slots free, O up to date)
     uint64_t q_full;      // sequence range r (phase r & 1): its queries are in shared memory
     uint64_t q_empty;     // the score MMAs of a range with a successor have finished
     uint64_t drain[2];
@@ -628,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ DecodeArgs a) {
     using C = Cfg<NB, DC, DR>;
     using M = Misc<C::NSTAGE>;
-    static_assert(C::NSP <= 3 && C::NROPE <= 4, "barrier arrays of Misc");
+    static_assert(C::NSP <= 4 && C::NROPE <= 4, "barrier arrays of Misc");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     M& misc = *reinterpret_cast<M*>(sm + C::OFF_MISC);
@@ -728,12 +728,14 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                 // the first range's queries; a later range's are loaded by the
                 // score MMA warp once the range before has its last scores, so
                 // the copies of the cache never wait for the query buffer
-                if (lane == 0 && sc == 0) load_queries<C>(maps, sm, misc.q_full, n, grp.h0);
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
-                ++sc;
+                // (the range's first window of block-table entries is in flight
+                // meanwhile: a lane per entry, a window of 32 pages)
                 const int32_t* bt = a.block_table + (size_t)n * a.max_pages;
-                int win_base = -(1 << 30), win_val = 0;
+                int win_base = tb * kT / P, win_val = 0;
+                if (win_base + lane < a.max_pages) win_val = __ldg(bt + win_base + lane);
+                if (lane == 0 && sc == 0) load_queries<C>(maps, sm, misc.q_full, n, grp.h0);
+                win_val = (win_val >= 0 && win_val < a.num_pages) ? win_val : 0;  // bad entries are reported by the softmax warps
+                ++sc;
                 for (int j = tb; j < te && ok; ++j) {
                     const int tok0 = j * kT;
                     const int valid = min(kT, L - tok0);

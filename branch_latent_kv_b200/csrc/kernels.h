@@ -136,7 +136,9 @@ struct PrepareArgs {
     __nv_bfloat16* rope_cache;    // [pages, P, d_r] one row per sequence written
     int* status;                  // optional device error word
     int batch, heads, branches, d_c, d_r, d_h, page_size, max_pages, num_pages;
-    float rope_base;
+    // RoPE pair i turns by rope_turns[i] * p full turns at position p:
+    // rope_base^(-2i/d_r) / (2 pi), formed on the host in fp64
+    double rope_turns[32];
 };
 
 // Query absorption, rotary embedding and the new token's append.

@@ -249,7 +249,8 @@ MLRA_API mlra_status mlra_up_proj_gated(int32_t batch, int32_t heads, int32_t br
  *  2. Rotary embedding (RoFormer's definition; the pages do not specify one)
  *     of the RoPE query and the new token's RoPE key at its position
  *     p = seqlens[n] - 1: pair i = (x[2i], x[2i+1]) turns by the angle
- *     p * rope_base^(-2i/d_r) (angles formed in fp64).
+ *     p * rope_base^(-2i/d_r) (the angle formed in turns in fp64, reduced to
+ *     a fraction of a turn, its sine and cosine in fp32).
  *  3. Append: latent_cache[page][slot] = c_new[n], rope_cache[page][slot] =
  *     the rotated key, page = block_table[n][p / P], slot = p mod P.
  *   dims         as mlra_decode's (batch, heads, branches, d_c, d_r,
@@ -272,7 +273,12 @@ MLRA_API mlra_status mlra_up_proj_gated(int32_t batch, int32_t heads, int32_t br
  *                MLRA_ERR_DEVICE_BAD_INDEX for a page outside the pool); such
  *                a sequence's row is not written (its queries still are)
  * Requires d_c a multiple of 8, d_r even and at most 64, 16-byte aligned
- * arrays.  Allocates nothing; fp32 arithmetic, bf16 results.
+ * arrays.  Allocates nothing; fp32 arithmetic (the absorption on the
+ * warp-level tensor cores: bf16 products, fp32 sums), bf16 results.
+ * The launch is a programmatic dependent of the preceding kernel in the
+ * stream: its CTAs may start while that kernel runs and read w_uk, seqlens
+ * and block_table then (every other input only after it has finished), so
+ * these three must not be written by that kernel.
  */
 MLRA_API mlra_status mlra_prepare(const mlra_dims* dims, int32_t d_h, const void* q_c, const void* q_r,
                                   const void* w_uk, const void* c_new, const void* kr_new,

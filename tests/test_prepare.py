@@ -9,7 +9,7 @@ import pytest
 import torch
 
 from branch_latent_kv_b200 import binding as b
-from branch_latent_kv_b200.inputs import WORKLOADS, make_inputs
+from branch_latent_kv_b200.inputs import Workload, WORKLOADS, make_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -45,10 +45,20 @@ def _pre_inputs(x, d_h, seed):
 
 @pytest.mark.parametrize("name,seqlens", [
     ("decode_2p9b", None), ("tiny", None), ("mla_equal_bytes", [1, 64, 65, 16384] * 8),
-    ("ragged", None),
+    ("ragged", None), ("odd", None), ("far", [2_000_001, 3]),
 ])
 def test_prepare_matches_oracle(oracle_lib, name, seqlens):
-    w = WORKLOADS[name]
+    """The workloads' shapes, plus one ("odd") whose head dimension is not a
+    multiple of the MMA's K = 16 (d_h = 24: zero-padded), whose d_c = 96
+    leaves a half column block, and whose 70 sequences take two chunks of
+    the absorption's 64 (the second a partial 16-row tile), and one ("far")
+    whose new token sits at position 2,000,000."""
+    w = WORKLOADS.get(name)
+    if name == "odd":
+        w = Workload("odd", batch=70, heads=3, branches=2, d_c=96, d_r=32, page_size=16, seqlen=100, d_h=24,
+                     page_order="permuted")
+    if name == "far":  # a position of two million: the angle's reduction to a fraction of a turn
+        w = Workload("far", batch=2, heads=4, branches=1, d_c=8, d_r=64, page_size=128, d_h=64)
     if name == "decode_2p9b":
         w = w.with_(seqlen=3000)
     if name == "ragged":
