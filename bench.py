@@ -62,10 +62,8 @@ FALLBACK_HBM_GBS = 6650.0
 # ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the
 # hash of the kernel sources it was taken on.  Reported as null whenever the
 # kernel sources differ from the captured ones.
-# DRAM bytes (read + write) of one decode launch from the committed ncu
-# capture, valid only for that workload and those kernel sources
-TRAFFIC_CAPTURE = {"workload": "decode_2p9b", "sources_sha1": "98efd80ef51673f256d36a0e78337dc871473fb0",
-                   "bytes_per_launch": 151417600 + 4464128}
+TRAFFIC_CAPTURE = {"workload": "decode_2p9b", "sources_sha1": "1584547f18bd63dcc52785ab37a754e4bec6fda9",
+                   "bytes_per_launch": 151392256 + 4140032}
 KERNEL_SOURCES = ["branch_latent_kv_b200/csrc/decode_tc.cu", "branch_latent_kv_b200/csrc/sm100.cuh",
                   "branch_latent_kv_b200/csrc/common.cuh"]
 
