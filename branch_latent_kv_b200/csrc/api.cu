@@ -38,7 +38,7 @@ mlra_status check_tc_coverage(const mlra_dims* d) {
     if (!is_pow2_in(d->page_size, 16, 128)) return MLRA_ERR_UNSUPPORTED;
     if (!decode_tc_supported(d->branches, d->d_c, d->d_r, d->heads)) return MLRA_ERR_UNSUPPORTED;
     // one block of split counters per head group
-    if ((int64_t)d->batch * tc_head_groups(d->heads) > kMaxBatch) return MLRA_ERR_UNSUPPORTED;
+    if ((int64_t)d->batch * tc_head_groups(d->heads, d->d_c) > kMaxBatch) return MLRA_ERR_UNSUPPORTED;
     return MLRA_OK;
 }
 

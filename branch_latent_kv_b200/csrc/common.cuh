@@ -23,14 +23,16 @@ constexpr float kLog2e = 1.4426950408889634f;
 //   [0, 256)        int32 error word (first device-side error code, else 0)
 //   split counters  int32 [kMaxBatch + 1]              (fixed place)
 //   lse partials    fp32 [slots][branches][HP]         (log2 domain; HP = the
-//                   head count rounded up to a multiple of 16)
+//                   head count rounded up to whole head tiles: 16 up to 16
+//                   heads, else a multiple of 32)
 //   o partials      fp32 [slots][branches][d_c][HP]    (normalised per split;
 //                   heads innermost)
 // slots = num_ctas + batch: the partial of CTA c for sequence n lives in slot
 // c + n (unique because CTA ranges are contiguous and ordered).  The
-// tensor-core kernel writes rows of 16 heads: with G = HP / 16 head groups,
-// group g owns the G-th part of the bytes, cpg + batch slots of 16-wide rows
-// (cpg = num_ctas / G), and split counters [g batch, (g + 1) batch).
+// tensor-core kernel writes rows of one head tile (T = 16 or 32 heads): with
+// G = HP / T head groups, group g owns the G-th part of the bytes, cpg + batch
+// slots of T-wide rows (cpg = num_ctas / G), and split counters
+// [g batch, (g + 1) batch).
 // ---------------------------------------------------------------------------
 struct WorkspaceLayout {
     size_t err_off, lse_off, o_off, cnt_off, total;
@@ -42,9 +44,15 @@ __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_
 // Largest batch the library accepts (int32 sequence ids, 16-bit grid rows).
 constexpr int kMaxBatch = 65535;
 
-// Heads the tensor-core kernel takes: groups of 16 (its MMA's N), at most 8.
+// Heads the tensor-core kernel takes: one tile of 16 heads (its MMA's N), or
+// tiles of 32 heads when there are more and a branch is at least 128 wide
+// (narrower branches put two in a step, and a softmax thread's registers hold
+// 16 heads of one branch or 8 heads of two); at most 128 heads.
 constexpr int kMaxTcHeads = 128;
-__host__ __device__ inline int tc_head_groups(int heads) { return (heads + 15) / 16; }
+__host__ __device__ inline int tc_head_tile(int heads, int d_c) { return heads <= 16 || d_c < 128 ? 16 : 32; }
+__host__ __device__ inline int tc_head_groups(int heads, int d_c) {
+    return (heads + tc_head_tile(heads, d_c) - 1) / tc_head_tile(heads, d_c);
+}
 
 __host__ __device__ inline WorkspaceLayout workspace_layout(int batch, int heads, int branches,
                                                             int d_c, int num_ctas) {
@@ -56,7 +64,7 @@ __host__ __device__ inline WorkspaceLayout workspace_layout(int batch, int heads
     // that reuse the workspace find them where they left them (at zero)
     w.cnt_off = 256;
     w.lse_off = align256(w.cnt_off + sizeof(int) * (size_t)(kMaxBatch + 1));
-    const size_t hp = 16 * (size_t)tc_head_groups(heads);  // heads padded to a multiple of 16
+    const size_t hp = (size_t)tc_head_tile(heads, d_c) * tc_head_groups(heads, d_c);  // heads padded to whole tiles
     w.o_off = align256(w.lse_off + sizeof(float) * (size_t)w.slots * branches * hp);
     w.total = align256(w.o_off + sizeof(float) * (size_t)w.slots * branches * d_c * hp);
     return w;

@@ -126,7 +126,7 @@ mlra_status mlra_decode_static_scratch(const mlra_dims* dims, const void* q_lat,
     // that no earlier call's state -- a stale count left by a kernel that gave
     // up on a bounded wait -- reaches this one.  Stream-ordered, no allocation.
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const size_t clear = reinterpret_cast<char*>(a.seq_cnt + (size_t)dims->batch * mlra::tc_head_groups(dims->heads)) -
+    const size_t clear = reinterpret_cast<char*>(a.seq_cnt + (size_t)dims->batch * mlra::tc_head_groups(dims->heads, dims->d_c)) -
                          static_cast<char*>(scratch);
     if (cudaMemsetAsync(scratch, 0, clear, st) != cudaSuccess) return MLRA_ERR_CUDA;
     if (mlra::launch_decode_tc(a, st) != cudaSuccess) return MLRA_ERR_CUDA;

@@ -49,15 +49,17 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kHP = 16;             // heads padded to the MMA N
-constexpr int kHG = kHP / 2;        // heads of one softmax group
+// Heads per MMA tile (the MMA's N): 16, or 32 when a step has more than 16
+// heads; each softmax warpgroup takes half of them.
 constexpr int kT = kTileTokens;     // tokens per tile = MMA M
 constexpr int kThreads = 352;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kSmemLimit = 232448;  // max dynamic shared memory per CTA on sm_100
 
-template <int NB, int DC, int DR>
+template <int NB, int DC, int DR, int HP_>
 struct Cfg {
+    static constexpr int HP = HP_;                          // heads per tile (MMA N)
+    static constexpr int HG = HP / 2;                       // heads per softmax warpgroup
     static constexpr int W = NB * DC;                       // latent elements per token
     static constexpr int NCHUNK = W / 64;                   // 64-column (128-byte) chunks
     // A step is the unit of the MMA <-> softmax pipeline: SBR branches whose
@@ -74,13 +76,13 @@ struct Cfg {
     static constexpr int PAIR_BYTES = 2 * CHUNK_BYTES;      // 32 KB
     static constexpr int ROPE_ROW = DR * 2;                 // 128 or 64 bytes
     static constexpr int ROPE_BYTES = kT * ROPE_ROW;
-    static constexpr int Q_CHUNK_BYTES = kHP * 128;         // [16 heads x 64 elements]
+    static constexpr int Q_CHUNK_BYTES = HP * 128;          // [HP heads x 64 elements]
     static constexpr int Q_BYTES = NCHUNK * Q_CHUNK_BYTES;
-    static constexpr int QR_BYTES = kHP * ROPE_ROW;                 // [16 heads x d_r]
+    static constexpr int QR_BYTES = HP * ROPE_ROW;                  // [HP heads x d_r]
     static constexpr int QR_SPAN = (QR_BYTES + 1023) / 1024 * 1024;  // keeps the next region aligned
-    static constexpr int P_BRANCH_BYTES = kT * kHP * 2;     // 4 KB
+    static constexpr int P_BRANCH_BYTES = kT * HP * 2;      // 4 KB per 16 heads
     static constexpr int P_BYTES = SBR * P_BRANCH_BYTES;   // one P slot (a step)
-    static constexpr int MISC_BYTES = 4096;
+    static constexpr int MISC_BYTES = HP == 16 ? 4096 : 8192;
     static constexpr int QSET_BYTES = Q_BYTES + QR_SPAN;  // one sequence's queries
     // Pipeline depths: NSP steps may be between their score MMA and their
     // output MMA at once (S slots in TMEM, P slots in shared memory); NROPE
@@ -93,7 +95,10 @@ struct Cfg {
     // output MMA NSP steps back, so the softmax has read every RoPE score
     // more than ceil(NSP / NSTEP) tiles back.
     static constexpr int NSP = NPAIR == 1 ? 4 : 3;
-    static constexpr int NROPE = NPAIR == 1 ? 4 : NPAIR == 2 ? 3 : 2;
+    // (one slot when a tile is four pairs of 32-head steps: a tile's RoPE
+    // score is taken at its first step, long before its last pair lands, and
+    // the wider queries and probabilities leave no room for a second)
+    static constexpr int NROPE = NPAIR == 1 ? 4 : NPAIR == 2 ? 3 : HP == 16 ? 2 : 1;
     static constexpr int NRS = (NSP + NSTEP - 1) / NSTEP > 2 ? (NSP + NSTEP - 1) / NSTEP : 2;
     static constexpr int FIXED = NROPE * ROPE_BYTES + QSET_BYTES + NSP * P_BYTES + MISC_BYTES;
     static constexpr int NSTAGE_FIT = (kSmemLimit - 1024 - FIXED) / PAIR_BYTES;
@@ -109,14 +114,15 @@ struct Cfg {
     // TMEM columns: O blocks first, then two S slots, then two slots of the
     // RoPE score shared by all branches of a tile
     static constexpr int O_BLOCKS = NPAIR * BPP;
-    static constexpr int S_COL0 = O_BLOCKS * kHP;
-    static constexpr int S_SLOT_COLS = SBR * kHP;
+    static constexpr int S_COL0 = O_BLOCKS * HP;
+    static constexpr int S_SLOT_COLS = SBR * HP;
     static constexpr int R_COL0 = S_COL0 + NSP * S_SLOT_COLS;
-    static constexpr int TMEM_COLS = R_COL0 + NRS * kHP <= 128 ? 128 : 256;
+    static constexpr int TMEM_COLS = R_COL0 + NRS * HP <= 128 ? 128 : R_COL0 + NRS * HP <= 256 ? 256 : 512;
     static_assert(NB % SBR == 0 && (SBR * DC) % 128 == 0, "branches must fill whole steps and pairs");
     static_assert(NSTEP * PPS == NPAIR, "step / pair bookkeeping");
     static_assert(NSTAGE >= PPS, "a step's pairs must fit the stage ring");
-    static_assert(R_COL0 + NRS * kHP <= TMEM_COLS, "TMEM budget");
+    static_assert(R_COL0 + NRS * HP <= TMEM_COLS, "TMEM budget");
+    static_assert(HP == 16 || HP == 32, "heads per tile");
     static_assert(SMEM_BYTES <= kSmemLimit, "shared-memory budget");
     static_assert(OFF_QR + QR_BYTES <= OFF_P && OFF_Q + Q_BYTES <= OFF_QR &&
                   OFF_P + NSP * P_BYTES <= OFF_MISC && QSET_BYTES % 1024 == 0 && ROPE_BYTES % 1024 == 0,
@@ -124,8 +130,8 @@ struct Cfg {
     static_assert(DR == 32 || DR == 64, "RoPE width");
 };
 
-// Barriers and scratch in the MISC region.
-template <int NSTAGE>
+// Barriers and scratch in the MISC region (HP heads per tile, at most 4 branches).
+template <int NSTAGE, int HP>
 struct Misc {
     uint64_t pair_full[NSTAGE];
     uint64_t pair_empty[NSTAGE];
@@ -143,14 +149,20 @@ struct Misc {
     int plan[4];      // -, chunk, first sequence, its cost start
     int last_seg[4];  // this CTA's last sequence range: sequence, cost start, tiles (-1: none), c1 merges
     int merge_flag;   // merge: bit 0 a split met a bad page, bit 1 a wait expired
-    float red_max[4][2 * kHP];
-    float red_sum[4][4 * kHP];
-    alignas(16) float m_run[8 * kHP];  // running max per (branch, head), base-2 logits; read as float4
-    float inv_l[8 * kHP];              // 1 / softmax denominator per (branch, head), epilogue only
+    float red_max[4][2 * HP];  // [quadrant][step branch, head]: column maxima of a rescale
+    float red_sum[4][4 * HP];  // [quadrant][group, branch, head]: denominator partials
+    alignas(16) float m_run[4 * HP];  // running max per (branch, head), base-2 logits; read as float4
+    float inv_l[4 * HP];              // 1 / softmax denominator per (branch, head), epilogue only
 };
 
-static_assert(offsetof(Misc<5>, m_run) % 16 == 0 && offsetof(Misc<4>, m_run) % 16 == 0 &&
-              offsetof(Misc<6>, m_run) % 16 == 0, "float4 access to m_run");
+template <int NSTAGE, int HP>
+constexpr bool m_run_aligned() {
+    using M = Misc<NSTAGE, HP>;
+    return offsetof(M, m_run) % 16 == 0;
+}
+static_assert(m_run_aligned<5, 16>() && m_run_aligned<4, 16>() && m_run_aligned<6, 16>() &&
+                  m_run_aligned<2, 32>() && m_run_aligned<3, 32>() && m_run_aligned<4, 32>(),
+              "float4 access to m_run");
 
 struct Maps {
     CUtensorMap lat;   // latent cache rows [pages * P][W]
@@ -159,14 +171,14 @@ struct Maps {
     CUtensorMap qr;    // q_rope [batch][H][d_r]
 };
 
-// Head groups.  The MMAs take 16 heads (N = 16); H > 16 heads run as
-// ceil(H / 16) groups side by side.  CTA g * cpg + i (cpg = grid / groups)
-// runs window i of one cost plan over cpg windows for heads
-// [16 g, 16 g + 16), so the groups stream the same tokens at about the same
-// time and every read of a cache line after the first hits L2 (the latents
-// are shared by all heads).  Each group has its own partial slots (a block
-// of cpg + batch) and split counters (a block of batch); CTAs past
-// groups * cpg only take part in the fused up-projection.
+// Head groups.  The MMAs take one tile of HP heads (N = 16, or 32 when there
+// are more than 16 heads); more heads run as ceil(H / HP) groups side by
+// side.  CTA g * cpg + i (cpg = grid / groups) runs window i of one cost plan
+// over cpg windows for heads [HP g, HP g + HP), so the groups stream the same
+// tokens at about the same time and every read of a cache line after the
+// first hits L2 (the latents are shared by all heads).  Each group has its own
+// partial slots (a block of cpg + batch) and split counters (a block of
+// batch); CTAs past groups * cpg only take part in the fused up-projection.
 struct HeadGroup {
     int ci, cpg;   // window of this CTA, windows (CTAs) per group
     int h0, hn;    // first head of the group, heads in it
@@ -175,9 +187,11 @@ struct HeadGroup {
     bool idle;     // no group: beyond groups * cpg
 };
 
+template <int HP>
 __device__ __forceinline__ HeadGroup head_group(const DecodeArgs& a) {
+    constexpr int kHP = HP;
     HeadGroup hg;
-    const int groups = tc_head_groups(a.heads);
+    const int groups = (a.heads + HP - 1) / HP;
     hg.cpg = a.num_ctas / groups;
     const int g = (int)blockIdx.x / hg.cpg;
     hg.ci = (int)blockIdx.x - g * hg.cpg;
@@ -195,6 +209,34 @@ __device__ __forceinline__ float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// Max over the 32 lanes of a warp of each of 16 values, reduce-scattered:
+// the result for column c ends up in lanes 2c and 2c+1.  16 shuffles.
+__device__ __forceinline__ float warp_colmax16(const float (&v)[16], int lane) {
+    float a8[8], a4[4], a2[2];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {  // lanes with bit 4 keep columns 8..15
+        const bool hi = lane & 16;
+        const float keep = hi ? v[i + 8] : v[i], send = hi ? v[i] : v[i + 8];
+        a8[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 16));
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const bool hi = lane & 8;
+        const float keep = hi ? a8[i + 4] : a8[i], send = hi ? a8[i] : a8[i + 4];
+        a4[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const bool hi = lane & 4;
+        const float keep = hi ? a4[i + 2] : a4[i], send = hi ? a4[i] : a4[i + 2];
+        a2[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+    }
+    const bool hi = lane & 2;
+    const float keep = hi ? a2[1] : a2[0], send = hi ? a2[0] : a2[1];
+    const float a1 = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
+    return fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
 }
 
 // Max over the 32 lanes of a warp of each of 8 values, reduce-scattered:
@@ -218,6 +260,26 @@ __device__ __forceinline__ float warp_colmax8(const float (&v)[8], int lane) {
     float a1 = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 4));
     a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 2));
     return fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
+}
+
+// The same for a softmax group's N = 8 or 16 heads: column c in lanes
+// [c 32 / N, (c + 1) 32 / N).
+template <int N>
+__device__ __forceinline__ float warp_colmax(const float (&v)[N], int lane) {
+    if constexpr (N == 8) return warp_colmax8(v, lane);
+    else return warp_colmax16(v, lane);
+}
+
+// TMEM loads and stores of a softmax group's N = 8 or 16 columns.
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[N]) {
+    if constexpr (N == 8) tmem_ld8(taddr, v);
+    else tmem_ld16(taddr, v);
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const float (&v)[N]) {
+    if constexpr (N == 8) tmem_st8(taddr, v);
+    else tmem_st16(taddr, v);
 }
 
 // Sum over the 32 lanes of a warp of each of N values (N = 16, 32, 64, 128),
@@ -323,9 +385,11 @@ __device__ __forceinline__ void load_queries(const Maps& maps, uint8_t* sm, uint
 // and the last of the S + G counts returns seq_cnt[n] to zero.  The arithmetic
 // is laid out for latency: every thread loads its values for up to 8 splits
 // at once before combining them.
-template <int NB, int DC>
+template <int NB, int DC, int HP>
 __device__ __forceinline__ void merge_tail(const DecodeArgs& a, const HeadGroup& grp, int n, int cum, int tiles,
                                            bool c1_member, int chunk, float* w_s, int* flag, uint64_t* bar) {
+    constexpr int kHP = HP;
+    constexpr int QD = HP / 4;    // head quads of a row
     constexpr int HB = NB * kHP;  // (branch, head) columns of a split's log-sum-exp row
     constexpr int R = NB * DC;    // (branch, latent column) rows
     const int tid = threadIdx.x;
@@ -436,8 +500,8 @@ __device__ __forceinline__ void merge_tail(const DecodeArgs& a, const HeadGroup&
 
     // items (row, head quad), quads fastest: conflict-free 16-byte reads; the
     // weighted sum over the splits in split order, eight splits' loads at once
-    for (int e = tid; e < rows * 4; e += kThreads) {
-        const int lr = e >> 2, q = e & 3, row = r0 + lr;
+    for (int e = tid; e < rows * QD; e += kThreads) {
+        const int lr = e / QD, q = e % QD, row = r0 + lr;
         const int b = row / DC, k = row % DC;
         const float* w = w_s + b * kHP + 4 * q;
         const float* src = part_s + lr * kHP + 4 * q;
@@ -623,18 +687,21 @@ __device__ __forceinline__ void up_proj_tail(const DecodeArgs& a, uint8_t* ring,
     if (tid == 0 && departed == a.num_ctas + workers - 1) *gcnt = 0;
 }
 
-template <int NB, int DC, int DR>
+template <int NB, int DC, int DR, int HP>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ DecodeArgs a) {
-    using C = Cfg<NB, DC, DR>;
-    using M = Misc<C::NSTAGE>;
+    using C = Cfg<NB, DC, DR, HP>;
+    using M = Misc<C::NSTAGE, HP>;
+    constexpr int kHP = HP;       // heads per tile (the MMAs' N)
+    constexpr int kHG = HP / 2;   // heads per softmax warpgroup
+    static_assert(sizeof(M) <= C::MISC_BYTES, "barriers and scratch fit the MISC region");
     static_assert(C::NSP <= 4 && C::NROPE <= 4, "barrier arrays of Misc");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     M& misc = *reinterpret_cast<M*>(sm + C::OFF_MISC);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int P = a.page_size;
-    const HeadGroup grp = head_group(a);
+    const HeadGroup grp = head_group<HP>(a);
 
     if (warp == 0 && lane < 4) {
         // descriptor fetches overlap the set-up below
@@ -1028,10 +1095,10 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                         tc_fence_after();
 
                         float x[C::SBR][kHG];
-                        if (st == 0) tmem_ld8(tmem + lane_off + C::R_COL0 + (tcnt % C::NRS) * kHP + hoff, r);
+                        if (st == 0) tmem_ld_cols<kHG>(tmem + lane_off + C::R_COL0 + (tcnt % C::NRS) * kHP + hoff, r);
 #pragma unroll
                         for (int g = 0; g < C::SBR; ++g)
-                            tmem_ld8(tmem + lane_off + C::S_COL0 + slot * C::S_SLOT_COLS + g * kHP + hoff, x[g]);
+                            tmem_ld_cols<kHG>(tmem + lane_off + C::S_COL0 + slot * C::S_SLOT_COLS + g * kHP + hoff, x[g]);
                         tmem_wait_ld();
 #pragma unroll
                         for (int g = 0; g < C::SBR; ++g)
@@ -1072,11 +1139,12 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                                 break;
                             }
                             // exact column max over the tile's 128 tokens: a warp
-                            // reduce-scatter leaves column (lane >> 2) in each lane
+                            // reduce-scatter leaves column lane / (32 / kHG) in each lane
+                            constexpr int CSPAN = 32 / kHG;
 #pragma unroll
                             for (int g = 0; g < C::SBR; ++g) {
-                                const float v = warp_colmax8(x[g], lane);
-                                if ((lane & 3) == 0) misc.red_max[quad][g * kHP + hoff + (lane >> 2)] = v;
+                                const float v = warp_colmax<kHG>(x[g], lane);
+                                if ((lane & (CSPAN - 1)) == 0) misc.red_max[quad][g * kHP + hoff + lane / CSPAN] = v;
                             }
                             named_bar_sync_id<128>(gbar);
                             float alpha[C::SBR][kHG];
@@ -1117,17 +1185,18 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                                         const int gl = DC >= 128 ? p * 128 / DC : p * C::BPP + g2;
                                         const uint32_t col = ((st * C::PPS + p) * C::BPP + g2) * kHP + hoff;
                                         float o[kHG];
-                                        tmem_ld8(tmem + lane_off + col, o);
+                                        tmem_ld_cols<kHG>(tmem + lane_off + col, o);
                                         tmem_wait_ld();
 #pragma unroll
                                         for (int i = 0; i < kHG; ++i) o[i] *= alpha[gl][i];
-                                        tmem_st8(tmem + lane_off + col, o);
+                                        tmem_st_cols<kHG>(tmem + lane_off + col, o);
                                     }
                                 tmem_wait_st();
                             }
                         }
-                        // probabilities -> bf16 P (MN-major, 8x8 core matrices; this
-                        // group's 8 heads are the core matrix at + 2048 sg)
+                        // probabilities -> bf16 P (MN-major, 8x8 core matrices of 8
+                        // heads at a stride of 2048 bytes; this group's kHG heads are
+                        // the core matrices from kHG / 8 sg)
                         uint8_t* p_slot = sm + C::OFF_P + slot * C::P_BYTES;
 #pragma unroll
                         for (int g = 0; g < C::SBR; ++g) {
@@ -1141,8 +1210,12 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                                 __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
                                 packed[i / 2] = *reinterpret_cast<uint32_t*>(&pr);
                             }
-                            uint8_t* dst = p_slot + g * C::P_BRANCH_BYTES + (row >> 3) * 128 + (row & 7) * 16 + sg * 2048;
-                            *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                            uint8_t* dst = p_slot + g * C::P_BRANCH_BYTES + (row >> 3) * 128 + (row & 7) * 16 +
+                                           sg * (kHG / 8) * 2048;
+#pragma unroll
+                            for (int c8 = 0; c8 < kHG / 8; ++c8)
+                                *reinterpret_cast<uint4*>(dst + c8 * 2048) =
+                                    make_uint4(packed[4 * c8], packed[4 * c8 + 1], packed[4 * c8 + 2], packed[4 * c8 + 3]);
                         }
                         // rows past the end of the sequence (stale or poisoned data)
                         // become zero before the output MMA reads them: this group
@@ -1187,7 +1260,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                 // (this group's 32 columns of red_sum), while the range's last
                 // output MMA may still run
                 constexpr int NV = NB * kHG;  // (branch, head) values of the group
-                static_assert(NV <= 32, "a group's denominators fit its half of red_sum");
+                static_assert(2 * NV <= 4 * kHP, "the groups' denominators fit red_sum");
                 {
                     float f[NV];
 #pragma unroll
@@ -1195,15 +1268,20 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
 #pragma unroll
                         for (int i = 0; i < kHG; ++i) f[b * kHG + i] = l[b][i];
                     warp_sum_scatter<NV, 16, NV>(f, lane);
-                    constexpr int SPAN = 32 / NV;  // lanes holding one value's total
-                    if ((lane & (SPAN - 1)) == 0) misc.red_sum[quad][32 * sg + lane / SPAN] = f[0];
+                    if constexpr (NV >= 32) {  // lane L holds values (NV / 32) L + r
+#pragma unroll
+                        for (int r2 = 0; r2 < NV / 32; ++r2) misc.red_sum[quad][NV * sg + (NV / 32) * lane + r2] = f[r2];
+                    } else {
+                        constexpr int SPAN = 32 / NV;  // lanes holding one value's total
+                        if ((lane & (SPAN - 1)) == 0) misc.red_sum[quad][NV * sg + lane / SPAN] = f[0];
+                    }
                 }
                 bad = named_bar_or_id<128>(gbar, bad);  // also publishes red_sum
                 // one window holds every tile of the sequence: no split
                 const bool single = cum >= A0 && cum + (tiles - 1) * kTileCost < A1;
                 const size_t slot = (size_t)grp.slot0 + grp.ci + n;
                 if (stid < NV) {
-                    const int c = 32 * sg + stid;
+                    const int c = NV * sg + stid;
                     const float lt = misc.red_sum[0][c] + misc.red_sum[1][c] + misc.red_sum[2][c] + misc.red_sum[3][c];
                     const int b = stid / kHG, i = hoff + stid % kHG;
                     misc.inv_l[b * kHP + i] = 1.0f / lt;
@@ -1226,7 +1304,7 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                 constexpr int WIDTH = DC >= 128 ? 128 : DC;  // valid rows per block
                 float o[C::O_BLOCKS][kHG];
 #pragma unroll
-                for (int blk = 0; blk < C::O_BLOCKS; ++blk) tmem_ld8(tmem + lane_off + blk * kHP + hoff, o[blk]);
+                for (int blk = 0; blk < C::O_BLOCKS; ++blk) tmem_ld_cols<kHG>(tmem + lane_off + blk * kHP + hoff, o[blk]);
                 tmem_wait_ld();
 #pragma unroll
                 for (int blk = 0; blk < C::O_BLOCKS; ++blk) {
@@ -1245,11 +1323,14 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
                         for (int i = 0; i < kHG; ++i)
                             if (hoff + i < grp.hn) dst[(size_t)i * NB * DC] = to_bf16(o[blk][i] * a.out_scale);
                     } else {
-                        // partial layout [slot][branch][k][16 heads]: this group's
-                        // 8 heads are one 32-byte store
+                        // partial layout [slot][branch][k][kHP heads]: this group's
+                        // heads are 32-byte stores of 8
                         float* dst = a.o_part + ((slot * NB + b) * DC + k) * kHP + hoff;
-                        st_global_v8(dst, o[blk][0], o[blk][1], o[blk][2], o[blk][3], o[blk][4], o[blk][5],
-                                     o[blk][6], o[blk][7]);
+#pragma unroll
+                        for (int c8 = 0; c8 < kHG / 8; ++c8)
+                            st_global_v8(dst + 8 * c8, o[blk][8 * c8], o[blk][8 * c8 + 1], o[blk][8 * c8 + 2],
+                                         o[blk][8 * c8 + 3], o[blk][8 * c8 + 4], o[blk][8 * c8 + 5], o[blk][8 * c8 + 6],
+                                         o[blk][8 * c8 + 7]);
                     }
                 }
                 if (bad && stid == 0) record_error(a.err, MLRA_ERR_DEVICE_BAD_INDEX);
@@ -1294,14 +1375,13 @@ decode_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Deco
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
     if (*abort_flag) return;
-    // the ring's shared memory is free from here on: the merge stages its
-    // partials at its start, the fused up-projection its weight columns at
-    // its end
-    __nv_bfloat16* wt = reinterpret_cast<__nv_bfloat16*>(sm + C::OFF_PAIR + C::NSTAGE * C::PAIR_BYTES -
-                                                         UpTile<NB * DC>::W_BYTES);
+    // every region below MISC (ring, RoPE slots, queries, probabilities) is
+    // free from here on: the merge stages its partials at its start, the
+    // fused up-projection its weight columns at its end
+    __nv_bfloat16* wt = reinterpret_cast<__nv_bfloat16*>(sm + C::OFF_MISC - UpTile<NB * DC>::W_BYTES);
     const bool fused = a.w_uv != nullptr;
     if (fused && (int)blockIdx.x < a.heads * a.d_h / 16) up_stage_weights<NB, DC>(a, wt, blockIdx.x);
-    merge_tail<NB, DC>(a, grp, misc.last_seg[0], misc.last_seg[1], misc.last_seg[2], misc.last_seg[3] != 0, chunk,
+    merge_tail<NB, DC, HP>(a, grp, misc.last_seg[0], misc.last_seg[1], misc.last_seg[2], misc.last_seg[3] != 0, chunk,
                        reinterpret_cast<float*>(sm + C::OFF_PAIR), &misc.merge_flag, &misc.merge_full);
     if (fused) up_proj_tail<NB, DC>(a, sm + C::OFF_PAIR, wt, &misc.merge_flag);
 }
@@ -1345,9 +1425,10 @@ bool encode_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t mid,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NB, int DC, int DR>
+template <int NB, int DC, int DR, int HP>
 cudaError_t launch_cfg(const DecodeArgs& a, cudaStream_t stream) {
-    using C = Cfg<NB, DC, DR>;
+    using C = Cfg<NB, DC, DR, HP>;
+    constexpr int kHP = HP;
     Maps maps;
     const uint64_t rows = (uint64_t)a.num_pages * a.page_size;
     const uint32_t box_rows = (uint32_t)a.page_size;
@@ -1359,19 +1440,25 @@ cudaError_t launch_cfg(const DecodeArgs& a, cudaStream_t stream) {
         !encode_3d(&maps.qr, a.q_rope, (uint64_t)DR, (uint64_t)a.heads, (uint64_t)a.batch, DR, kHP,
                    DR == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
-    auto kernel = decode_tc_kernel<NB, DC, DR>;
+    auto kernel = decode_tc_kernel<NB, DC, DR, HP>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    // the merge stages in the ring: for all S <= grid splits of a sequence the
-    // log-sum-exp rows (S NB 16 floats) and S row slices of at most
-    // R / (S - 1) + 1 rows of 16 floats (at most 2 R + S rows in all)
-    const size_t merge_bytes = sizeof(float) * ((size_t)a.num_ctas * NB * kHP + (2 * (size_t)C::W + a.num_ctas) * kHP);
-    const size_t ring = (size_t)C::NSTAGE * C::PAIR_BYTES;
-    if (merge_bytes > ring) return cudaErrorInvalidConfiguration;
+    // the merge stages below MISC, for every S <= grid splits of a sequence:
+    // the log-sum-exp rows (S NB kHP floats) and S row slices of at most
+    // ceil(R / (S - 1)) rows of kHP floats (a member's share: at least S - 1
+    // members divide the R rows)
+    size_t merge_bytes = 0;
+    for (int S = 2; S <= a.num_ctas; ++S) {
+        const size_t rows = ((size_t)C::W + S - 2) / (S - 1);
+        const size_t bytes = sizeof(float) * ((size_t)S * NB * kHP + (size_t)S * rows * kHP);
+        merge_bytes = bytes > merge_bytes ? bytes : merge_bytes;
+    }
+    const size_t room = (size_t)C::OFF_MISC;  // all shared memory below MISC, idle after the main loop
+    if (merge_bytes > room) return cudaErrorInvalidConfiguration;
     // the fused up-projection: weight columns at the ring's end (staged while
     // the merge uses its start), then its rows and sums from the start
     if (a.w_uv != nullptr &&
-        (merge_bytes + UpTile<NB * DC>::W_BYTES > ring || (size_t)UpTile<NB * DC>::BYTES > ring))
+        (merge_bytes + UpTile<NB * DC>::W_BYTES > room || (size_t)UpTile<NB * DC>::BYTES > room))
         return cudaErrorInvalidConfiguration;
     // Cooperative: every CTA is resident at once, so the merge's wait for the
     // other splits of a sequence always ends.
@@ -1393,6 +1480,17 @@ cudaError_t launch_cfg(const DecodeArgs& a, cudaStream_t stream) {
     return cudaLaunchKernelEx(&cfg, kernel, maps, a);
 }
 
+// The head tile of a shape: 16 heads, or 32 when there are more and a
+// branch is at least 128 wide (no 32-head instantiation for narrower ones).
+template <int NB, int DC>
+cudaError_t launch_shape(const DecodeArgs& a, cudaStream_t stream) {
+    if constexpr (DC >= 128) {
+        if (tc_head_tile(a.heads, DC) == 32)
+            return a.d_r == 64 ? launch_cfg<NB, DC, 64, 32>(a, stream) : launch_cfg<NB, DC, 32, 32>(a, stream);
+    }
+    return a.d_r == 64 ? launch_cfg<NB, DC, 64, 16>(a, stream) : launch_cfg<NB, DC, 32, 16>(a, stream);
+}
+
 }  // namespace
 
 bool decode_tc_supported(int branches, int d_c, int d_r, int heads) {
@@ -1407,9 +1505,8 @@ bool decode_tc_supported(int branches, int d_c, int d_r, int heads) {
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
-#define MLRA_TC_CASE(NB_, DC_)                                                          \
-    if (a.branches == NB_ && a.d_c == DC_)                                              \
-        return a.d_r == 64 ? launch_cfg<NB_, DC_, 64>(a, stream) : launch_cfg<NB_, DC_, 32>(a, stream);
+#define MLRA_TC_CASE(NB_, DC_) \
+    if (a.branches == NB_ && a.d_c == DC_) return launch_shape<NB_, DC_>(a, stream);
     MLRA_TC_CASE(2, 64)
     MLRA_TC_CASE(4, 64)
     MLRA_TC_CASE(1, 128)

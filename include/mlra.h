@@ -118,11 +118,12 @@ MLRA_API size_t mlra_decode_workspace_bytes(const mlra_dims* dims, int32_t num_c
  *
  * Runs on the tensor cores (tcgen05, operands staged by TMA) as one
  * cooperative kernel (one CTA per SM, all resident; the CTAs that share a
- * sequence merge their partials at the end).  The MMAs take 16 heads at a
- * time: more heads run as ceil(heads / 16) groups on as many equal parts of
- * the grid, which walk the same tokens together so that the cache crosses
- * HBM about once (the repeat reads of a line hit L2).  Supported
- * shapes: heads <= 128 with batch * ceil(heads / 16) <= 65535;
+ * sequence merge their partials at the end).  The MMAs take one tile of
+ * T heads at a time, T = 16 up to 16 heads, else 32 when d_c >= 128 and 16
+ * when d_c = 64: more heads run as ceil(heads / T) groups on as many equal
+ * parts of the grid, which walk the same tokens together so that the cache
+ * crosses HBM about once (the repeat reads of a line hit L2).  Supported
+ * shapes: heads <= 128 with batch * ceil(heads / T) <= 65535;
  * (branches, d_c) in {(2,64), (4,64), (1,128), (2,128),
  * (4,128), (1,256), (2,256), (1,512)}; d_r in {32, 64}; page_size in
  * {16, 32, 64, 128}.  Other shapes return MLRA_ERR_UNSUPPORTED

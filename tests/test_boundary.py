@@ -56,10 +56,14 @@ def test_workspace_bytes_layout():
     lse_off = a256(cnt_off + 4 * 65536)     # sized for the largest batch
     o_off = a256(lse_off + 4 * slots * 4 * 16)
     assert n == a256(o_off + 4 * slots * 4 * 128 * 16)  # partial rows padded to 16 heads
-    # 40 heads: three groups of 16, rows padded to 48 heads
+    # 40 heads, d_c 128: two tiles of 32 heads, rows padded to 64 heads
     n40 = b.mlra_decode_workspace_bytes(_dims(heads=40), 148)
-    o40 = a256(lse_off + 4 * slots * 4 * 48)
-    assert n40 == a256(o40 + 4 * slots * 4 * 128 * 48)
+    o40 = a256(lse_off + 4 * slots * 4 * 64)
+    assert n40 == a256(o40 + 4 * slots * 4 * 128 * 64)
+    # 40 heads, d_c 64 (two branches per step): three tiles of 16, rows of 48
+    n40s = b.mlra_decode_workspace_bytes(_dims(heads=40, d_c=64), 148)
+    o40s = a256(lse_off + 4 * slots * 4 * 48)
+    assert n40s == a256(o40s + 4 * slots * 4 * 64 * 48)
     assert b.library().mlra_decode_workspace_bytes(ctypes.byref(_dims(batch=0)), 148) == 0
 
 
@@ -69,7 +73,7 @@ def test_workspace_bytes_layout():
     (dict(num_pages=0), b.MLRA_ERR_INVALID_ARG),
     (dict(num_pages=2 ** 30), b.MLRA_ERR_INVALID_ARG),
     (dict(heads=129), b.MLRA_ERR_UNSUPPORTED),
-    (dict(heads=128, batch=8192), b.MLRA_ERR_UNSUPPORTED),  # 8 groups x 8192 split counters
+    (dict(heads=128, batch=16384), b.MLRA_ERR_UNSUPPORTED),  # 4 tiles x 16384 split counters
     (dict(d_c=96), b.MLRA_ERR_UNSUPPORTED),
     (dict(d_c=256, branches=4), b.MLRA_ERR_UNSUPPORTED),
     (dict(d_r=48), b.MLRA_ERR_UNSUPPORTED),

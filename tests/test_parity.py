@@ -211,8 +211,10 @@ def test_repeat_calls_are_deterministic():
 
 def _split_counters(ws, dims):
     """The per-sequence split counters: int32 from byte 256 of the workspace
-    (after the error word), one per sequence and group of 16 heads."""
-    groups = (dims.heads + 15) // 16
+    (after the error word), one per sequence and head tile (16 heads, or 32
+    when there are more and d_c >= 128)."""
+    tile = 16 if dims.heads <= 16 or dims.d_c < 128 else 32
+    groups = (dims.heads + tile - 1) // tile
     return ws[256:256 + 4 * dims.batch * groups].view(torch.int32)
 
 
