@@ -113,6 +113,26 @@ def test_every_supported_shape_matches_oracle(oracle_lib, branches, d_c, d_r, pa
     _assert_close(out, ref, what=f"B={branches} d_c={d_c} d_r={d_r} P={page_size}")
 
 
+@pytest.mark.parametrize("branches,d_c", SHAPES)
+@pytest.mark.parametrize("d_r", [32, 64])
+def test_every_supported_shape_with_40_heads(oracle_lib, branches, d_c, d_r):
+    """Every (branches, d_c) at 40 heads: two tiles of 32 heads (the second
+    with 8) for d_c >= 128, three groups of 16 (the third with 8) for
+    d_c = 64; ragged lengths with splits in every group, peaked scores."""
+    import os
+    oracle_lib.set_num_threads(len(os.sched_getaffinity(0)))
+    w = Workload("shape40", batch=5, heads=40, branches=branches, d_c=d_c, d_r=d_r, page_size=64,
+                 page_order="permuted")
+    seqlens = torch.tensor([3000, 1, 640, 129, 2047], dtype=torch.int32)
+    x = make_inputs(w, seed=13, q_gain=_score_gain(w, 4.0), slack_pages=3, nan_fill_unused=True,
+                    seqlens=seqlens).to("cuda")
+    out = _run(x)
+    ref, status = _oracle(oracle_lib, x)
+    assert status == 0
+    assert torch.isfinite(out.float()).all()
+    _assert_close(out, ref, what=f"H=40 B={branches} d_c={d_c} d_r={d_r}")
+
+
 @pytest.mark.parametrize("heads", [1, 5, 16, 17, 32, 64, 128])
 @pytest.mark.parametrize("page_size", [32, 128])
 def test_head_counts_and_page_sizes(oracle_lib, heads, page_size):

@@ -57,6 +57,10 @@ def test_two_calls_in_a_row_match_mlra_decode(lib, oracle_lib):
         make_inputs(WORKLOADS["decode_2p9b"].with_(batch=6, seqlen=None), seed=21, device="cuda",
                     seqlens=torch.tensor([5000, 1, 777, 128, 4097, 2500], dtype=torch.int32)),
         make_inputs(WORKLOADS["ragged"], seed=22, device="cuda"),
+        # 40 heads on one 128-wide branch: two head tiles, two blocks of split
+        # counters cleared before the launch
+        make_inputs(WORKLOADS["tp_shard"].with_(heads=40, batch=4, seqlen=None), seed=24, device="cuda",
+                    seqlens=torch.tensor([9000, 3, 2100, 640], dtype=torch.int32)),
     ]
     status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
     for x in cases:
