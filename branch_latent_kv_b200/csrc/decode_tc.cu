@@ -59,7 +59,6 @@ constexpr int kSmemLimit = 232448;  // max dynamic shared memory per CTA on sm_1
 template <int NB, int DC, int DR, int HP_>
 struct Cfg {
     static constexpr int HP = HP_;                          // heads per tile (MMA N)
-    static constexpr int HG = HP / 2;                       // heads per softmax warpgroup
     static constexpr int W = NB * DC;                       // latent elements per token
     static constexpr int NCHUNK = W / 64;                   // 64-column (128-byte) chunks
     // A step is the unit of the MMA <-> softmax pipeline: SBR branches whose
