@@ -16,16 +16,16 @@
 //              latent rows (one 2-D box per page) into a ring of stages.
 //   warp 1     score MMA issuer (one thread) and TMEM owner:
 //                S^T_b[t, h]  = C_b[t, :] . Q_b[h, :] + K_r[t, :] . Q_r[h, :]
-//                               M = 128 tokens, N = 16 heads, K = d_c + d_r
+//                               M = 128 tokens, N = 16 (or 32) heads, K = d_c + d_r
 //   warp 6     output MMA issuer (one thread):
 //                O^T_b[k, h] += C_b[:, k]^T . P_b[:, h]
-//                               M = 128 latent columns, N = 16 heads, K = 128 tokens
+//                               M = 128 latent columns, N = 16 (or 32) heads, K = 128 tokens
 //              (the same shared-memory tile is the K-major A operand of the
 //              score MMA and the MN-major A operand of the output MMA).  An
 //              MMA issue stalls the issuing warp for about one MMA's duration,
 //              so two issuers keep the tensor pipe busy while either waits.
-//   warps 2-5  softmax and epilogue, heads 0-7, and
-//   warps 7-10 the same for heads 8-15 (two warps per scheduler, so that
+//   warps 2-5  softmax and epilogue, the first half of the tile's heads, and
+//   warps 7-10 the same for the second half (two warps per scheduler, so that
 //              each hides the other's latency): a thread owns one token of
 //              the tile (a TMEM lane); scores are base-2 logits; each (head, branch) has
 //              its own running max, rescaled only when a score exceeds it by
