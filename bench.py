@@ -62,8 +62,8 @@ FALLBACK_HBM_GBS = 6650.0
 # ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the
 # hash of the kernel sources it was taken on.  Reported as null whenever the
 # kernel sources differ from the captured ones.
-TRAFFIC_CAPTURE = {"workload": "decode_2p9b", "sources_sha1": "57bdf9ee041307b4f2fa611c377a9fec87245314",
-                   "bytes_per_launch": 151394048 + 3511552}
+TRAFFIC_CAPTURE = {"workload": "decode_2p9b", "sources_sha1": "986c9c488856f853531d268efd1ab4d111935fab",
+                   "bytes_per_launch": 151393280 + 3135232}
 KERNEL_SOURCES = ["branch_latent_kv_b200/csrc/decode_tc.cu", "branch_latent_kv_b200/csrc/sm100.cuh",
                   "branch_latent_kv_b200/csrc/common.cuh"]
 
